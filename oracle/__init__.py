@@ -1,0 +1,150 @@
+"""fp64 CPU oracle for exact attention -- test infrastructure only.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+arm of ``bench.py`` may import this package.  It never imports the CUDA
+package and shares no code with it; the two meet only through the seeded input
+generators, which hold none of the method's arithmetic.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP); this module
+compiles it with gcc on first use and marshals numpy arrays to it.  The
+definition it evaluates is standard attention (Phase 08 page, Lab 01 step 1;
+screna.ai FlashAttention answer): S = scale * Q K^T over the visible keys,
+P = softmax(S) row-wise, O = P V, L = m + ln(sum exp(s - m)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f32p = ctypes.POINTER(ctypes.c_float)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        ci, cd = ctypes.c_int, ctypes.c_double
+        lib.oracle_attn.argtypes = [f32p, f32p, f32p, f64p, f64p,
+                                    ci, ci, ci, ci, ci, ci, cd, ci, ci]
+        lib.oracle_attn.restype = ci
+        lib.oracle_attn_rows.argtypes = [f32p, f32p, f32p, f64p, f64p,
+                                         ci, ci, ci, ci, ci, ci, cd, ci,
+                                         i64p, ci, ci]
+        lib.oracle_attn_rows.restype = ci
+        lib.oracle_decode_paged.argtypes = [f32p, u16p, u16p, i32p, i32p, f64p, f64p,
+                                            ci, ci, ci, ci, ci, ci, ci, cd,
+                                            i32p, ci, ci]
+        lib.oracle_decode_paged.restype = ci
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = ci
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def attention(q, k, v, scale: float, causal: bool = False, nthreads: int | None = None):
+    """Standard attention in fp64.  q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (float32 values).
+
+    Returns (O [B,Hq,Nq,d] float64, L [B,Hq,Nq] float64).  Causal: key j is
+    visible to query i iff j <= i.
+    """
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    o = np.zeros((B, Hq, Nq, d), dtype=np.float64)
+    lse = np.zeros((B, Hq, Nq), dtype=np.float64)
+    rc = _load().oracle_attn(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                             _ptr(v, ctypes.c_float), _ptr(o, ctypes.c_double),
+                             _ptr(lse, ctypes.c_double), B, Hq, Hkv, Nq, Nk, d,
+                             float(scale), int(bool(causal)),
+                             int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn failed with code %d" % rc)
+    return o, lse
+
+
+def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | None = None):
+    """The same definition for selected rows; rows[r] = (b*Hq + h)*Nq + i."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    o = np.zeros((rows.size, d), dtype=np.float64)
+    lse = np.zeros((rows.size,), dtype=np.float64)
+    rc = _load().oracle_attn_rows(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                  _ptr(v, ctypes.c_float), _ptr(o, ctypes.c_double),
+                                  _ptr(lse, ctypes.c_double), B, Hq, Hkv, Nq, Nk, d,
+                                  float(scale), int(bool(causal)),
+                                  _ptr(rows, ctypes.c_int64), int(rows.size),
+                                  int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn_rows failed with code %d" % rc)
+    return o, lse
+
+
+def decode_paged(q, k_pages_bf16_bits, v_pages_bf16_bits, block_table, seq_lens,
+                 scale: float, seq_ids=None, nthreads: int | None = None):
+    """Single-token paged decode in fp64 for the sequences in seq_ids.
+
+    q [S,Hq,d] float32 values; k/v pages [num_pages,Hkv,page_size,d] as uint16
+    bf16 bit patterns; block_table [S,max_blocks] int32; seq_lens [S] int32.
+    Returns (O [nseq,Hq,d], L [nseq,Hq]) in float64.
+    """
+    q = _f32(q)
+    kp = np.ascontiguousarray(np.asarray(k_pages_bf16_bits, dtype=np.uint16))
+    vp = np.ascontiguousarray(np.asarray(v_pages_bf16_bits, dtype=np.uint16))
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    S, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = kp.shape
+    if d2 != d or vp.shape != kp.shape:
+        raise ValueError("page pool shape mismatch")
+    max_blocks = bt.shape[1]
+    if seq_ids is None:
+        seq_ids = np.arange(S, dtype=np.int32)
+    seq_ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32))
+    o = np.zeros((seq_ids.size, Hq, d), dtype=np.float64)
+    lse = np.zeros((seq_ids.size, Hq), dtype=np.float64)
+    rc = _load().oracle_decode_paged(_ptr(q, ctypes.c_float), _ptr(kp, ctypes.c_uint16),
+                                     _ptr(vp, ctypes.c_uint16), _ptr(bt, ctypes.c_int32),
+                                     _ptr(sl, ctypes.c_int32), _ptr(o, ctypes.c_double),
+                                     _ptr(lse, ctypes.c_double), S, Hq, Hkv, d, page_size,
+                                     max_blocks, num_pages, float(scale),
+                                     _ptr(seq_ids, ctypes.c_int32), int(seq_ids.size),
+                                     int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_decode_paged failed with code %d" % rc)
+    return o, lse

@@ -1,0 +1,254 @@
+/*
+ * attn_oracle.c -- plain, slow fp64 CPU oracle for exact attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference arm of bench.py may load this library.  It shares
+ * no code, header, table or helper with the CUDA path and never imports it.
+ *
+ * What it computes is the plain definition of standard attention, which the
+ * tiled method reaches exactly up to rounding order:
+ *
+ *   "Phase 08 -- Inference Optimization at Depth", Lab 01, Steps (1): standard
+ *   attention is the reference; screna.ai interview page, FlashAttention answer:
+ *   S = Q K^T and P = softmax(S), with O = P V.  Online-softmax answer on the
+ *   same page: softmax exponentiates every score and divides by their sum.
+ *
+ *   For each batch b and query head h, with key/value head g = h / (Hq/Hkv)
+ *   (grouped-query sharing, screna.ai MHA/MQA/GQA answer: heads are grouped and
+ *   each group shares one K and V; contiguous groups):
+ *     s_ij = scale * sum_c q[b,h,i,c] * k[b,g,j,c]      for j in V_i
+ *     V_i  = { j : j <= i } when causal (Lab 01 step 4), else { 0 .. Nk-1 }
+ *     m_i  = max_{j in V_i} s_ij
+ *     l_i  = sum_{j in V_i} exp(s_ij - m_i)
+ *     O_i  = sum_{j in V_i} exp(s_ij - m_i) / l_i * v[b,g,j,:]
+ *     L_i  = m_i + ln(l_i)        (the logsumexp "L", Concepts: backward)
+ *   An empty V_i (a decode sequence of length 0) gives O_i = 0, L_i = -inf.
+ *
+ * oracle_attn materialises S for one (b, h) at a time (N x N doubles), takes
+ * the row maximum, then exponentials and row sums, then P V -- the "standard
+ * attention" of the pages, O(N^2) memory.  oracle_attn_rows evaluates the same
+ * definition one requested row at a time, for sampled checks at full size.
+ * oracle_decode_paged gathers a sequence's keys and values from the page pool
+ * through the block table (Lab 03 step 4: pages reached through an
+ * indirection table), then evaluates the same definition for its one query.
+ *
+ * Inputs are float (the exact values the GPU sees: fp32, or bf16 upcast) or,
+ * for the page pool, raw bf16 bit patterns; arithmetic is double throughout.
+ * Return value: 0 on success, -1 on a bad argument, -2 on allocation failure.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double bf16_bits_to_double(uint16_t bits)
+{
+    /* A bf16 value is the top half of an IEEE binary32 pattern. */
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Softmax-weighted sum of the rows of v for one query, given its scores.
+ * s has n entries and is overwritten with the unnormalised weights. */
+static void softmax_row_times_v(double *s, int n, const double *v, int d,
+                                double *o_row, double *lse)
+{
+    int j, c;
+    double m, l;
+    for (c = 0; c < d; ++c) o_row[c] = 0.0;
+    if (n == 0) { *lse = -INFINITY; return; }
+    m = s[0];
+    for (j = 1; j < n; ++j) if (s[j] > m) m = s[j];
+    l = 0.0;
+    for (j = 0; j < n; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+    for (j = 0; j < n; ++j) {
+        double p = s[j] / l;
+        const double *vj = v + (size_t)j * d;
+        for (c = 0; c < d; ++c) o_row[c] += p * vj[c];
+    }
+    *lse = m + log(l);
+}
+
+static int check_dims(int B, int Hq, int Hkv, int Nq, int Nk, int d)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    return 0;
+}
+
+/* Full evaluation: q [B,Hq,Nq,d], k,v [B,Hkv,Nk,d] (float), o [B,Hq,Nq,d],
+ * lse [B,Hq,Nq] (double).  Causal means key j is visible to query i iff j <= i. */
+int oracle_attn(const float *q, const float *k, const float *v,
+                double *o, double *lse,
+                int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                double scale, int causal, int nthreads)
+{
+    int b, h, G;
+    double *S, *Kd, *Vd, *Qd;
+    if (check_dims(B, Hq, Hkv, Nq, Nk, d)) return -1;
+    if (!q || !k || !v || !o || !lse) return -1;
+    G = Hq / Hkv;
+    if (nthreads <= 0) nthreads = 1;
+    S = (double *)malloc(sizeof(double) * ((size_t)Nq * Nk + 1));
+    Kd = (double *)malloc(sizeof(double) * ((size_t)Nk * d + 1));
+    Vd = (double *)malloc(sizeof(double) * ((size_t)Nk * d + 1));
+    Qd = (double *)malloc(sizeof(double) * ((size_t)Nq * d + 1));
+    if (!S || !Kd || !Vd || !Qd) { free(S); free(Kd); free(Vd); free(Qd); return -2; }
+
+    for (b = 0; b < B; ++b) {
+        for (h = 0; h < Hq; ++h) {
+            int g = h / G;
+            const float *qh = q + ((size_t)b * Hq + h) * (size_t)Nq * d;
+            const float *kh = k + ((size_t)b * Hkv + g) * (size_t)Nk * d;
+            const float *vh = v + ((size_t)b * Hkv + g) * (size_t)Nk * d;
+            double *oh = o + ((size_t)b * Hq + h) * (size_t)Nq * d;
+            double *lh = lse + ((size_t)b * Hq + h) * (size_t)Nq;
+            long i;
+            for (i = 0; i < (long)Nq * d; ++i) Qd[i] = (double)qh[i];
+            for (i = 0; i < (long)Nk * d; ++i) { Kd[i] = (double)kh[i]; Vd[i] = (double)vh[i]; }
+
+            /* S = scale * Q K^T, the whole Nq x Nk matrix of this head. */
+            #pragma omp parallel for num_threads(nthreads) schedule(static)
+            for (i = 0; i < Nq; ++i) {
+                int j, c;
+                for (j = 0; j < Nk; ++j) {
+                    double acc = 0.0;
+                    for (c = 0; c < d; ++c) acc += Qd[(size_t)i * d + c] * Kd[(size_t)j * d + c];
+                    S[(size_t)i * Nk + j] = scale * acc;
+                }
+            }
+            /* Row-wise softmax over the visible keys, then P V and L. */
+            #pragma omp parallel for num_threads(nthreads) schedule(static)
+            for (i = 0; i < Nq; ++i) {
+                int n = Nk;
+                if (causal) n = (i + 1 < Nk) ? (int)(i + 1) : Nk;
+                softmax_row_times_v(S + (size_t)i * Nk, n, Vd, d,
+                                    oh + (size_t)i * d, lh + i);
+            }
+        }
+    }
+    free(S); free(Kd); free(Vd); free(Qd);
+    return 0;
+}
+
+/* Selected rows only.  rows[r] = (b*Hq + h)*Nq + i.  o_rows [nrows,d],
+ * lse_rows [nrows].  Same definition, one row at a time. */
+int oracle_attn_rows(const float *q, const float *k, const float *v,
+                     double *o_rows, double *lse_rows,
+                     int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     double scale, int causal,
+                     const int64_t *rows, int nrows, int nthreads)
+{
+    int G, r, bad = 0;
+    if (check_dims(B, Hq, Hkv, Nq, Nk, d)) return -1;
+    if (!q || !k || !v || !o_rows || !lse_rows || (!rows && nrows > 0) || nrows < 0) return -1;
+    for (r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq * Nq) return -1;
+    G = Hq / Hkv;
+    if (nthreads <= 0) nthreads = 1;
+
+    #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) reduction(|:bad)
+    for (r = 0; r < nrows; ++r) {
+        int64_t id = rows[r];
+        int i = (int)(id % Nq);
+        int bh = (int)(id / Nq);
+        int h = bh % Hq, b = bh / Hq, g = h / G;
+        int n = causal ? ((i + 1 < Nk) ? i + 1 : Nk) : Nk;
+        const float *qi = q + (((size_t)b * Hq + h) * Nq + i) * (size_t)d;
+        const float *kh = k + ((size_t)b * Hkv + g) * (size_t)Nk * d;
+        const float *vh = v + ((size_t)b * Hkv + g) * (size_t)Nk * d;
+        double *s = (double *)malloc(sizeof(double) * ((size_t)n + 1));
+        double *vd = (double *)malloc(sizeof(double) * ((size_t)n * d + 1));
+        int j, c;
+        if (!s || !vd) { free(s); free(vd); bad = 1; continue; }
+        for (j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (c = 0; c < d; ++c) acc += (double)qi[c] * (double)kh[(size_t)j * d + c];
+            s[j] = scale * acc;
+            for (c = 0; c < d; ++c) vd[(size_t)j * d + c] = (double)vh[(size_t)j * d + c];
+        }
+        softmax_row_times_v(s, n, vd, d, o_rows + (size_t)r * d, lse_rows + r);
+        free(s); free(vd);
+    }
+    return bad ? -2 : 0;
+}
+
+/* Single-token decode over a paged KV cache, for the sequences listed in
+ * seq_ids.  q [S,Hq,d] float; k_pages, v_pages [num_pages,Hkv,page_size,d] as
+ * bf16 bit patterns; block_table [S,max_blocks]; seq_lens [S].
+ * Token t of sequence s lives in page block_table[s, t / page_size], slot
+ * t % page_size.  o [nseq,Hq,d], lse [nseq,Hq].  Returns -1 if a page id the
+ * sequence needs is outside [0, num_pages) or a length is out of range. */
+int oracle_decode_paged(const float *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                        const int32_t *block_table, const int32_t *seq_lens,
+                        double *o, double *lse,
+                        int S, int Hq, int Hkv, int d, int page_size, int max_blocks,
+                        int num_pages, double scale,
+                        const int32_t *seq_ids, int nseq, int nthreads)
+{
+    int G, r, bad = 0;
+    if (S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || page_size <= 0 || max_blocks <= 0 ||
+        num_pages <= 0 || Hq % Hkv != 0 || nseq < 0) return -1;
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse ||
+        (!seq_ids && nseq > 0)) return -1;
+    G = Hq / Hkv;
+    for (r = 0; r < nseq; ++r) {
+        int s = seq_ids[r], t, len;
+        if (s < 0 || s >= S) return -1;
+        len = seq_lens[s];
+        if (len < 0 || len > max_blocks * page_size) return -1;
+        for (t = 0; t < len; t += page_size) {
+            int32_t p = block_table[(size_t)s * max_blocks + t / page_size];
+            if (p < 0 || p >= num_pages) return -1;
+        }
+    }
+    if (nthreads <= 0) nthreads = 1;
+
+    #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) reduction(|:bad)
+    for (r = 0; r < nseq * Hkv; ++r) {
+        int s = seq_ids[r / Hkv], g = r % Hkv;
+        int len = seq_lens[s];
+        int t, c, hh;
+        double *kd = (double *)malloc(sizeof(double) * ((size_t)len * d + 1));
+        double *vd = (double *)malloc(sizeof(double) * ((size_t)len * d + 1));
+        double *sc = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+        if (!kd || !vd || !sc) { free(kd); free(vd); free(sc); bad = 1; continue; }
+        /* Gather: follow the block table to contiguous [len, d] keys/values. */
+        for (t = 0; t < len; ++t) {
+            int32_t p = block_table[(size_t)s * max_blocks + t / page_size];
+            size_t base = (((size_t)p * Hkv + g) * page_size + (t % page_size)) * (size_t)d;
+            for (c = 0; c < d; ++c) {
+                kd[(size_t)t * d + c] = bf16_bits_to_double(k_pages[base + c]);
+                vd[(size_t)t * d + c] = bf16_bits_to_double(v_pages[base + c]);
+            }
+        }
+        for (hh = 0; hh < G; ++hh) {
+            int h = g * G + hh;
+            const float *qs = q + ((size_t)s * Hq + h) * (size_t)d;
+            for (t = 0; t < len; ++t) {
+                double acc = 0.0;
+                for (c = 0; c < d; ++c) acc += (double)qs[c] * kd[(size_t)t * d + c];
+                sc[t] = scale * acc;
+            }
+            softmax_row_times_v(sc, len, vd, d,
+                                o + ((size_t)(r / Hkv) * Hq + h) * (size_t)d,
+                                lse + (size_t)(r / Hkv) * Hq + h);
+        }
+        free(kd); free(vd); free(sc);
+    }
+    return bad ? -2 : 0;
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,398 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+The oracle is trusted only because these checks tie it to what the pages and
+the mathematics fix, independently of the oracle's own code:
+
+* closed forms: one key (O = v0), identical keys (O = mean of V, L = s + ln N),
+  constant values (weights sum to one), causal row 0, two keys (logistic weights);
+* hand-derived worked examples under tests/golden/ (powers of two);
+* a brute force in 50-digit decimal arithmetic, written without the max-shift
+  that the oracle uses, on tiny inputs;
+* the online recurrence of the Phase 08 page (Lab 01 talking points) for tile
+  sizes 1, 7 and N;
+* structural invariants: GQA equals MHA with repeated K/V heads, key/value
+  permutation invariance, shift invariance under large offsets, causal rows
+  equal non-causal attention over the prefix, paged equals contiguous;
+* mutation checks: plausible one-token mistakes planted in a copy of the
+  oracle's C source are each caught by at least one pin.
+"""
+from __future__ import annotations
+
+import decimal
+import json
+import math
+import os
+import subprocess
+import sys
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+from oracle.online import online_attention  # noqa: E402
+
+RNG = np.random.default_rng(12345)
+
+
+def rand(*shape, rng=RNG):
+    return rng.standard_normal(shape).astype(np.float32)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_single_key_returns_its_value():
+    q, k, v = rand(2, 3, 1, 8), rand(2, 3, 1, 8), rand(2, 3, 1, 8)
+    o, lse = oracle.attention(q, k, v, scale=0.37)
+    np.testing.assert_allclose(o, v.astype(np.float64), rtol=0, atol=1e-15)
+    s = 0.37 * np.einsum("bhnd,bhnd->bhn", q.astype(np.float64), k.astype(np.float64))
+    np.testing.assert_allclose(lse, s, rtol=0, atol=1e-13)
+
+
+def test_identical_keys_average_the_values():
+    N, d = 11, 16
+    q, v = rand(1, 2, N, d), rand(1, 2, N, d)
+    krow = rand(1, 2, 1, d)
+    k = np.repeat(krow, N, axis=2)
+    o, lse = oracle.attention(q, k, v, scale=0.25)
+    mean_v = v.astype(np.float64).mean(axis=2, keepdims=True)
+    np.testing.assert_allclose(o, np.broadcast_to(mean_v, o.shape), rtol=0, atol=1e-13)
+    s = 0.25 * np.einsum("bhnd,bhd->bhn", q.astype(np.float64), krow[:, :, 0].astype(np.float64))
+    np.testing.assert_allclose(lse, s + math.log(N), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_weights_sum_to_one(causal):
+    # With every value row equal to c, O = (sum_j p_ij) c, so O == c iff the
+    # softmax weights of each row sum to one.
+    N, d = 37, 8
+    q, k = rand(1, 1, N, d) * 3, rand(1, 1, N, d) * 3
+    c = rand(d)
+    v = np.broadcast_to(c, (1, 1, N, d)).copy()
+    o, _ = oracle.attention(q, k, v, scale=0.5, causal=causal)
+    np.testing.assert_allclose(o, np.broadcast_to(c.astype(np.float64), o.shape), rtol=0, atol=1e-12)
+
+
+def test_weights_are_nonnegative_and_normalised():
+    # v_j = e_j (one-hot) exposes each row of P in O directly.
+    N = 9
+    q, k = rand(1, 1, N, N), rand(1, 1, N, N)  # d = N so v can be one-hot
+    v = np.eye(N, dtype=np.float32)[None, None]
+    for causal in (False, True):
+        P, _ = oracle.attention(q, k, v, scale=1.0, causal=causal)
+        P = P[0, 0]
+        assert (P >= 0).all()
+        np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+        if causal:
+            assert np.all(np.triu(P, 1) == 0.0)
+
+
+def test_causal_row_zero_sees_only_key_zero():
+    q, k, v = rand(1, 2, 6, 4), rand(1, 2, 6, 4), rand(1, 2, 6, 4)
+    o, lse = oracle.attention(q, k, v, scale=0.7, causal=True)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0].astype(np.float64), rtol=0, atol=1e-15)
+    s00 = 0.7 * np.einsum("bhd,bhd->bh", q[:, :, 0].astype(np.float64), k[:, :, 0].astype(np.float64))
+    np.testing.assert_allclose(lse[:, :, 0], s00, rtol=0, atol=1e-14)
+
+
+def test_two_keys_logistic_weights():
+    d = 6
+    q, k, v = rand(1, 1, 1, d), rand(1, 1, 2, d), rand(1, 1, 2, d)
+    o, lse = oracle.attention(q, k, v, scale=0.9)
+    qd, kd, vd = q[0, 0, 0].astype(float), k[0, 0].astype(float), v[0, 0].astype(float)
+    s0, s1 = 0.9 * float(qd @ kd[0]), 0.9 * float(qd @ kd[1])
+    w0 = 1.0 / (1.0 + math.exp(s1 - s0))
+    np.testing.assert_allclose(o[0, 0, 0], w0 * vd[0] + (1 - w0) * vd[1], rtol=0, atol=1e-14)
+    hi, lo = max(s0, s1), min(s0, s1)
+    np.testing.assert_allclose(lse[0, 0, 0], hi + math.log1p(math.exp(lo - hi)), rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------ golden examples
+
+def _val(x):
+    if isinstance(x, str):
+        if x == "ln2":
+            return math.log(2.0)
+        if x.startswith("ln"):
+            return math.log(float(x[2:]))
+        return float(Fraction(x))
+    if isinstance(x, list):
+        return [_val(y) for y in x]
+    return float(x)
+
+
+def _golden():
+    with open(os.path.join(ROOT, "tests", "golden", "hand_examples.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden()["prefill"], ids=lambda c: c["name"])
+def test_golden_prefill(case):
+    q, k, v = (np.array(_val(case[n]), dtype=np.float32) for n in ("q", "k", "v"))
+    o, lse = oracle.attention(q, k, v, scale=_val(case["scale"]), causal=case["causal"])
+    np.testing.assert_allclose(o, np.array(_val(case["o"])), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(_val(case["lse"])), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("case", _golden()["decode"], ids=lambda c: c["name"])
+def test_golden_decode(case):
+    import torch
+    to_bits = lambda a: torch.tensor(a, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    kp, vp = to_bits(_val(case["k_pages"])), to_bits(_val(case["v_pages"]))
+    o, lse = oracle.decode_paged(np.array(case["q"], dtype=np.float32), kp, vp,
+                                 np.array(case["block_table"], dtype=np.int32),
+                                 np.array(case["seq_lens"], dtype=np.int32),
+                                 scale=_val(case["scale"]))
+    np.testing.assert_allclose(o, np.array(_val(case["o"])), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(_val(case["lse"])), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------ decimal brute force
+
+def _brute_decimal(q, k, v, scale, causal, G):
+    """Per-element evaluation in 50-digit decimals: p_ij = e^{s_ij} / sum_j e^{s_ij}."""
+    ctx = decimal.Context(prec=50)
+    D = lambda x: ctx.create_decimal_from_float(float(x))
+    B, Hq, N, d = q.shape
+    o = np.zeros(q.shape)
+    lse = np.zeros(q.shape[:3])
+    sc = D(scale)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for i in range(N):
+                js = range(i + 1) if causal else range(k.shape[2])
+                e = {}
+                for j in js:
+                    s = ctx.multiply(sc, sum((ctx.multiply(D(q[b, h, i, c]), D(k[b, g, j, c])) for c in range(d)), decimal.Decimal(0)))
+                    e[j] = ctx.exp(s)
+                tot = sum(e.values(), decimal.Decimal(0))
+                for c in range(d):
+                    acc = sum((ctx.multiply(ctx.divide(e[j], tot), D(v[b, g, j, c])) for j in js), decimal.Decimal(0))
+                    o[b, h, i, c] = float(acc)
+                lse[b, h, i] = float(ctx.ln(tot))
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d,Hq,Hkv", [(1, 1, 1, 1), (3, 2, 2, 1), (5, 4, 2, 2), (8, 3, 4, 2)])
+def test_decimal_brute_force(N, d, Hq, Hkv, causal):
+    rng = np.random.default_rng(N * 100 + d * 10 + Hq + causal)
+    q, k, v = (rng.standard_normal(s).astype(np.float32) * 2 for s in
+               ((2, Hq, N, d), (2, Hkv, N, d), (2, Hkv, N, d)))
+    o, lse = oracle.attention(q, k, v, scale=0.6, causal=causal)
+    ob, lb = _brute_decimal(q, k, v, 0.6, causal, Hq // Hkv)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lb, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- online recurrence
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("block", [1, 7, 64])
+def test_online_recurrence_equals_two_pass(block, causal):
+    N, d = 64, 16
+    q, k, v = rand(1, 1, N, d) * 2, rand(1, 1, N, d) * 2, rand(1, 1, N, d)
+    o, lse = oracle.attention(q, k, v, scale=0.25, causal=causal)
+    oo, lo = online_attention(q[0, 0], k[0, 0], v[0, 0], 0.25, block, causal=causal)
+    np.testing.assert_allclose(oo, o[0, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lo, lse[0, 0], rtol=0, atol=1e-12)
+
+
+# -------------------------------------------------------------- invariants
+
+def test_gqa_equals_mha_with_repeated_heads():
+    B, Hq, Hkv, N, d = 2, 8, 2, 19, 8
+    q, k, v = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d)
+    for causal in (False, True):
+        o1, l1 = oracle.attention(q, k, v, scale=0.3, causal=causal)
+        G = Hq // Hkv
+        o2, l2 = oracle.attention(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1),
+                                  scale=0.3, causal=causal)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+    # head h uses kv head h // G (contiguous groups): head 1 must differ from
+    # what kv head 1 would give.
+    o_alt, _ = oracle.attention(q[:, 1:2], k[:, 1:2], v[:, 1:2], scale=0.3)
+    o_ref, _ = oracle.attention(q[:, 1:2], k[:, 0:1], v[:, 0:1], scale=0.3)
+    o_all, _ = oracle.attention(q, k, v, scale=0.3)
+    np.testing.assert_array_equal(o_all[:, 1:2], o_ref)
+    assert np.abs(o_all[:, 1:2] - o_alt).max() > 1e-3
+
+
+def test_key_permutation_invariance():
+    N, d = 23, 8
+    q, k, v = rand(1, 2, N, d), rand(1, 2, N, d), rand(1, 2, N, d)
+    perm = RNG.permutation(N)
+    o1, l1 = oracle.attention(q, k, v, scale=0.4)
+    o2, l2 = oracle.attention(q, k[:, :, perm], v[:, :, perm], scale=0.4)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+
+
+def test_shift_invariance_large_offsets():
+    # Adding u to every key adds scale*q.u to a row's scores: O is unchanged
+    # and L moves by scale*q.u.  Offsets of ~1e3 overflow exp() unless the
+    # maximum is subtracted first.
+    N, d = 17, 4
+    q, k, v = rand(1, 1, N, d), rand(1, 1, N, d), rand(1, 1, N, d)
+    q = q * 40.0
+    k = np.round(k * 64) / 64  # k + u stays exact in float32
+    u = np.full(d, 25.0, dtype=np.float32)
+    o1, l1 = oracle.attention(q, k, v, scale=0.5)
+    o2, l2 = oracle.attention(q, k + u, v, scale=0.5)
+    shift = 0.5 * (q[0, 0].astype(np.float64) @ u.astype(np.float64))
+    assert np.isfinite(o2).all() and np.abs(shift).max() > 700
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(l2[0, 0], l1[0, 0] + shift, rtol=1e-14, atol=1e-9)
+
+
+def test_causal_rows_equal_prefix_attention():
+    N, d = 12, 4
+    q, k, v = rand(1, 1, N, d), rand(1, 1, N, d), rand(1, 1, N, d)
+    o, lse = oracle.attention(q, k, v, scale=0.8, causal=True)
+    for i in range(N):
+        oi, li = oracle.attention(q[:, :, i:i + 1], k[:, :, :i + 1], v[:, :, :i + 1], scale=0.8)
+        np.testing.assert_array_equal(o[0, 0, i], oi[0, 0, 0])
+        np.testing.assert_array_equal(lse[0, 0, i], li[0, 0, 0])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_evaluator_matches_full(causal):
+    B, Hq, Hkv, N, d = 2, 4, 2, 33, 16
+    q, k, v = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d)
+    o, lse = oracle.attention(q, k, v, scale=0.25, causal=causal)
+    rows = RNG.choice(B * Hq * N, size=40, replace=False)
+    orow, lrow = oracle.attention_rows(q, k, v, 0.25, causal, rows)
+    np.testing.assert_allclose(orow, o.reshape(-1, d)[rows], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lrow, lse.reshape(-1)[rows], rtol=0, atol=1e-14)
+
+
+def _bf16_bits(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _bits_to_f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def test_paged_decode_equals_contiguous_and_is_placement_free():
+    # Paging is memory management only: the same tokens scattered over two
+    # different page placements give identical results, equal to attention
+    # over the contiguous cache.
+    S, Hq, Hkv, d, ps, P = 5, 8, 2, 16, 4, 40
+    lens = np.array([1, 4, 5, 13, 0], dtype=np.int32)
+    maxb = 4
+    kc = [_bf16_bits(rand(Hkv, int(n), d)) for n in lens]
+    vc = [_bf16_bits(rand(Hkv, int(n), d)) for n in lens]
+    q = _bits_to_f32(_bf16_bits(rand(S, Hq, d)))
+    results = []
+    for seed in (1, 2):
+        rng = np.random.default_rng(seed)
+        perm = rng.permutation(P).astype(np.int32)
+        kp = _bf16_bits(rand(P, Hkv, ps, d, rng=rng))  # unrelated filler everywhere
+        vp = _bf16_bits(rand(P, Hkv, ps, d, rng=rng))
+        bt = np.full((S, maxb), -1, dtype=np.int32)
+        nxt = 0
+        for s in range(S):
+            n = -(-int(lens[s]) // ps)
+            bt[s, :n] = perm[nxt:nxt + n]
+            nxt += n
+            for t in range(int(lens[s])):
+                kp[bt[s, t // ps], :, t % ps] = kc[s][:, t]
+                vp[bt[s, t // ps], :, t % ps] = vc[s][:, t]
+        o, lse = oracle.decode_paged(q, kp, vp, bt, lens, scale=0.25)
+        results.append((o, lse))
+        for s in range(S):
+            if lens[s] == 0:
+                assert np.all(o[s] == 0) and np.all(np.isneginf(lse[s]))
+                continue
+            oc, lc = oracle.attention(q[s][None, :, None, :], _bits_to_f32(kc[s])[None],
+                                      _bits_to_f32(vc[s])[None], scale=0.25)
+            np.testing.assert_array_equal(o[s], oc[0, :, 0])
+            np.testing.assert_array_equal(lse[s], lc[0, :, 0])
+    np.testing.assert_array_equal(results[0][0], results[1][0])
+    np.testing.assert_array_equal(results[0][1], results[1][1])
+
+
+def test_decode_equals_causal_prefill_row():
+    # Autoregressive check (Lab 01 "How to Test"): decoding token t against the
+    # cache of tokens 0..t gives row t of the causal prefill.
+    N, H, d, ps = 10, 2, 8, 4
+    q = _bits_to_f32(_bf16_bits(rand(1, H, N, d)))
+    kb, vb = _bf16_bits(rand(1, H, N, d)), _bf16_bits(rand(1, H, N, d))
+    o, lse = oracle.attention(q, _bits_to_f32(kb), _bits_to_f32(vb), scale=0.35, causal=True)
+    npages = -(-N // ps)
+    kp = np.zeros((npages, H, ps, d), dtype=np.uint16)
+    vp = np.zeros_like(kp)
+    for t in range(N):
+        kp[t // ps, :, t % ps] = kb[0, :, t]
+        vp[t // ps, :, t % ps] = vb[0, :, t]
+    bt = np.arange(npages, dtype=np.int32)[None]
+    for t in range(N):
+        od, ld = oracle.decode_paged(q[0, :, t][None], kp, vp, bt, np.array([t + 1], np.int32), scale=0.35)
+        np.testing.assert_allclose(od[0], o[0, :, t], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(ld[0], lse[0, :, t], rtol=0, atol=1e-13)
+
+
+def test_decode_rejects_bad_page_ids():
+    kp = np.zeros((2, 1, 2, 1), dtype=np.uint16)
+    with pytest.raises(ValueError):
+        oracle.decode_paged(np.ones((1, 1, 1), np.float32), kp, kp,
+                            np.array([[0, 5]], np.int32), np.array([3], np.int32), scale=1.0)
+
+
+# ------------------------------------------------------------- mutations
+
+MUTANTS = {
+    "no_max_shift_sign": ("s[j] = exp(s[j] - m)", "s[j] = exp(m - s[j])"),
+    "drop_normalisation": ("double p = s[j] / l;", "double p = s[j];"),
+    "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "causal_off_by_one": ("if (causal) n = (i + 1 < Nk) ? (int)(i + 1) : Nk;",
+                          "if (causal) n = (i < Nk) ? (int)(i) + (i == 0) : Nk;"),
+    "wrong_gqa_group": ("int g = h / G;\n            const float *qh", "int g = h % Hkv;\n            const float *qh"),
+    "dropped_term": ("for (c = 0; c < d; ++c) acc += Qd", "for (c = 1; c < d; ++c) acc += Qd"),
+    "log_base_two": ("*lse = m + log(l);", "*lse = m + log2(l);"),
+    "scale_dropped": ("S[(size_t)i * Nk + j] = scale * acc;", "S[(size_t)i * Nk + j] = acc;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name, tmp_path):
+    """Each mutant of the oracle's C source fails at least one closed-form pin."""
+    src = open(os.path.join(ROOT, "oracle", "attn_oracle.c")).read()
+    old, new = MUTANTS[name]
+    assert old in src, name
+    mutated = src.replace(old, new, 1)
+    cpath = tmp_path / "mut.c"
+    cpath.write_text(mutated)
+    lib = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(lib), str(cpath), "-lm"])
+    import ctypes
+    saved = oracle._lib
+    try:
+        oracle._lib = None
+        real_build = oracle.build
+        oracle.build = lambda force=False: str(lib)
+        failures = 0
+        checks = [test_single_key_returns_its_value, test_identical_keys_average_the_values,
+                  lambda: test_weights_sum_to_one(True), test_causal_row_zero_sees_only_key_zero,
+                  test_two_keys_logistic_weights, test_gqa_equals_mha_with_repeated_heads,
+                  lambda: test_decimal_brute_force(5, 4, 2, 2, True),
+                  lambda: test_decimal_brute_force(8, 3, 4, 2, False),
+                  test_causal_rows_equal_prefix_attention]
+        for golden in _golden()["prefill"]:
+            checks.append(lambda g=golden: test_golden_prefill(g))
+        for chk in checks:
+            try:
+                chk()
+            except (AssertionError, ValueError, FloatingPointError):
+                failures += 1
+        assert failures > 0, "mutant %s survived every pin" % name
+    finally:
+        oracle.build = real_build
+        oracle._lib = saved
