@@ -1,0 +1,446 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one forward pass of bf16 non-causal multi-head attention over the
+seq_len sweep of the Phase 08 page's Lab 01 benchmark (B=2, H=16, d=128,
+N = 512, 1024, 2048, 4096, 8192), on synthetic N(0,1) inputs resident in HBM.
+L2 is flushed (a 256 MiB write) before every launch and the flush is outside the
+per-launch CUDA-event pairs that give the kernel time.
+
+The JSON line also carries, measured in the same run:
+  * ``components``: causal N=8192 (H=32), GQA causal N=4096 (B=4, Hq=32,
+    Hkv=8) prefill TFLOP/s, and the paged GQA decode (64 sequences, context
+    U[512, 8192], 16-token pages) in HBM GB/s, each as a fraction of the
+    measured peak;
+  * ``roofline`` for the prefill kernel (tensor-bound);
+  * ``e2e``: the same sweep through the public API with pinned host buffers,
+    host->device and device->host copies inside the timed region;
+  * ``cpu_baseline``: the fp64 CPU oracle timed on a bounded sample.
+
+``--impl reference`` times the CPU oracle on the same workload instead (a few
+heads per step, all host cores), as the reference arm.
+Multi-GPU (torchrun): every rank runs the whole workload on its own GPU (the
+path needs no collective); value = work of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_101_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, causal/non) & decode HBM GB/s, % of roofline"
+WORKLOAD = "bf16 MHA non-causal prefill sweep B=2 H=16 d=128 N=512..8192"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(name: str) -> str:
+    with open(os.path.join(ROOT, "exact_io_aware_101_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(summary: str, kernel_src: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", summary)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_src = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_src or not m_b or m_src.group(1) != source_digest(kernel_src):
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over all ranks (CUDA-event times are per rank)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(work_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return work_per_rank * world / max_seconds
+
+
+# ------------------------------------------------------------ GPU workloads
+class Prefill:
+    def __init__(self, cfg, lib):
+        self.cfg = cfg
+        self.lib = lib
+        self.q, self.k, self.v = syn.prefill_inputs(cfg, device="cuda")
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(cfg.B, cfg.Hq, cfg.N, dtype=torch.float32, device="cuda")
+
+    def launch(self):
+        c = self.cfg
+        rc = self.lib.attn_fwd(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                               self.o.data_ptr(), self.lse.data_ptr(), c.B, c.Hq, c.Hkv, c.N, c.d,
+                               c.scale, int(c.causal), torch.cuda.current_stream().cuda_stream)
+        if rc != 0:
+            raise RuntimeError("attn_fwd failed: %d" % rc)
+        return 1  # kernels launched
+
+
+class Decode:
+    def __init__(self, cfg, lib):
+        import exact_io_aware_101_b200 as ea
+        self.cfg = cfg
+        self.lib = lib
+        self.inp = syn.decode_inputs(cfg, device="cuda")
+        self.o = torch.empty_like(self.inp["q"])
+        self.lse = torch.empty(cfg.S, cfg.Hq, dtype=torch.float32, device="cuda")
+        self.ws_bytes = ea.decode_workspace_bytes(cfg.S, cfg.Hq, cfg.d, cfg.max_blocks)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.bytes = syn.decode_bytes(self.inp["seq_lens"].cpu().tolist(), cfg.Hkv, cfg.d, cfg.Hq,
+                                      cfg.page_size)
+
+    def launch(self):
+        c, i = self.cfg, self.inp
+        rc = self.lib.attn_decode_paged(
+            i["q"].data_ptr(), i["k_pages"].data_ptr(), i["v_pages"].data_ptr(),
+            i["block_table"].data_ptr(), i["seq_lens"].data_ptr(), self.o.data_ptr(),
+            self.lse.data_ptr(), c.S, c.Hq, c.Hkv, c.d, c.page_size, c.max_blocks, c.num_pages,
+            c.scale, self.ws.data_ptr(), self.ws_bytes, torch.cuda.current_stream().cuda_stream)
+        if rc != 0:
+            raise RuntimeError("attn_decode_paged failed: %d" % rc)
+        return 2  # split + combine
+
+
+def timed_launches(items, flush, reps):
+    """Per-item list of CUDA-event durations (ms), L2 flushed before each launch."""
+    times = [[] for _ in items]
+    launches = 0
+    for _ in range(reps):
+        for idx, it in enumerate(items):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            launches += it.launch()
+            e1.record()
+            times[idx].append((e0, e1))
+    torch.cuda.synchronize()
+    return [[a.elapsed_time(b) for a, b in row] for row in times], launches
+
+
+def e2e_sweep(items, reps):
+    """The sweep through the public API with pinned host buffers (H2D + call + D2H)."""
+    import exact_io_aware_101_b200 as ea
+    host = []
+    for it in items:
+        host.append(dict(q=it.q.cpu().pin_memory(), k=it.k.cpu().pin_memory(),
+                         v=it.v.cpu().pin_memory(), o=torch.empty(it.o.shape, dtype=it.o.dtype).pin_memory(),
+                         l=torch.empty(it.lse.shape, dtype=torch.float32).pin_memory()))
+    h2d = sum(h["q"].nbytes + h["k"].nbytes + h["v"].nbytes for h in host)
+    d2h = sum(h["o"].nbytes + h["l"].nbytes for h in host)
+
+    def once():
+        for it, h in zip(items, host):
+            q = h["q"].to("cuda", non_blocking=True)
+            k = h["k"].to("cuda", non_blocking=True)
+            v = h["v"].to("cuda", non_blocking=True)
+            o, l = ea.attn_fwd(q, k, v, causal=it.cfg.causal, scale=it.cfg.scale)
+            h["o"].copy_(o, non_blocking=True)
+            h["l"].copy_(l, non_blocking=True)
+
+    once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps, h2d, d2h
+
+
+def cpu_oracle_sample(target_s=12.0, cap_heads=64):
+    """Time the fp64 oracle on whole heads of the N=4096 MHA workload."""
+    import oracle
+    cfg = syn.MHA_SWEEP[3]
+    q, k, v = syn.prefill_inputs(cfg)
+    qf, kf, vf = q.float().numpy(), k.float().numpy(), v.float().numpy()
+    threads = oracle.max_threads()
+    heads, elapsed = 1, 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.attention(qf[:1, :heads], kf[:1, :heads], vf[:1, :heads], scale=cfg.scale)
+        elapsed = time.perf_counter() - t0
+        if elapsed >= target_s / 4 or heads >= cap_heads:
+            break
+        heads = min(cap_heads, heads * max(2, int(target_s / 4 / max(elapsed, 1e-3))))
+    flops = 4.0 * heads * cfg.N * cfg.N * cfg.d
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": "fp64 oracle (materialised S, two-pass softmax) on %d head(s) of the "
+                      "N=4096 MHA workload: %.1f GFLOP in %.2f s" % (heads, flops / 1e9, elapsed)}
+
+
+# --------------------------------------------------------------- arms
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    threads = oracle.max_threads()
+    data = []
+    for cfg in syn.MHA_SWEEP:
+        q, k, v = syn.prefill_inputs(cfg)
+        data.append((cfg, q[:1, :1].float().numpy(), k[:1, :1].float().numpy(),
+                     v[:1, :1].float().numpy()))
+
+    def step():
+        for cfg, q, k, v in data:
+            oracle.attention(q, k, v, scale=cfg.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = sum(4.0 * c.N * c.N * c.d for c, *_ in data)
+    value = flops / dt / 1e12
+    sample = ("fp64 CPU oracle, one (batch, head) of each N in the sweep per step "
+              "(%.1f GFLOP per step)" % (flops / 1e9))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": "one head per N"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import exact_io_aware_101_b200 as ea
+    rank, world, local = dist_setup(args)
+    lib = ea.library()
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    sweep = [Prefill(c, lib) for c in syn.MHA_SWEEP]
+    sweep_flops = sum(p.cfg.flops for p in sweep)
+
+    # warm-up, then exactly K timed steps bracketed by barrier + synchronize
+    for _ in range(args.warmup):
+        for p in sweep:
+            flush.zero_()
+            p.launch()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_wall0 = time.perf_counter()
+        times, launches = timed_launches(sweep, flush, args.steps)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall0
+    barrier(world)
+    torch.cuda.synchronize()
+    if ea.device_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+
+    kernel_s = sum(sum(row) for row in times) / 1e3
+    kernel_s_max = max_over_ranks(kernel_s, world)
+    value = aggregate(sweep_flops * args.steps, world, kernel_s_max) / 1e12
+    ms_per_step = kernel_s_max * 1e3 / args.steps
+    per_n = {p.cfg.name: p.cfg.flops / (sum(t) / len(t) / 1e3) / 1e12 for p, t in zip(sweep, times)}
+
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = profiled_traffic("prefill_bf16_mha_sweep.md", "prefill_sm100.cu")
+    roofline = {"bound": "tensor", "achieved": sweep_flops * args.steps / kernel_s / 1e12,
+                "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": sweep_flops * args.steps / kernel_s / 1e12 / peak_tf,
+                "traffic": traffic, "peak_source": peak_kind + " (bf16_tflops, burst)",
+                "kernel": "prefill_bf16_kernel<128>",
+                "per_launch": "FLOP-weighted over the 5 sweep launches"}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 2 * world, "seq_len": "512..8192",
+                       "parallelism": "replicas x%d" % world,
+                       "l2": "flushed before every launch (256 MiB write, outside the timing)"},
+            "per_seq_len_tflops": per_n, "roofline": roofline, "gpu_launches": launches,
+            "wall_s_timed_region": t_wall}
+    clocks = clk.summary()
+    if clocks:
+        line["clocks"] = clocks
+
+    if not args.skip_components:
+        comps = {}
+        for cfg in (syn.CAUSAL, syn.GQA):
+            it = Prefill(cfg, lib)
+            timed_launches([it], flush, 3)
+            t, _ = timed_launches([it], flush, args.component_reps)
+            sec = sum(t[0]) / len(t[0]) / 1e3
+            tf = cfg.flops / sec / 1e12
+            comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3}
+            del it
+        dec = Decode(syn.DECODE, lib)
+        timed_launches([dec], flush, 3)
+        t, _ = timed_launches([dec], flush, args.component_reps)
+        sec = sum(t[0]) / len(t[0]) / 1e3
+        gbs = dec.bytes / sec / 1e9
+        comps["decode_paged_gqa"] = {"gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3,
+                                     "algorithmic_bytes": dec.bytes,
+                                     "peak_gbs": peak_hbm,
+                                     "traffic": profiled_traffic("decode_paged_gqa.md",
+                                                                 "decode_paged.cu")}
+        if ea.device_status() != 0:
+            raise RuntimeError("device status word set in the component runs")
+        line["components"] = comps
+        del dec
+
+    if not args.skip_e2e:
+        ms, h2d, d2h = e2e_sweep(sweep, max(1, min(args.steps, 5)))
+        e2e_s = max_over_ranks(ms / 1e3, world)
+        line["e2e"] = {"value": aggregate(sweep_flops, world, e2e_s) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_oracle_sample()
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--component-reps", type=int, default=10)
+    ap.add_argument("--skip-components", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: at least 3 warm-up steps are required; using 3", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,187 @@
+"""exact_io_aware_101_b200 -- exact, IO-aware attention on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libexattn.so`` (C ABI in ``include/exattn.h``).
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks tensors, allocates outputs with PyTorch and passes device pointers
+and the current CUDA stream.  There is no fallback: if the library is missing
+or the device is not sm_100, calls raise.
+
+    o, lse = attn_fwd(q, k, v, causal=True)                  # bf16 prefill
+    o, lse = attn_fwd_f32(q, k, v)                           # fp32 prefill
+    o, lse = attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "attn_fwd", "attn_fwd_f32", "attn_decode_paged", "decode_workspace_bytes",
+    "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
+    "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "AttnError",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
+EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_decode_workspace_bytes",
+                    "attn_decode_paged", "attn_device_status", "attn_status_string",
+                    "attn_version")
+ATTN_DEV_BAD_PAGE = 0x1
+ATTN_DEV_TIMEOUT = 0x2
+_STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_CUDA"}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s" % (what, _STATUS.get(code, "status %d" % code)))
+        self.code = code
+
+
+def library() -> ctypes.CDLL:
+    """Load libexattn.so (built by ``python -m exact_io_aware_101_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libexattn.so is not built (%s); run "
+                              "`python -m exact_io_aware_101_b200.build`" % LIB_PATH)
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+        lib.attn_fwd.restype = ci
+        lib.attn_fwd_f32.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+        lib.attn_fwd_f32.restype = ci
+        lib.attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+        lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+        lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
+                                          cf, vp, ctypes.c_size_t, vp]
+        lib.attn_decode_paged.restype = ci
+        lib.attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
+        lib.attn_device_status.restype = ci
+        lib.attn_status_string.argtypes = [ci]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        lib.attn_version.argtypes = []
+        lib.attn_version.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return library().attn_status_string(int(code)).decode()
+
+
+def version() -> str:
+    return library().attn_version().decode()
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got shape %s" % (name, ndim, tuple(t.shape)))
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _raise(rc: int, what: str):
+    if rc != 0:
+        raise AttnError(rc, what)
+
+
+def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, dtype, 4)
+    B, Hq, N, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError("k/v must be [B, Hkv, N, d] matching q %s" % (tuple(q.shape),))
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check(out, "out", dtype, 4)
+    _check(lse, "lse", torch.float32, 3)
+    if tuple(out.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, N):
+        raise ValueError("out/lse shapes do not match q")
+    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _stream(q))
+    _raise(rc, what)
+    return out, lse
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """bf16 prefill: q [B,Hq,N,d], k/v [B,Hkv,N,d] -> (O bf16 [B,Hq,N,d], L fp32 [B,Hq,N])."""
+    return _prefill(library().attn_fwd, "attn_fwd", q, k, v, causal, scale, out, lse,
+                    torch.bfloat16)
+
+
+def attn_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """fp32 prefill with fp32 arithmetic throughout."""
+    return _prefill(library().attn_fwd_f32, "attn_fwd_f32", q, k, v, causal, scale, out, lse,
+                    torch.float32)
+
+
+def decode_workspace_bytes(S: int, Hq: int, d: int, max_blocks: int, page_size: int = 16) -> int:
+    return int(library().attn_decode_workspace_bytes(S, Hq, d, max_blocks, page_size))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float | None = None,
+                      out=None, lse=None, workspace=None):
+    """Paged single-token decode.
+
+    q [S,Hq,d] bf16; k_pages/v_pages [num_pages,Hkv,page_size,d] bf16;
+    block_table [S,max_blocks] int32; seq_lens [S] int32 (all on the GPU).
+    Returns (O bf16 [S,Hq,d], L fp32 [S,Hq]).  ``workspace`` (uint8, at least
+    decode_workspace_bytes(...) bytes) is allocated when not given.
+    """
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    S, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = k_pages.shape
+    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("page pools must be [num_pages, Hkv, page_size, d]")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table/seq_lens must have S rows")
+    max_blocks = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 3)
+    _check(lse, "lse", torch.float32, 2)
+    need = decode_workspace_bytes(S, Hq, d, max_blocks, page_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace", torch.uint8, 1)
+    rc = library().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                     block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+                                     lse.data_ptr(), S, Hq, Hkv, d, page_size, max_blocks,
+                                     num_pages, float(scale), workspace.data_ptr(),
+                                     workspace.numel(), _stream(q))
+    _raise(rc, "attn_decode_paged")
+    return out, lse
+
+
+def device_status(clear: bool = False) -> int:
+    """Status bits (ATTN_DEV_*) raised by kernels on the current device; syncs the device."""
+    st = ctypes.c_uint(0)
+    _raise(library().attn_device_status(ctypes.byref(st), int(bool(clear))), "attn_device_status")
+    return int(st.value)

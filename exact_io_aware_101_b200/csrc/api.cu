@@ -1,0 +1,147 @@
+// api.cu -- the C ABI declared in include/exattn.h: argument checks, device
+// checks and the per-device status word, then a launch of the right kernel.
+// Nothing here allocates, frees or synchronises (except attn_device_status).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "internal.h"
+
+namespace exattn {
+namespace {
+
+// Status bits raised by kernels on this device (ATTN_DEV_*).
+__device__ unsigned g_status = 0;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+unsigned *g_status_ptr[kMaxDevices] = {};
+int g_is_sm100[kMaxDevices] = {};  // 0 unknown, 1 yes, -1 no
+
+// Device address of this device's status word, looked up once per device
+// (a __device__ variable's address is only meaningful on the device side).
+bool device_state(unsigned **status, bool *sm100) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return false;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return false;
+    g_is_sm100[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    g_status_ptr[dev] = static_cast<unsigned *>(p);
+  }
+  *status = g_status_ptr[dev];
+  *sm100 = g_is_sm100[dev] == 1;
+  return true;
+}
+
+bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool good_scale(float s) { return isfinite(s) && s >= 0.f; }
+
+attn_status_t check_prefill(const void *q, const void *k, const void *v, const void *o,
+                            const void *lse, int B, int Hq, int Hkv, int N, int d, float scale) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse))
+    return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || Hq % Hkv != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!good_scale(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq * N * d >= (1LL << 40)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace exattn
+
+using namespace exattn;
+
+extern "C" {
+
+attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                       int Hq, int Hkv, int N, int d, float scale, int causal,
+                       attn_stream_t stream) {
+  attn_status_t st = check_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
+  if (st != ATTN_OK) return st;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_prefill_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal,
+                             reinterpret_cast<cudaStream_t>(stream), status);
+}
+
+attn_status_t attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           attn_stream_t stream) {
+  attn_status_t st = check_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
+  if (st != ATTN_OK) return st;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_prefill_f32(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_blocks, int page_size) {
+  if (S <= 0 || Hq <= 0 || max_blocks <= 0 || page_size != 16 || (d != 64 && d != 128)) return 0;
+  return decode_workspace_bytes(S, Hq, d, max_blocks);
+}
+
+attn_status_t attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                const int32_t *block_table, const int32_t *seq_lens, void *o,
+                                float *lse, int S, int Hq, int Hkv, int d, int page_size,
+                                int max_blocks, int num_pages, float scale, void *workspace,
+                                size_t workspace_bytes, attn_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned4(block_table) ||
+      !aligned4(seq_lens) || !aligned16(o) || !aligned4(lse) || !aligned16(workspace))
+    return ATTN_ERR_INVALID_ARG;
+  if (S <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || page_size <= 0 ||
+      max_blocks <= 0 || num_pages <= 0 || !good_scale(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || page_size != 16) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks) * page_size > (1LL << 30)) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < decode_workspace_bytes(S, Hq, d, max_blocks)) return ATTN_ERR_INVALID_ARG;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_decode_paged(q, k_pages, v_pages, block_table, seq_lens, o, lse, S, Hq, Hkv, d,
+                             max_blocks, num_pages, scale, workspace,
+                             reinterpret_cast<cudaStream_t>(stream), status);
+}
+
+attn_status_t attn_device_status(unsigned *status, int clear) {
+  if (!status) return ATTN_ERR_INVALID_ARG;
+  unsigned *dev_ptr = nullptr;
+  bool sm100 = false;
+  if (!device_state(&dev_ptr, &sm100)) return ATTN_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpy(status, dev_ptr, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (clear && cudaMemset(dev_ptr, 0, sizeof(unsigned)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (clear && cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+const char *attn_status_string(attn_status_t status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+  }
+  return "ATTN_UNKNOWN_STATUS";
+}
+
+const char *attn_version(void) { return "exattn 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,30 @@
+// internal.h -- launchers shared between the kernel files and the C ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/exattn.h"
+
+namespace exattn {
+
+attn_status_t launch_prefill_bf16(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                                  cudaStream_t stream, unsigned *status);
+
+attn_status_t launch_prefill_f32(const float *q, const float *k, const float *v, float *o,
+                                 float *lse, int B, int Hq, int Hkv, int N, int d, float scale,
+                                 int causal, cudaStream_t stream);
+
+// Number of key chunks (pages per chunk fixed) a sequence of max_blocks pages
+// can be split into, and the workspace layout that follows from it.
+int decode_max_splits(int max_blocks);
+size_t decode_workspace_bytes(int S, int Hq, int d, int max_blocks);
+
+attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                  const int *block_table, const int *seq_lens, void *o, float *lse,
+                                  int S, int Hq, int Hkv, int d, int max_blocks, int num_pages,
+                                  float scale, void *workspace, cudaStream_t stream,
+                                  unsigned *status);
+
+}  // namespace exattn

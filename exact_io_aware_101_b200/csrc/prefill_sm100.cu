@@ -1,0 +1,440 @@
+// prefill_sm100.cu -- bf16 exact attention forward on B200 tensor cores.
+//
+// What it computes: O = softmax(scale * Q K^T [causal]) V and the logsumexp L
+// for every query row, exactly up to float32 rounding ("Phase 08 -- Inference
+// Optimization at Depth", Concepts: FlashAttention tiling and online softmax;
+// Lab 01 steps 2 and 4).  Q is split into 128-row tiles; each tile walks the
+// 128-key K/V tiles keeping a running max m and sum l per row, rescaling the
+// accumulator when m grows, and writes O / l and L = m + ln l once.  The N x N
+// score matrix exists only one 128 x 128 tile at a time, in tensor memory.
+//
+// How it maps to sm_100a:
+//  * one CTA = 2 Q tiles (256 rows) of one (batch, head); 12 warps:
+//      warp 0      TMA producer: Q once, then K0 V0 K1 V1 ... into a ring of
+//                  NST shared-memory slots (128B-swizzled, no multicast);
+//      warp 1      allocates the 512 TMEM columns and issues every tcgen05.mma
+//                  from one thread;
+//      warps 4-7   softmax/correction/epilogue for Q tile 0 (TMEM lanes 0-127);
+//      warps 8-11  the same for Q tile 1.
+//  * TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [384,384+d).
+//    P (bf16) overwrites the first 64 columns of its S tile and feeds the
+//    second GEMM straight from TMEM, so P never touches shared memory.
+//  * S_t = Q_t K^T: 128x128x16 kind::f16 MMAs, both operands K-major.
+//    O_t += P_t V: A = P from TMEM, B = V as an MN-major operand.
+//  * The two Q tiles ping-pong: while softmax works on S0(j) the tensor pipe
+//    runs S1(j) and PV of the other tile, and vice versa.
+//  * exp2-based online softmax with scale*log2(e) folded into one FMA and a
+//    lazy rescale: the reference max m only moves (and O is rescaled in TMEM)
+//    when a row's max grows by more than 8 in log2 units; O/l stays exact.
+//  * Causal: KV tiles above the diagonal are never loaded or multiplied; only
+//    diagonal tiles are masked (Concepts: causal masking; Lab 01 step 4).
+//  * Grid: one CTA per (Q-tile pair, batch*head), heaviest causal pairs first;
+//    consecutive CTAs are the query heads that share one K/V head, so GQA's K/V
+//    tiles are reused from L2.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace exattn {
+
+namespace {
+
+constexpr int BM = 128;       // query rows per Q tile
+constexpr int BN = 128;       // keys per K/V tile
+constexpr int NUM_THREADS = 384;
+constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 128-byte swizzle column block
+
+template <int D>
+struct Cfg {
+  static constexpr int CH = D / 64;                  // 64-element (128 B) column blocks
+  static constexpr int TILE_BYTES = BM * D * 2;      // a Q, K or V tile
+  static constexpr int NST = (D == 64) ? 8 : 4;      // ring slots
+  static constexpr int Q_OFF = 0;
+  static constexpr int RING_OFF = 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = RING_OFF + NST * TILE_BYTES;
+  static constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;  // + barriers + 1 KB align slack
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+};
+
+struct Bars {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Params {
+  void *o;
+  float *lse;
+  unsigned *status;
+  int B, Hq, Hkv, N;
+  int pairs;  // ceil(N / 256)
+  float scale_log2;
+  int causal;
+};
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem + C::Q_OFF;
+  uint8_t *sRing = smem + C::RING_OFF;
+  Bars *bars = reinterpret_cast<Bars *>(smem + C::BAR_OFF);
+  volatile int *abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: Q-tile pair and (batch, head); heaviest causal pairs first
+  const int BH = p.B * p.Hq;
+  const int pair = p.pairs - 1 - static_cast<int>(blockIdx.x / BH);
+  const int bh = static_cast<int>(blockIdx.x % BH);
+  const int b = bh / p.Hq;
+  const int hq = bh % p.Hq;
+  const int hkv = hq / (p.Hq / p.Hkv);
+  const int row0 = pair * 2 * BM;
+  const int nkv = (p.N + BN - 1) / BN;
+  const int n0 = p.causal ? min(2 * pair + 1, nkv) : nkv;
+  const int n1 = (row0 + BM < p.N) ? (p.causal ? min(2 * pair + 2, nkv) : nkv) : 0;
+  const int n = max(n0, n1);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NST; ++i) {
+      mbar_init(&bars->full[i], 1);
+      mbar_init(&bars->empty[i], 1);
+    }
+    mbar_init(&bars->q_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], BM);
+      mbar_init(&bars->o_full[t], 1);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int zq = b * p.Hq + hq;
+      const int zkv = b * p.Hkv + hkv;
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
+                      row0 + t * BM, zq);
+      int issued = 0;
+      for (int i = 0; i < 2 * n; ++i) {
+        const int slot = i % C::NST;
+        const int round = i / C::NST;
+        if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
+        const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
+                      64 * c, (i >> 1) * BN, zkv);
+        issued = i + 1;
+      }
+      // Drain: no copy may still be writing shared memory when the CTA exits.
+      // Normally these phases completed long ago and each wait returns at once.
+      mbar_wait_drain(&bars->q_full, 0, p.status);
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
+        mbar_wait_drain(&bars->full[i % C::NST], (i / C::NST) & 1, p.status);
+    }
+  } else if (warp == 1) {
+    // ================================================================== MMA
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t ring_base = smem_u32(sRing);
+      auto slot_of = [](int i) { return i % C::NST; };
+      auto wait_full = [&](int i) {
+        return mbar_wait(&bars->full[i % C::NST], (i / C::NST) & 1, abort_flag, p.status);
+      };
+      auto issue_s = [&](int t, int kidx) {  // S_t = Q_t K^T
+        const uint32_t kb = ring_base + slot_of(kidx) * C::TILE_BYTES;
+        const uint32_t qb = q_base + t * C::TILE_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * CHUNK_BYTES + (ks & 3) * 32;
+          mma_ss(tmem + t * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                 C::IDESC_QK, ks > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int vidx, bool acc) {  // O_t (+)= P_t V
+        const uint32_t vb = ring_base + slot_of(vidx) * C::TILE_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          mma_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8,
+                 sdesc_sw128(vb + ks * 16 * 128, CHUNK_BYTES, 1024), C::IDESC_PV,
+                 (acc || ks > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.status);
+      ok = ok && wait_full(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        tc_commit(&bars->s_full[0]);
+        if (n1 > 0) {
+          issue_s(1, 0);
+          tc_commit(&bars->s_full[1]);
+        }
+        tc_commit(&bars->empty[slot_of(0)]);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const uint32_t ph = j & 1;
+        bool v_ready = false;
+        if (j < n0) {
+          if (!(ok = mbar_wait(&bars->p_full[0], ph, abort_flag, p.status) && wait_full(2 * j + 1)))
+            break;
+          v_ready = true;
+          tc_fence_after();
+          issue_pv(0, 2 * j + 1, j > 0);
+          tc_commit(&bars->o_full[0]);
+        }
+        if (j + 1 < n && !(ok = wait_full(2 * j + 2))) break;
+        if (j + 1 < n0) {
+          // P0(j) aliases S0: the next S0 may only be written once PV0(j) has read it.
+          if (!(ok = mbar_wait(&bars->o_full[0], ph, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_s(0, 2 * j + 2);
+          tc_commit(&bars->s_full[0]);
+        }
+        if (j < n1) {
+          if (!(ok = mbar_wait(&bars->p_full[1], ph, abort_flag, p.status))) break;
+          if (!v_ready && !(ok = wait_full(2 * j + 1))) break;
+          tc_fence_after();
+          issue_pv(1, 2 * j + 1, j > 0);
+          tc_commit(&bars->o_full[1]);
+        }
+        tc_commit(&bars->empty[slot_of(2 * j + 1)]);  // V(j) no longer needed
+        if (j + 1 < n1) {
+          if (!(ok = mbar_wait(&bars->o_full[1], ph, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_s(1, 2 * j + 2);
+          tc_commit(&bars->s_full[1]);
+        }
+        if (j + 1 < n) tc_commit(&bars->empty[slot_of(2 * j + 2)]);  // K(j+1) done
+      }
+      // Every MMA issued above must finish before TMEM is released.
+      tc_commit(&bars->mma_done);
+      mbar_wait_drain(&bars->mma_done, 0, p.status);
+    }
+  } else if (warp >= 4) {
+    // ====================================================== softmax / epilogue
+    const int t = (warp - 4) >> 2;        // Q tile of this warpgroup
+    const int quarter = warp & 3;         // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;    // row within the Q tile
+    const int qtile = 2 * pair + t;
+    const int row = qtile * BM + r;
+    const int nt = t == 0 ? n0 : n1;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + t * 128;
+    const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+    const float c = p.scale_log2;
+    float m = -INFINITY;  // reference max, in log2 units of scaled scores
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      ok = mbar_wait(&bars->s_full[t], j & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      int limit = min(BN, p.N - j * BN);
+      if (p.causal && j == qtile) limit = min(limit, r + 1);
+      uint32_t sv[32];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        tmem_ld32(s_addr + cc * 32, sv);
+        tmem_ld_wait(sv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float s = __uint_as_float(sv[i]);
+          mx = fmaxf(mx, (cc * 32 + i < limit) ? s : -INFINITY);
+        }
+      }
+      const float m_new = fmaxf(m, mx * c);
+      const bool resc = m_new > m + 8.0f;
+      const float alpha = resc ? ex2(m - m_new) : 1.0f;
+      if (resc) m = m_new;
+      l *= alpha;
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // O is stable here: S(j) completing implies PV(j-1) completed.
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+          tmem_ld_wait(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(o_addr + cc * 32, ov);
+        }
+      }
+      const float neg_m = -m;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        tmem_ld32(s_addr + cc * 32, sv);
+        tmem_ld_wait(sv);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int col = cc * 32 + i;
+          const float p0 = (col < limit) ? ex2(fmaf(__uint_as_float(sv[i]), c, neg_m)) : 0.f;
+          const float p1 = (col + 1 < limit) ? ex2(fmaf(__uint_as_float(sv[i + 1]), c, neg_m)) : 0.f;
+          l += p0 + p1;
+          pk[i >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_addr + cc * 16, pk);  // P columns [16cc, 16cc+16) <- S columns already read
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[t]);
+    }
+    if (ok && nt > 0) {
+      ok = mbar_wait(&bars->o_full[t], (nt - 1) & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l;
+        const bool valid = row < p.N;
+        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                              ((static_cast<size_t>(b) * p.Hq + hq) * p.N + (valid ? row : 0)) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+          tmem_ld_wait(ov);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            pk[i >> 1] = pack_bf16x2(__uint_as_float(ov[i]) * inv_l, __uint_as_float(ov[i + 1]) * inv_l);
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+        if (valid)
+          p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.N + row] =
+              (m + log2f(l)) * 0.6931471805599453f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [BH][N][D] bf16 viewed as a 3-D tensor; boxes of 64 x 128 x 1, 128B swizzle.
+bool make_map(CUtensorMap *map, const void *base, int D, int N, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+attn_status_t launch(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                     int Hq, int Hkv, int N, float scale, int causal, cudaStream_t stream,
+                     unsigned *status) {
+  using C = Cfg<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, N, B * Hq) || !make_map(&mk, k, D, N, B * Hkv) ||
+      !make_map(&mv, v, D, N, B * Hkv))
+    return ATTN_ERR_CUDA;
+  Params prm;
+  prm.o = o;
+  prm.lse = lse;
+  prm.status = status;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.N = N;
+  prm.pairs = (N + 2 * BM - 1) / (2 * BM);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.causal = causal ? 1 : 0;
+  const long long ctas = static_cast<long long>(prm.pairs) * B * Hq;
+  if (ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  prefill_bf16_kernel<D><<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(
+      mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+attn_status_t launch_prefill_bf16(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                                  cudaStream_t stream, unsigned *status) {
+  if (d == 128) return launch<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, stream, status);
+  if (d == 64) return launch<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, stream, status);
+  return ATTN_ERR_UNSUPPORTED;
+}
+
+}  // namespace exattn

@@ -1,0 +1,149 @@
+/*
+ * exattn.h -- C ABI of the exact, IO-aware attention library (libexattn.so).
+ *
+ * The library computes exact scaled-dot-product attention on one NVIDIA B200
+ * (sm_100a):
+ *
+ *   O = softmax(scale * Q K^T [+ causal mask]) V,   L = logsumexp of each row
+ *
+ * tile by tile with an online softmax, never writing the N x N score matrix to
+ * memory ("Phase 08 -- Inference Optimization at Depth", Concepts: standard
+ * attention memory, FlashAttention tiling, online softmax, logsumexp L for the
+ * backward pass; Lab 01 steps 2 and 4), for grouped-/multi-query heads
+ * (screna.ai interview page, MHA/MQA/GQA answer) and as a single-token decode
+ * over a paged KV cache (Phase 08 page, Concepts: KV cache and paged attention;
+ * Lab 03 step 4: pages reached through an indirection table).
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers to dense, row-major (C order)
+ *    arrays owned by the caller.  The library never allocates, frees or
+ *    synchronises; work is enqueued on `stream` (0 = legacy default stream) and
+ *    the call returns before it finishes.
+ *  - Pointers must be 16-byte aligned.
+ *  - Errors are reported only through the return value; nothing is written when
+ *    a call returns anything but ATTN_OK.  No call aborts or traps.
+ *  - Device-side conditions that the host cannot see in advance (a block-table
+ *    entry outside the page pool, a bounded wait that ran out) set bits in a
+ *    per-device status word read with attn_device_status().
+ *  - `causal` means key j is visible to query i iff j <= i (queries and keys
+ *    share positions 0..N-1).
+ *  - L is the natural logarithm of sum_j exp(scale * q_i . k_j) over the
+ *    visible keys, stored as float32.
+ *  - Query head h reads key/value head h / (Hq / Hkv): consecutive groups of
+ *    Hq/Hkv query heads share one K/V head (Hkv == Hq is multi-head,
+ *    Hkv == 1 is multi-query attention).
+ */
+#ifndef EXATTN_H_
+#define EXATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EXATTN_API __attribute__((visibility("default")))
+#else
+#define EXATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Stream handle: the CUDA runtime's cudaStream_t (a CUstream_st pointer). */
+typedef struct CUstream_st *attn_stream_t;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, Hq % Hkv != 0, bad scale */
+    ATTN_ERR_UNSUPPORTED = 2,   /* head dim / page size not built, or no sm_100 device */
+    ATTN_ERR_CUDA = 3           /* a CUDA runtime or driver call failed */
+} attn_status_t;
+
+/* Bits of the per-device status word (attn_device_status). */
+#define ATTN_DEV_BAD_PAGE 0x1u  /* a decode sequence referenced a page outside the pool or
+                                   had a length outside [0, max_blocks*page_size]; its
+                                   outputs are NaN */
+#define ATTN_DEV_TIMEOUT 0x2u   /* a bounded wait inside the prefill kernel expired; the
+                                   kernel returned early and its outputs are undefined */
+
+/*
+ * attn_fwd -- bf16 prefill, forward only.  Lab 01 steps 2 and 4 of the Phase 08
+ * page: Q is split into row tiles; for each, the kernel walks the K/V column
+ * tiles with a running max and sum, rescales the accumulator, and writes O and
+ * L once.  With causal != 0, tiles wholly above the diagonal are skipped and
+ * only diagonal tiles are masked (Concepts: causal masking in FlashAttention).
+ *
+ *   q    [B, Hq,  N, d] bf16        k, v [B, Hkv, N, d] bf16
+ *   o    [B, Hq,  N, d] bf16 (out)  lse  [B, Hq, N] float32 (out)
+ *   d in {64, 128}; N >= 1; B, Hq, Hkv >= 1; Hq % Hkv == 0;
+ *   scale finite and >= 0 (the workloads use 1/sqrt(d)).
+ * Accumulation is float32; O is rounded to nearest-even bf16.
+ * Returns ATTN_ERR_UNSUPPORTED if the current device is not sm_100.
+ */
+EXATTN_API attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                       attn_stream_t stream);
+
+/*
+ * attn_fwd_f32 -- the same operation on float32 tensors (o is float32), with
+ * float32 arithmetic throughout; the correctness path for the fp32 workload
+ * (Lab 01 step 3: match standard attention within 1e-4).  d in {64, 128}.
+ */
+EXATTN_API attn_status_t attn_fwd_f32(const float *q, const float *k, const float *v, float *o,
+                           float *lse, int B, int Hq, int Hkv, int N, int d, float scale,
+                           int causal, attn_stream_t stream);
+
+/*
+ * attn_decode_workspace_bytes -- bytes of device workspace attn_decode_paged
+ * needs for S sequences, Hq query heads, head dim d and at most max_blocks
+ * pages per sequence.  Returns 0 for invalid sizes.
+ */
+EXATTN_API size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_blocks, int page_size);
+
+/*
+ * attn_decode_paged -- one query token per sequence against its paged KV cache
+ * (Phase 08 page, Concepts: KV cache, paged attention; Lab 03 step 4).  Token t
+ * of sequence s lives in page block_table[s, t / page_size] at slot
+ * t % page_size; each sequence sees all of its seq_lens[s] tokens (the query is
+ * the newest token, so no mask applies).  The key range of a sequence is split
+ * into fixed-size chunks processed in parallel; a second kernel merges the
+ * chunks' partial outputs with their logsumexp weights.
+ *
+ *   q            [S, Hq, d] bf16
+ *   k_pages      [num_pages, Hkv, page_size, d] bf16   v_pages likewise
+ *   block_table  [S, max_blocks] int32 (entries past a sequence's last page are not read)
+ *   seq_lens     [S] int32, each in [0, max_blocks * page_size]
+ *   o            [S, Hq, d] bf16 (out)      lse [S, Hq] float32 (out)
+ *   workspace    device scratch of at least attn_decode_workspace_bytes(...) bytes,
+ *                owned by the caller; its contents need no initialisation.
+ * d in {64, 128}; page_size == 16; Hq / Hkv in {1, 2, 4, 8, 16, 32, ...} (any divisor).
+ * A sequence of length 0 gets O = 0 and L = -inf.  A sequence with a page id
+ * outside [0, num_pages) or an out-of-range length gets NaN outputs and sets
+ * ATTN_DEV_BAD_PAGE; no out-of-range address is ever dereferenced.
+ */
+EXATTN_API attn_status_t attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                const int32_t *block_table, const int32_t *seq_lens,
+                                void *o, float *lse,
+                                int S, int Hq, int Hkv, int d, int page_size,
+                                int max_blocks, int num_pages, float scale,
+                                void *workspace, size_t workspace_bytes,
+                                attn_stream_t stream);
+
+/*
+ * attn_device_status -- read (and, if clear != 0, reset) the status word of the
+ * current device.  Synchronises the device first, so call it between steps, not
+ * inside stream capture.
+ */
+EXATTN_API attn_status_t attn_device_status(unsigned *status, int clear);
+
+/* attn_status_string -- a static, human-readable name for a status code. */
+EXATTN_API const char *attn_status_string(attn_status_t status);
+
+/* attn_version -- library version string. */
+EXATTN_API const char *attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXATTN_H_ */

@@ -1,0 +1,127 @@
+"""The C ABI boundary on the CPU: the library loads, exports every entry point
+that include/exattn.h declares, and rejects bad arguments before touching the
+GPU.  No call here reaches a kernel launch."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+import exact_io_aware_101_b200 as ea  # noqa: E402
+from exact_io_aware_101_b200 import build as eabuild  # noqa: E402
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.fixture(scope="module")
+def lib():
+    eabuild.build()
+    return ea.library()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert {"attn_fwd", "attn_fwd_f32", "attn_decode_paged",
+            "attn_decode_workspace_bytes"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(ea.EXPORTED_SYMBOLS) >= declared_functions()
+
+
+def test_only_the_c_abi_is_exported(lib):
+    # -fvisibility=hidden keeps internal C++ symbols out of the dynamic table.
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ea.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert {s for s in exported if s.startswith("attn_")} == declared_functions()
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in ea.version()
+    assert ea.status_string(0) == "ATTN_OK"
+    assert ea.status_string(1) == "ATTN_ERR_INVALID_ARG"
+    assert ea.status_string(2) == "ATTN_ERR_UNSUPPORTED"
+    assert ea.status_string(3) == "ATTN_ERR_CUDA"
+    assert ea.status_string(99) == "ATTN_UNKNOWN_STATUS"
+
+
+A = 1 << 20  # a fake, 16-byte-aligned address: validation fails before any use
+
+
+def fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, Hq=2, Hkv=1, N=16, d=128, scale=0.1, causal=0):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(o=A + 8), INVALID), (dict(lse=A + 2), INVALID),
+    (dict(B=0), INVALID), (dict(N=0), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(Hkv=0), INVALID), (dict(scale=float("nan")), INVALID), (dict(scale=-1.0), INVALID),
+    (dict(scale=float("inf")), INVALID), (dict(d=96), UNSUPPORTED), (dict(d=256), UNSUPPORTED),
+])
+def test_prefill_argument_checks(lib, kw, code):
+    assert fwd(lib, **kw) == code
+    assert lib.attn_fwd_f32(*(kw.get(n, A) for n in ("q", "k", "v", "o", "lse")),
+                            kw.get("B", 1), kw.get("Hq", 2), kw.get("Hkv", 1), kw.get("N", 16),
+                            kw.get("d", 128), kw.get("scale", 0.1), 0, None) == code
+
+
+def test_decode_workspace_size(lib):
+    # 512 pages of 16 tokens in chunks of 32 pages -> 16 chunks per sequence.
+    n = ea.decode_workspace_bytes(64, 32, 128, 512)
+    parts = 64 * 32 * 16
+    assert n >= parts * 129 * 4 and n % 256 == 0 and n < parts * 129 * 4 + 512
+    assert ea.decode_workspace_bytes(64, 32, 96, 512) == 0
+    assert ea.decode_workspace_bytes(64, 32, 128, 512, page_size=32) == 0
+    assert ea.decode_workspace_bytes(0, 32, 128, 512) == 0
+
+
+def dec(lib, ws_bytes=None, **kw):
+    a = dict(q=A, kp=A, vp=A, bt=A, sl=A, o=A, lse=A, S=4, Hq=8, Hkv=2, d=128, ps=16, maxb=8,
+             npages=100, scale=0.1, ws=A)
+    a.update(kw)
+    need = lib.attn_decode_workspace_bytes(a["S"], a["Hq"], a["d"], a["maxb"], 16) or 1 << 20
+    return lib.attn_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["o"], a["lse"],
+                                 a["S"], a["Hq"], a["Hkv"], a["d"], a["ps"], a["maxb"],
+                                 a["npages"], a["scale"], a["ws"],
+                                 need if ws_bytes is None else ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(ws=None), INVALID), (dict(kp=A + 4), INVALID),
+    (dict(bt=A + 2), INVALID), (dict(S=0), INVALID), (dict(Hq=6, Hkv=4), INVALID),
+    (dict(maxb=0), INVALID), (dict(npages=0), INVALID), (dict(scale=-0.5), INVALID),
+    (dict(d=80), UNSUPPORTED), (dict(ps=8), UNSUPPORTED),
+])
+def test_decode_argument_checks(lib, kw, code):
+    assert dec(lib, **kw) == code
+
+
+def test_decode_rejects_small_workspace(lib):
+    assert dec(lib, ws_bytes=64) == INVALID
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ea.attn_fwd(q, q, q)
+    with pytest.raises(TypeError):
+        ea.attn_fwd(q.float(), q.float(), q.float())

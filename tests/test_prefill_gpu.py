@@ -1,0 +1,156 @@
+"""GPU parity of the prefill paths (attn_fwd bf16, attn_fwd_f32) against the
+fp64 oracle, through the C ABI, on seeded synthetic inputs.
+
+Small shapes are compared element by element over every output; they span
+several 128-row tiles, ragged tails, single rows, both head dims, causal and
+not, and MHA / GQA / MQA head sharing.  The full-size workloads run in the
+same launch configuration as bench.py and are compared on sampled rows the
+oracle evaluates one by one, plus properties that hold at any size.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import exact_io_aware_101_b200 as ea
+from exact_io_aware_101_b200 import synthetic as syn
+from parity_helpers import assert_bf16_parity, assert_f32_parity, f32
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+SMALL = [
+    # B, Hq, Hkv, N, d, causal
+    (1, 1, 1, 1, 64, False),
+    (1, 1, 1, 1, 128, True),
+    (1, 2, 2, 17, 128, False),
+    (1, 2, 2, 17, 128, True),
+    (2, 4, 1, 127, 64, True),      # MQA
+    (1, 4, 2, 128, 128, False),
+    (1, 4, 2, 129, 128, True),
+    (2, 8, 2, 255, 128, True),     # GQA, ragged second tile
+    (1, 2, 2, 256, 64, False),
+    (1, 2, 1, 257, 128, True),
+    (1, 3, 1, 384, 128, False),    # last CTA holds one valid Q tile
+    (1, 2, 2, 1000, 128, False),
+    (1, 2, 2, 1000, 128, True),
+    (1, 2, 2, 1000, 64, True),
+    (1, 1, 1, 2048, 128, True),    # many causal tile pairs
+    (3, 6, 3, 640, 128, True),
+]
+
+
+def run_small(B, Hq, Hkv, N, d, causal, seed):
+    q, k, v = syn.random_qkv(B, Hq, Hkv, N, d, seed=seed)
+    scale = 1.0 / math.sqrt(d)
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=scale, causal=causal)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    out = torch.full_like(qd, float("nan"))   # poison: every row must be written
+    lse = torch.full((B, Hq, N), float("nan"), device=DEV)
+    o, l = ea.attn_fwd(qd, kd, vd, causal=causal, scale=scale, out=out, lse=lse)
+    torch.cuda.synchronize()
+    return o, l, o_ref, l_ref
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", SMALL)
+def test_bf16_small_shapes(B, Hq, Hkv, N, d, causal):
+    o, l, o_ref, l_ref = run_small(B, Hq, Hkv, N, d, causal, seed=100 + N + d + Hq)
+    assert_bf16_parity(o, l, o_ref, l_ref, (B, Hq, Hkv, N, d, causal))
+    assert ea.device_status() == 0
+
+
+def test_bf16_deterministic_and_gqa_equals_repeated_heads():
+    B, Hq, Hkv, N, d = 2, 8, 2, 700, 128
+    q, k, v = (t.to(DEV) for t in syn.random_qkv(B, Hq, Hkv, N, d, seed=7))
+    o1, l1 = ea.attn_fwd(q, k, v, causal=True)
+    o2, l2 = ea.attn_fwd(q, k, v, causal=True)
+    G = Hq // Hkv
+    o3, l3 = ea.attn_fwd(q, k.repeat_interleave(G, 1).contiguous(),
+                         v.repeat_interleave(G, 1).contiguous(), causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
+
+
+def test_bf16_large_scores_stay_finite():
+    # Scores of several hundred: only the running-max shift keeps exp finite.
+    B, H, N, d = 1, 2, 300, 64
+    q, k, v = syn.random_qkv(B, H, H, N, d, seed=11)
+    q = (q.float() * 8).to(torch.bfloat16)
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=1.0, causal=True)
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=1.0)
+    torch.cuda.synchronize()
+    assert np.abs(l_ref).max() > 100
+    # L is large in magnitude here; hold it to the same absolute bound relative to |L|.
+    e = np.abs(f32(l) - l_ref) / np.maximum(1.0, np.abs(l_ref))
+    assert e.max() <= 5e-3
+    assert np.abs(f32(o) - o_ref).max() <= 2e-2
+
+
+def test_fp32_tiny_workload():
+    cfg = syn.TINY
+    q, k, v = syn.prefill_inputs(cfg)
+    o_ref, l_ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale=cfg.scale)
+    o, l = ea.attn_fwd_f32(q.to(DEV), k.to(DEV), v.to(DEV), scale=cfg.scale)
+    torch.cuda.synchronize()
+    assert_f32_parity(o, l, o_ref, l_ref, cfg.name)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [
+    (1, 1, 1, 1, 64, False), (1, 2, 1, 33, 128, True), (2, 4, 2, 200, 64, True),
+    (1, 2, 2, 513, 128, False), (1, 8, 1, 100, 128, False)])
+def test_fp32_shapes(B, Hq, Hkv, N, d, causal):
+    q, k, v = syn.random_qkv(B, Hq, Hkv, N, d, seed=5 + N, dtype=torch.float32)
+    o_ref, l_ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale=0.1, causal=causal)
+    o, l = ea.attn_fwd_f32(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=0.1)
+    torch.cuda.synchronize()
+    assert_f32_parity(o, l, o_ref, l_ref, (B, Hq, Hkv, N, d, causal))
+
+
+def sample_rows(B, Hq, N, n_random, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 129, 255, 256, N // 2, N - 129, N - 128, N - 2, N - 1]
+    rows = []
+    for r in fixed:
+        if 0 <= r < N:
+            rows.append((int(rng.integers(B)), int(rng.integers(Hq)), r))
+    for _ in range(n_random):
+        rows.append((int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(N))))
+    return np.array([(b * Hq + h) * N + i for b, h, i in rows], dtype=np.int64)
+
+
+def full_size_check(cfg, n_random=64):
+    q, k, v = syn.prefill_inputs(cfg, device=DEV)
+    o, l = ea.attn_fwd(q, k, v, causal=cfg.causal, scale=cfg.scale)
+    torch.cuda.synchronize()
+    assert ea.device_status() == 0
+    # properties at any size: finite, and each output column inside the range of
+    # the values it averages (a convex combination of rows of V).
+    assert torch.isfinite(o.float()).all() and torch.isfinite(l).all()
+    G = cfg.Hq // cfg.Hkv
+    vmin = v.float().amin(dim=2).repeat_interleave(G, 1)[:, :, None, :]
+    vmax = v.float().amax(dim=2).repeat_interleave(G, 1)[:, :, None, :]
+    of = o.float()
+    assert bool((of >= vmin - 1e-2).all()) and bool((of <= vmax + 1e-2).all())
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.N, n_random, cfg.seed)
+    qh, kh, vh = q.float().cpu().numpy(), k.float().cpu().numpy(), v.float().cpu().numpy()
+    o_ref, l_ref = oracle.attention_rows(qh, kh, vh, cfg.scale, cfg.causal, rows)
+    o_s = o.reshape(-1, cfg.d)[torch.from_numpy(rows).to(DEV)]
+    l_s = l.reshape(-1)[torch.from_numpy(rows).to(DEV)]
+    return assert_bf16_parity(o_s, l_s, o_ref, l_ref, cfg.name)
+
+
+@pytest.mark.parametrize("cfg", syn.MHA_SWEEP, ids=lambda c: c.name)
+def test_full_size_mha(cfg):
+    full_size_check(cfg)
+
+
+@pytest.mark.parametrize("cfg", [syn.CAUSAL, syn.GQA], ids=lambda c: c.name)
+def test_full_size_causal_and_gqa(cfg):
+    full_size_check(cfg)
