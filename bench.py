@@ -161,7 +161,8 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -263,25 +264,29 @@ def e2e_sweep(items, reps):
     return e0.elapsed_time(e1) / reps, h2d, d2h
 
 
-def cpu_oracle_sample(target_s=12.0, cap_heads=64):
-    """Time the fp64 oracle on whole heads of the N=4096 MHA workload."""
+def cpu_oracle_sample(target_s=10.0):
+    """Time the fp64 oracle on whole (batch, head) slices of the N=8192 MHA workload."""
     import oracle
-    cfg = syn.MHA_SWEEP[3]
+    cfg = syn.MHA_SWEEP[4]
     q, k, v = syn.prefill_inputs(cfg)
-    qf, kf, vf = q.float().numpy(), k.float().numpy(), v.float().numpy()
+    BH = cfg.B * cfg.Hq
+    qf = q.float().reshape(1, BH, cfg.N, cfg.d).numpy()
+    kf = k.float().reshape(1, BH, cfg.N, cfg.d).numpy()
+    vf = v.float().reshape(1, BH, cfg.N, cfg.d).numpy()
     threads = oracle.max_threads()
-    heads, elapsed = 1, 0.0
+    heads = 1
     while True:
         t0 = time.perf_counter()
-        oracle.attention(qf[:1, :heads], kf[:1, :heads], vf[:1, :heads], scale=cfg.scale)
+        oracle.attention(qf[:, :heads], kf[:, :heads], vf[:, :heads], scale=cfg.scale)
         elapsed = time.perf_counter() - t0
-        if elapsed >= target_s / 4 or heads >= cap_heads:
+        if elapsed >= target_s or heads >= BH:
             break
-        heads = min(cap_heads, heads * max(2, int(target_s / 4 / max(elapsed, 1e-3))))
+        heads = min(BH, max(heads + 1, int(heads * target_s / max(elapsed, 1e-3)) + 1))
     flops = 4.0 * heads * cfg.N * cfg.N * cfg.d
     return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": "fp64 oracle (materialised S, two-pass softmax) on %d head(s) of the "
-                      "N=4096 MHA workload: %.1f GFLOP in %.2f s" % (heads, flops / 1e9, elapsed)}
+            "sample": "fp64 oracle (materialised S, two-pass softmax) on %d (batch, head) slice(s) "
+                      "of the N=8192 MHA workload: %.1f GFLOP in %.2f s"
+                      % (heads, flops / 1e9, elapsed)}
 
 
 # --------------------------------------------------------------- arms
