@@ -19,15 +19,18 @@ import os
 import torch
 
 __all__ = [
-    "attn_fwd", "attn_fwd_f32", "attn_decode_paged", "decode_workspace_bytes",
+    "attn_fwd", "attn_fwd_f32", "attn_decode_paged", "attn_decode_paged_noalloc",
+    "decode_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
     "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
     "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "AttnError",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_decode_workspace_bytes",
-                    "attn_decode_paged", "attn_device_status", "attn_status_string",
-                    "attn_version")
+                    "attn_decode_paged", "attn_decode_paged_noalloc", "attn_device_status",
+                    "attn_status_string", "attn_version")
+# Size of the library's fixed per-device scratch used by attn_decode_paged_noalloc.
+DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 ATTN_DEV_BAD_PAGE = 0x1
 ATTN_DEV_TIMEOUT = 0x2
 _STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_CUDA"}
@@ -59,6 +62,9 @@ def library() -> ctypes.CDLL:
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
                                           cf, vp, ctypes.c_size_t, vp]
         lib.attn_decode_paged.restype = ci
+        lib.attn_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
+                                                  ci, ci, cf, vp]
+        lib.attn_decode_paged_noalloc.restype = ci
         lib.attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
         lib.attn_device_status.restype = ci
         lib.attn_status_string.argtypes = [ci]
@@ -177,6 +183,40 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float |
                                      num_pages, float(scale), workspace.data_ptr(),
                                      workspace.numel(), _stream(q))
     _raise(rc, "attn_decode_paged")
+    return out, lse
+
+
+def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens,
+                              scale: float | None = None, out=None, lse=None):
+    """Paged decode that allocates no device memory inside the library.
+
+    For callers that may not call cudaMalloc (for example a plugin whose host
+    program owns all device memory, or a decode loop that must not wait on the
+    allocator): the chunk partials live in the library's fixed per-device scratch
+    (DECODE_NOALLOC_SCRATCH_BYTES), shared by every such call on the device, so
+    calls that overlap on the GPU race.  Pass ``out`` and ``lse`` to avoid torch
+    allocating the outputs here.  Arguments as for attn_decode_paged.
+    """
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    S, Hq, d = q.shape
+    num_pages, Hkv, page_size, _ = k_pages.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 3)
+    _check(lse, "lse", torch.float32, 2)
+    rc = library().attn_decode_paged_noalloc(
+        q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+        seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, page_size,
+        block_table.shape[1], num_pages, float(scale), _stream(q))
+    _raise(rc, "attn_decode_paged_noalloc")
     return out, lse
 
 

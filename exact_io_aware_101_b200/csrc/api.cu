@@ -119,6 +119,35 @@ attn_status_t attn_decode_paged(const void *q, const void *k_pages, const void *
                              reinterpret_cast<cudaStream_t>(stream), status);
 }
 
+// The workspace-free decode: same checks and kernels as attn_decode_paged, with
+// the library's fixed per-device scratch array standing in for the workspace.
+attn_status_t attn_decode_paged_noalloc(const void *q, const void *k_pages, const void *v_pages,
+                                        const int32_t *block_table, const int32_t *seq_lens,
+                                        void *o, float *lse, int S, int Hq, int Hkv, int d,
+                                        int page_size, int max_blocks, int num_pages, float scale,
+                                        attn_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned4(block_table) ||
+      !aligned4(seq_lens) || !aligned16(o) || !aligned4(lse))
+    return ATTN_ERR_INVALID_ARG;
+  if (S <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || page_size <= 0 ||
+      max_blocks <= 0 || num_pages <= 0 || !good_scale(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || page_size != 16) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks) * page_size > (1LL << 30)) return ATTN_ERR_INVALID_ARG;
+  if (decode_workspace_bytes(S, Hq, d, max_blocks) > ATTN_DECODE_NOALLOC_SCRATCH_BYTES)
+    return ATTN_ERR_INVALID_ARG;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  attn_status_t st = noalloc_scratch_address(&scratch);
+  if (st != ATTN_OK) return st;
+  return launch_decode_paged(q, k_pages, v_pages, block_table, seq_lens, o, lse, S, Hq, Hkv, d,
+                             max_blocks, num_pages, scale, scratch,
+                             reinterpret_cast<cudaStream_t>(stream), status);
+}
+
 attn_status_t attn_device_status(unsigned *status, int clear) {
   if (!status) return ATTN_ERR_INVALID_ARG;
   unsigned *dev_ptr = nullptr;

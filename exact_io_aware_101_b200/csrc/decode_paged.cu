@@ -23,6 +23,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "internal.h"
 
 namespace exattn {
@@ -296,6 +298,33 @@ bool dispatch_split(int GB, dim3 grid, cudaStream_t st, const void *q, const voi
 }
 
 }  // namespace
+
+// Scratch of attn_decode_paged_noalloc.  A fixed array in the module's device
+// memory: every GPU that loads this library holds it until the process exits,
+// and all no-allocation calls on a device share it.  Host code must not pass
+// the symbol itself to a kernel -- on the host it names a stand-in, not a
+// device address -- so its device address is looked up below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[64] = {};
+}  // namespace
+
+// Device address of g_noalloc_scratch on the current device; looked up once
+// per device (with that device current) on its first no-allocation call.
+attn_status_t noalloc_scratch_address(void **addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return ATTN_OK;
+}
 
 int decode_max_splits(int max_blocks) { return (max_blocks + kPagesPerSplit - 1) / kPagesPerSplit; }
 

@@ -27,4 +27,8 @@ attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void
                                   float scale, void *workspace, cudaStream_t stream,
                                   unsigned *status);
 
+// Device address of the fixed scratch array used by attn_decode_paged_noalloc
+// (ATTN_DECODE_NOALLOC_SCRATCH_BYTES bytes) on the current device.
+attn_status_t noalloc_scratch_address(void **addr);
+
 }  // namespace exattn

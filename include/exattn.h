@@ -130,6 +130,45 @@ EXATTN_API attn_status_t attn_decode_paged(const void *q, const void *k_pages, c
                                 attn_stream_t stream);
 
 /*
+ * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot
+ * allocate device memory.  The pages have no counterpart to this entry point; it
+ * exists for how the library is used, not for the method.
+ *
+ * Some callers may not call cudaMalloc at all: a plugin inside a host program
+ * that owns every byte of device memory through its own pool, or a decode loop
+ * that must never wait on the allocator (cudaMalloc and cudaFree can block until
+ * the device is idle).  They still pass q, the page pools, block_table,
+ * seq_lens, o and lse exactly as for attn_decode_paged, but no workspace: the
+ * chunk partials go to a fixed scratch array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES
+ * that lives in the library's device memory.  This call allocates nothing and
+ * frees nothing.
+ *
+ * - The scratch exists once per GPU that loads the library and stays allocated
+ *   until the process exits.
+ * - The first call on a device looks up the scratch's device address (with that
+ *   device current) and caches it; make that first call before any stream
+ *   capture.
+ * - All calls on a device share the one array and leave their partials in it.
+ *   Calls whose kernels overlap on the GPU (different streams, no ordering
+ *   between them) race on it; order them on one stream or use attn_decode_paged
+ *   with separate workspaces.  Nothing in the scratch needs to start at zero:
+ *   each call writes every partial it later reads.
+ * - A request whose workspace, as attn_decode_workspace_bytes(S, Hq, d,
+ *   max_blocks, page_size) reports it, exceeds ATTN_DECODE_NOALLOC_SCRATCH_BYTES
+ *   returns ATTN_ERR_INVALID_ARG without launching anything.  (64 sequences x
+ *   32 heads x d=128 with up to 512 pages of 16 tokens need 16.9 MB.)
+ * Results are identical to attn_decode_paged's for the same arguments.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+EXATTN_API attn_status_t attn_decode_paged_noalloc(const void *q, const void *k_pages,
+                                                   const void *v_pages,
+                                                   const int32_t *block_table,
+                                                   const int32_t *seq_lens, void *o, float *lse,
+                                                   int S, int Hq, int Hkv, int d, int page_size,
+                                                   int max_blocks, int num_pages, float scale,
+                                                   attn_stream_t stream);
+
+/*
  * attn_device_status -- read (and, if clear != 0, reset) the status word of the
  * current device.  Synchronises the device first, so call it between steps, not
  * inside stream capture.
