@@ -428,6 +428,26 @@ def run_ours(args):
     return 0
 
 
+def run_only(args):
+    """Launch one workload's kernels a few times (no flush, no JSON): for ncu captures."""
+    import exact_io_aware_101_b200 as ea
+    torch.cuda.set_device(0)
+    lib = ea.library()
+    table = {c.name: c for c in syn.MHA_SWEEP + (syn.CAUSAL, syn.GQA)}
+    if args.only == syn.DECODE.name:
+        it = Decode(syn.DECODE, lib)
+    elif args.only in table:
+        it = Prefill(table[args.only], lib)
+    else:
+        raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table) + [syn.DECODE.name]))
+    for _ in range(args.reps):
+        it.launch()
+    torch.cuda.synchronize()
+    st = ea.device_status()
+    print("ran %s x%d, device status %d" % (args.only, args.reps, st))
+    return 0 if st == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -438,7 +458,11 @@ def main():
     ap.add_argument("--skip-components", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--only", default=None, help="profile mode: run one workload --reps times")
+    ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
+    if args.only:
+        return run_only(args)
     if args.warmup < 3 and args.impl == "ours":
         print("note: at least 3 warm-up steps are required; using 3", file=sys.stderr)
         args.warmup = 3

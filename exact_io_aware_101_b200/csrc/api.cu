@@ -44,7 +44,7 @@ bool device_state(unsigned **status, bool *sm100) {
 
 bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
-bool good_scale(float s) { return isfinite(s) && s >= 0.f; }
+bool good_scale(float s) { return isfinite(s) && s > 0.f; }
 
 attn_status_t check_prefill(const void *q, const void *k, const void *v, const void *o,
                             const void *lse, int B, int Hq, int Hkv, int N, int d, float scale) {

@@ -28,9 +28,9 @@
 //    when a row's max grows by more than 8 in log2 units; O/l stays exact.
 //  * Causal: KV tiles above the diagonal are never loaded or multiplied; only
 //    diagonal tiles are masked (Concepts: causal masking; Lab 01 step 4).
-//  * Grid: one CTA per (Q-tile pair, batch*head), heaviest causal pairs first;
-//    consecutive CTAs are the query heads that share one K/V head, so GQA's K/V
-//    tiles are reused from L2.
+//  * Grid: one CTA per (Q-tile pair, batch*head).  Consecutive CTAs share K/V
+//    (same head, or the query heads of one K/V group), so re-reads hit L2;
+//    causal grids go heaviest pair first within groups of 8 heads.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -48,6 +48,10 @@ namespace {
 constexpr int BM = 128;       // query rows per Q tile
 constexpr int BN = 128;       // keys per K/V tile
 constexpr int NUM_THREADS = 384;
+constexpr int kRegsLow = 56;    // per thread, producer/MMA warpgroup
+constexpr int kRegsHigh = 224;  // per thread, softmax warpgroups
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= NUM_THREADS * 168, "register split");
+constexpr int kHeadGroup = 8;  // causal schedule: heads whose K/V share L2 at a time
 constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 128-byte swizzle column block
 
 template <int D>
@@ -102,10 +106,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: Q-tile pair and (batch, head); heaviest causal pairs first
+  // ---- work item: Q-tile pair and (batch, head).  Non-causal: head-major, so
+  // the CTAs resident at one time share a few heads' K/V in L2.  Causal: groups
+  // of kHeadGroup heads, heaviest pairs first inside each group (load balance)
+  // while a group's K/V stays in L2.
   const int BH = p.B * p.Hq;
-  const int pair = p.pairs - 1 - static_cast<int>(blockIdx.x / BH);
-  const int bh = static_cast<int>(blockIdx.x % BH);
+  int pair, bh;
+  {
+    const int lin = static_cast<int>(blockIdx.x);
+    if (!p.causal) {
+      bh = lin / p.pairs;
+      pair = lin % p.pairs;
+    } else {
+      const int grp = lin / (kHeadGroup * p.pairs);
+      const int first = grp * kHeadGroup;
+      const int hg = min(kHeadGroup, BH - first);
+      const int rr = lin - grp * kHeadGroup * p.pairs;
+      pair = p.pairs - 1 - rr / hg;
+      bh = first + rr % hg;
+    }
+  }
   const int b = bh / p.Hq;
   const int hq = bh % p.Hq;
   const int hkv = hq / (p.Hq / p.Hkv);
@@ -138,9 +158,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // Registers (set inside each role's branch): the producer/MMA warpgroup needs
+  // few, the softmax warpgroups hold a 128-column score row each.
+  // 128*kRegsLow + 256*kRegsHigh = 384*168, the block's launch budget.
 
   if (warp == 0) {
     // ================================================================ producer
+    regs_dec<kRegsLow>();
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -173,6 +197,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ================================================================== MMA
+    regs_dec<kRegsLow>();
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t ring_base = smem_u32(sRing);
@@ -251,8 +276,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, p.status);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();  // warps 2-3: idle members of the first warpgroup
+  } else {
     // ====================================================== softmax / epilogue
+    regs_inc<kRegsHigh>();
     const int t = (warp - 4) >> 2;        // Q tile of this warpgroup
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;    // row within the Q tile
@@ -273,25 +301,61 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       int limit = min(BN, p.N - j * BN);
       if (p.causal && j == qtile) limit = min(limit, r + 1);
-      uint32_t sv[32];
-      float mx = -INFINITY;
+      // The whole 128-column score row of this thread, in one TMEM load.
+      uint32_t sv[128];
+      tmem_ld128(s_addr, sv);
+      tmem_ld_wait128(sv);
+      // Only diagonal and last tiles carry masked columns; elsewhere the warp
+      // takes the branch-free path.
+      const bool masked = !__all_sync(0xffffffffu, limit == BN);
+      if (masked) {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        tmem_ld32(s_addr + cc * 32, sv);
-        tmem_ld_wait(sv);
+        for (int i = 0; i < 128; ++i)
+          if (i >= limit) sv[i] = 0xff800000u;  // -inf
+      }
+      float mx;
+      {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float s = __uint_as_float(sv[i]);
-          mx = fmaxf(mx, (cc * 32 + i < limit) ? s : -INFINITY);
+        for (int i = 0; i < 128; i += 8) {
+          m0 = fmax3(m0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          m1 = fmax3(m1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
+          m2 = fmax3(m2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
+          m3 = fmax3(m3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
         }
+        mx = fmax3(m0, m1, fmaxf(m2, m3));
       }
       const float m_new = fmaxf(m, mx * c);
       const bool resc = m_new > m + 8.0f;
       const float alpha = resc ? ex2(m - m_new) : 1.0f;
       if (resc) m = m_new;
       l *= alpha;
+      // P = 2^(s*c - m): one packed FMA per pair, rounded to bf16 and written
+      // over the (already read) S columns; the row sum stays in fp32.
+      const float2 c2 = make_float2(c, c);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 sum_a = make_float2(0.f, 0.f), sum_b = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const int col = cc * 32 + i;
+          const float2 x0 = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), c2, nm2);
+          const float2 x1 = fma2(make_float2(__uint_as_float(sv[col + 2]), __uint_as_float(sv[col + 3])), c2, nm2);
+          const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+          const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+          sum_a = add2(sum_a, p0);
+          sum_b = add2(sum_b, p1);
+          pk[i >> 1] = pack_bf16x2(p0.x, p0.y);
+          pk[(i >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+        }
+        tmem_st16(s_addr + cc * 16, pk);
+      }
+      l += (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
       if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        // O is stable here: S(j) completing implies PV(j-1) completed.
+        // Lazy rescale of O (rare once the max settles).  O is stable here:
+        // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t ov[32];
@@ -301,22 +365,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
           tmem_st32(o_addr + cc * 32, ov);
         }
-      }
-      const float neg_m = -m;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        tmem_ld32(s_addr + cc * 32, sv);
-        tmem_ld_wait(sv);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int col = cc * 32 + i;
-          const float p0 = (col < limit) ? ex2(fmaf(__uint_as_float(sv[i]), c, neg_m)) : 0.f;
-          const float p1 = (col + 1 < limit) ? ex2(fmaf(__uint_as_float(sv[i + 1]), c, neg_m)) : 0.f;
-          l += p0 + p1;
-          pk[i >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(s_addr + cc * 16, pk);  // P columns [16cc, 16cc+16) <- S columns already read
       }
       tmem_st_wait();
       tc_fence_before();

@@ -76,7 +76,7 @@ typedef enum {
  *   q    [B, Hq,  N, d] bf16        k, v [B, Hkv, N, d] bf16
  *   o    [B, Hq,  N, d] bf16 (out)  lse  [B, Hq, N] float32 (out)
  *   d in {64, 128}; N >= 1; B, Hq, Hkv >= 1; Hq % Hkv == 0;
- *   scale finite and >= 0 (the workloads use 1/sqrt(d)).
+ *   scale finite and > 0 (the workloads use 1/sqrt(d)).
  * Accumulation is float32; O is rounded to nearest-even bf16.
  * Returns ATTN_ERR_UNSUPPORTED if the current device is not sm_100.
  */

@@ -74,7 +74,7 @@ def fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, Hq=2, Hkv=1, N=16, d=128, scale=0.1
     (dict(q=None), INVALID), (dict(o=A + 8), INVALID), (dict(lse=A + 2), INVALID),
     (dict(B=0), INVALID), (dict(N=0), INVALID), (dict(Hq=3, Hkv=2), INVALID),
     (dict(Hkv=0), INVALID), (dict(scale=float("nan")), INVALID), (dict(scale=-1.0), INVALID),
-    (dict(scale=float("inf")), INVALID), (dict(d=96), UNSUPPORTED), (dict(d=256), UNSUPPORTED),
+    (dict(scale=float("inf")), INVALID), (dict(scale=0.0), INVALID), (dict(d=96), UNSUPPORTED), (dict(d=256), UNSUPPORTED),
 ])
 def test_prefill_argument_checks(lib, kw, code):
     assert fwd(lib, **kw) == code
