@@ -25,6 +25,7 @@
 
 #include <mutex>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace exattn {
@@ -33,14 +34,6 @@ namespace {
 constexpr int kPageSize = 16;
 constexpr int kPagesPerSplit = 32;  // 512 tokens per chunk
 constexpr int kWarps = 4;
-
-__device__ __forceinline__ uint4 ld_stream(const void *p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -57,10 +50,21 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+constexpr int kStages = 8;  // shared-memory ring of (K page, V page) slices
+
+template <int D>
+constexpr int stage_bytes() { return 2 * kPageSize * D * 2; }
+
 // Workspace: o_part [S][Hq][nsplit][D] f32 (normalised), l2_part [S][Hq][nsplit]
 // f32 (log2-sum-exp of scale*log2(e)*scores over the chunk; NaN marks a bad sequence).
+//
+// Warps 0..kWarps-1 compute; warp kWarps is the producer: its lane 0 copies the
+// visible rows of each page's K and V slices into a kStages-deep shared-memory
+// ring with bulk async copies, so the bytes in flight do not depend on how many
+// registers the compute warps hold.  Page i of the chunk goes to stage
+// i % kStages and is consumed by warp i % kWarps.
 template <int D, int GB>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
     decode_split_kernel(const __nv_bfloat16 *__restrict__ q,
                         const __nv_bfloat16 *__restrict__ k_pages,
                         const __nv_bfloat16 *__restrict__ v_pages,
@@ -68,139 +72,225 @@ __global__ void __launch_bounds__(kWarps * 32)
                         float *__restrict__ o_part, float *__restrict__ l2_part, int Hq, int Hkv,
                         int max_blocks, int num_pages, float scale_log2, int nsplit,
                         int head_chunks, unsigned *status) {
-  constexpr int LPT = D / 8;          // lanes per token row (8 bf16 = 16 B each)
-  constexpr int TPI = 32 / LPT;       // token rows per warp-wide load
-  constexpr int IT = kPageSize / TPI; // loads per page per lane
+  constexpr int LPT = D / 8;           // lanes per token row (8 bf16 = 16 B each)
+  constexpr int TPI = 32 / LPT;        // token rows per warp-wide access
+  constexpr int IT = kPageSize / TPI;  // accesses per page per lane
+  constexpr int SLICE = kPageSize * D; // elements of one page's K (or V) slice
+  static_assert(kPagesPerSplit <= 32, "one block-table entry per producer lane");
   const int split = blockIdx.x;
   const int g = blockIdx.y / head_chunks;
   const int h0 = g * (Hq / Hkv) + (blockIdx.y % head_chunks) * GB;
   const int s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane / LPT;         // which token row of a load this lane holds
-  const int dc = lane % LPT;          // which 8-column slice
+  const int sub = lane / LPT;          // token row of an access held by this lane
+  const int dc = lane % LPT;           // 8-column slice held by this lane
 
   const int len = seq_lens[s];
-  const int cap = max_blocks * kPageSize;
-  const bool bad_len = len < 0 || len > cap;
+  const bool bad_len = len < 0 || len > max_blocks * kPageSize;
   const int page_begin = split * kPagesPerSplit;
   const int n_pages = bad_len ? 0 : (len + kPageSize - 1) / kPageSize;
   if (!bad_len && page_begin >= n_pages) return;  // chunk past the end: nothing to do
-  const int page_end = min(n_pages, page_begin + kPagesPerSplit);
+  const int npg = bad_len ? 0 : min(n_pages, page_begin + kPagesPerSplit) - page_begin;
 
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[kStages], empty[kStages];
+  __shared__ int stage_ntok[kStages];
+  __shared__ int sm_pid[kPagesPerSplit];
   __shared__ float sm_m[kWarps][GB], sm_l[kWarps][GB];
   __shared__ float sm_acc[kWarps][GB][D];
-  __shared__ int sm_bad;
-  if (threadIdx.x == 0) sm_bad = bad_len ? 1 : 0;
+  __shared__ int sm_bad, sm_abort;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    sm_bad = bad_len ? 1 : 0;
+    sm_abort = 0;
+    fence_mbar_init();
+  }
   __syncthreads();
 
-  // Query slice of this lane, pre-multiplied by scale*log2(e).
-  float qf[GB][8];
-#pragma unroll
-  for (int hh = 0; hh < GB; ++hh) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(q + (static_cast<size_t>(s) * Hq + h0 + hh) * D + dc * 8);
-    bf16x8_to_f32(u, qf[hh]);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qf[hh][e] *= scale_log2;
-  }
-
-  float m[GB], l[GB], acc[GB][8];
-#pragma unroll
-  for (int hh = 0; hh < GB; ++hh) {
-    m[hh] = -INFINITY;
-    l[hh] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
-  }
-
-  for (int pg = page_begin + warp; !bad_len && pg < page_end; pg += kWarps) {
-    const int pid = block_table[static_cast<size_t>(s) * max_blocks + pg];
-    if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
-      if (lane == 0) sm_bad = 1;
-      continue;
-    }
-    const size_t base = (static_cast<size_t>(pid) * Hkv + g) * kPageSize * D;
-    uint4 kr[IT], vr[IT];
-#pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      const int tok = pg * kPageSize + it * TPI + sub;
-      const size_t off = base + static_cast<size_t>(it * TPI + sub) * D + dc * 8;
-      if (tok < len) {
-        kr[it] = ld_stream(k_pages + off);
-        vr[it] = ld_stream(v_pages + off);
-      } else {
-        kr[it] = make_uint4(0, 0, 0, 0);
-        vr[it] = make_uint4(0, 0, 0, 0);
+  if (warp == kWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane < npg) sm_pid[lane] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + lane];
+    __syncwarp();
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < npg; ++i) {
+        const int st = i % kStages;
+        if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1, &sm_abort, status)) break;
+        const int pid = sm_pid[i];
+        const int ntok = min(kPageSize, len - (page_begin + i) * kPageSize);
+        if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
+          sm_bad = 1;
+          stage_ntok[st] = 0;
+          mbar_arrive(&full[st]);
+        } else {
+          stage_ntok[st] = ntok;
+          const uint32_t bytes = static_cast<uint32_t>(ntok * D * 2);
+          const size_t base = (static_cast<size_t>(pid) * Hkv + g) * SLICE;
+          uint8_t *dst = ring + st * stage_bytes<D>();
+          mbar_arrive_expect_tx(&full[st], 2 * bytes);
+          bulk_load(dst, k_pages + base, bytes, &full[st]);
+          bulk_load(dst + SLICE * 2, v_pages + base, bytes, &full[st]);
+        }
+        issued = i + 1;
       }
+      // Let every copy land before the CTA (and its shared memory) goes away.
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        mbar_wait_drain(&full[i % kStages], (i / kStages) & 1, status);
     }
-    // Scores (log2 units) of this lane's token rows for every head of the group.
-    float sc[GB][IT];
-#pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      float kf[8];
-      bf16x8_to_f32(kr[it], kf);
-      const bool vis = pg * kPageSize + it * TPI + sub < len;
-#pragma unroll
-      for (int hh = 0; hh < GB; ++hh) {
-        float part = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) part = fmaf(qf[hh][e], kf[e], part);
-#pragma unroll
-        for (int o = LPT / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        sc[hh][it] = vis ? part : -INFINITY;
-      }
-    }
+  } else {
+    // ------------------------------------------------------------ compute
+    // Query slice of this lane (8 columns, every head of the group) as float2
+    // pairs, pre-multiplied by scale*log2(e).
+    float2 q2[GB][4];
 #pragma unroll
     for (int hh = 0; hh < GB; ++hh) {
-      float mx = sc[hh][0];
+      const uint4 u = *reinterpret_cast<const uint4 *>(
+          q + (static_cast<size_t>(s) * Hq + h0 + hh) * D + dc * 8);
+      float f[8];
+      bf16x8_to_f32(u, f);
 #pragma unroll
-      for (int it = 1; it < IT; ++it) mx = fmaxf(mx, sc[hh][it]);
-#pragma unroll
-      for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_new = fmaxf(m[hh], mx);  // finite: every page holds a visible token
-      const float alpha = ex2f(m[hh] - m_new);
-      float psum = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[hh][e] *= alpha;
-#pragma unroll
-      for (int it = 0; it < IT; ++it) {
-        const float pw = ex2f(sc[hh][it] - m_new);  // 0 for masked rows
-        psum += pw;
-        float vf[8];
-        bf16x8_to_f32(vr[it], vf);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(pw, vf[e], acc[hh][e]);
-      }
-      l[hh] = l[hh] * alpha + psum;
-      m[hh] = m_new;
+      for (int e = 0; e < 4; ++e) q2[hh][e] = make_float2(f[2 * e] * scale_log2, f[2 * e + 1] * scale_log2);
     }
-  }
-
-  // Merge the token-row groups of the warp (lanes that share a column slice).
+    // After the transposed reduction below, this lane holds the score of one head
+    // of the group: my_head; the lane holding head hh in a row group is
+    // hh * (LPT / GB) within it.
+    int my_head = 0;
+    {
+      int n = GB;
 #pragma unroll
-  for (int hh = 0; hh < GB; ++hh) {
+      for (int o = LPT / 2; o > 0; o >>= 1) {
+        if (n > 1) {
+          if (lane & o) my_head += n / 2;
+          n /= 2;
+        }
+      }
+    }
+    float m = -INFINITY, l = 0.f;  // running max / sum of my_head, over this lane's rows
+    float2 acc[GB][4];             // every head, this lane's 8 columns, this lane's rows
+#pragma unroll
+    for (int hh = 0; hh < GB; ++hh)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[hh][e] = make_float2(0.f, 0.f);
+
+    for (int i = warp; i < npg; i += kWarps) {
+      const int st = i % kStages;
+      bool ok = mbar_wait(&full[st], (i / kStages) & 1, &sm_abort, status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int ntok = stage_ntok[st];
+      if (ntok > 0) {
+        const uint8_t *ks = ring + st * stage_bytes<D>();
+        const uint8_t *vs = ks + SLICE * 2;
+        // q . k for this lane's rows: partial dot over 8 columns per head, then a
+        // butterfly over the LPT lanes of the row that also transposes, so each
+        // lane ends with one head's full score (log2 units).
+        float sc[IT];
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+          const int row = it * TPI + sub;
+          float kf[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4 *>(ks + (row * D + dc * 8) * 2), kf);
+          float v[GB];
+#pragma unroll
+          for (int hh = 0; hh < GB; ++hh) {
+            float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) a = fma2(q2[hh][e], make_float2(kf[2 * e], kf[2 * e + 1]), a);
+            v[hh] = a.x + a.y;
+          }
+          int n = GB;
+#pragma unroll
+          for (int o = LPT / 2; o > 0; o >>= 1) {
+            if (n > 1) {
+              const bool up = (lane & o) != 0;
+#pragma unroll
+              for (int x = 0; x < n / 2; ++x) {
+                const float send = up ? v[x] : v[x + n / 2];
+                const float keep = up ? v[x + n / 2] : v[x];
+                v[x] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+              }
+              n /= 2;
+            } else {
+              v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+            }
+          }
+          sc[it] = row < ntok ? v[0] : -INFINITY;
+        }
+        // Online softmax for my_head over this page (all rows: reduce over the
+        // row groups of the warp).
+        float mx = sc[0];
+#pragma unroll
+        for (int it = 1; it < IT; ++it) mx = fmaxf(mx, sc[it]);
+#pragma unroll
+        for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_new = fmaxf(m, mx);  // finite: row 0 of a page is always visible
+        const float alpha = ex2f(m - m_new);
+        m = m_new;
+        l *= alpha;
+#pragma unroll
+        for (int hh = 0; hh < GB; ++hh) {
+          const float a = __shfl_sync(0xffffffffu, alpha, hh * (LPT / GB));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[hh][e] = make_float2(acc[hh][e].x * a, acc[hh][e].y * a);
+        }
+        // P V: each lane needs every head's weight for its rows.
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+          const int row = it * TPI + sub;
+          const float pw = ex2f(sc[it] - m);  // 0 for rows past the sequence end
+          l += pw;
+          float vf[8];
+          // Rows past ntok were not copied this time: read zeros, never stale data.
+          const uint4 vraw = row < ntok ? *reinterpret_cast<const uint4 *>(vs + (row * D + dc * 8) * 2)
+                                        : make_uint4(0, 0, 0, 0);
+          bf16x8_to_f32(vraw, vf);
+#pragma unroll
+          for (int hh = 0; hh < GB; ++hh) {
+            const float ph = __shfl_sync(0xffffffffu, pw, sub * LPT + hh * (LPT / GB));
+            const float2 p2 = make_float2(ph, ph);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[hh][e] = fma2(p2, make_float2(vf[2 * e], vf[2 * e + 1]), acc[hh][e]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
+    }
+
+    // Merge the row groups of the warp: acc over lanes sharing a column slice,
+    // l over lanes sharing a head.
 #pragma unroll
     for (int o = LPT; o < 32; o <<= 1) {
-      l[hh] += __shfl_xor_sync(0xffffffffu, l[hh], o);
+      l += __shfl_xor_sync(0xffffffffu, l, o);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[hh][e] += __shfl_xor_sync(0xffffffffu, acc[hh][e], o);
+      for (int hh = 0; hh < GB; ++hh)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[hh][e].x += __shfl_xor_sync(0xffffffffu, acc[hh][e].x, o);
+          acc[hh][e].y += __shfl_xor_sync(0xffffffffu, acc[hh][e].y, o);
+        }
     }
-  }
-  if (lane < LPT) {
+    if (lane < LPT) {
 #pragma unroll
-    for (int hh = 0; hh < GB; ++hh) {
+      for (int hh = 0; hh < GB; ++hh)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sm_acc[warp][hh][dc * 8 + e] = acc[hh][e];
-      if (lane == 0) {
-        sm_m[warp][hh] = m[hh];
-        sm_l[warp][hh] = l[hh];
+        for (int e = 0; e < 4; ++e) {
+          sm_acc[warp][hh][dc * 8 + 2 * e] = acc[hh][e].x;
+          sm_acc[warp][hh][dc * 8 + 2 * e + 1] = acc[hh][e].y;
+        }
+      if (lane % (LPT / GB) == 0) {
+        sm_m[warp][my_head] = m;
+        sm_l[warp][my_head] = l;
       }
     }
   }
   __syncthreads();
 
   // Merge the warps and write this chunk's normalised partial per head.
-  const bool bad = sm_bad != 0;
-  if (bad && threadIdx.x == 0) atomicOr(status, ATTN_DEV_BAD_PAGE);
+  const bool bad = sm_bad != 0 || sm_abort != 0;
+  if (bad && threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
   for (int idx = threadIdx.x; idx < GB * D; idx += blockDim.x) {
     const int hh = idx / D, c = idx % D;
     float M = -INFINITY;
@@ -277,7 +367,13 @@ template <int D, int GB>
 void launch_split(dim3 grid, cudaStream_t st, const void *q, const void *kp, const void *vp,
                   const int *bt, const int *sl, float *op, float *lp, int Hq, int Hkv, int maxb,
                   int npages, float sl2, int nsplit, int hc, unsigned *status) {
-  decode_split_kernel<D, GB><<<grid, kWarps * 32, 0, st>>>(
+  constexpr int kSmem = kStages * stage_bytes<D>();
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(decode_split_kernel<D, GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kSmem);
+  });
+  decode_split_kernel<D, GB><<<grid, (kWarps + 1) * 32, kSmem, st>>>(
       static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kp),
       static_cast<const __nv_bfloat16 *>(vp), bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit,
       hc, status);
