@@ -77,14 +77,17 @@ def test_bf16_deterministic_and_gqa_equals_repeated_heads():
     assert torch.equal(o1, o3) and torch.equal(l1, l3)
 
 
-def test_bf16_large_scores_stay_finite():
-    # Scores of several hundred: only the running-max shift keeps exp finite.
-    B, H, N, d = 1, 2, 300, 64
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_large_scores_stay_finite(causal, d):
+    # Scores of several hundred: only the running-max shift keeps exp finite, and
+    # exponents far below -126 reach the polynomial exp2 of unmasked tiles.
+    B, H, N = 1, 2, 300
     q, k, v = syn.random_qkv(B, H, H, N, d, seed=11)
     q = (q.float() * 8).to(torch.bfloat16)
     o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
-                                    scale=1.0, causal=True)
-    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=1.0)
+                                    scale=1.0, causal=causal)
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=1.0)
     torch.cuda.synchronize()
     assert np.abs(l_ref).max() > 100
     # L is large in magnitude here; hold it to the same absolute bound relative to |L|.
