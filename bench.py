@@ -378,13 +378,19 @@ def run_ours(args):
 
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    traffic = profiled_traffic("prefill_bf16_mha_sweep.md", "prefill_sm100.cu")
-    roofline = {"bound": "tensor", "achieved": sweep_flops * args.steps / kernel_s / 1e12,
-                "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": sweep_flops * args.steps / kernel_s / 1e12 / peak_tf,
-                "traffic": traffic, "peak_source": peak_kind + " (bf16_tflops, burst)",
-                "kernel": "prefill_bf16_kernel<128>",
-                "per_launch": "FLOP-weighted over the 5 sweep launches"}
+    # Roofline of the dominant launch: the N=8192 prefill, about two thirds of a step.
+    big = max(range(len(sweep)), key=lambda i: sweep[i].cfg.flops)
+    big_s = sum(times[big]) / len(times[big]) / 1e3
+    big_tf = sweep[big].cfg.flops / big_s / 1e12
+    roofline = {"bound": "tensor", "achieved": big_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": big_tf / peak_tf,
+                "traffic": profiled_traffic("prefill_bf16_mha_n8192.md", "prefill_sm100.cu"),
+                "peak_source": peak_kind + " bf16_tflops (burst)",
+                "kernel": "prefill_bf16_kernel<128>, %s launch (%.0f%% of the step)"
+                          % (sweep[big].cfg.name, 100.0 * sum(times[big]) / sum(sum(t) for t in times)),
+                "algorithmic": "4*B*H*N^2*d = %.4g FLOP per launch; %d bytes (Q,K,V read, O,L written)"
+                               % (sweep[big].cfg.flops, sweep[big].cfg.bytes),
+                "sweep_achieved": sweep_flops * args.steps / kernel_s / 1e12}
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -418,7 +424,8 @@ def run_ours(args):
                                      "algorithmic_bytes": dec.bytes,
                                      "peak_gbs": peak_hbm,
                                      "traffic": profiled_traffic("decode_paged_gqa.md",
-                                                                 "decode_paged.cu")}
+                                                                 "decode_paged.cu"),
+                                     "bound": "hbm"}
         if ea.device_status() != 0:
             raise RuntimeError("device status word set in the component runs")
         line["components"] = comps
