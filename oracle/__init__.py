@@ -47,10 +47,10 @@ def _load():
         u16p = ctypes.POINTER(ctypes.c_uint16)
         ci, cd = ctypes.c_int, ctypes.c_double
         lib.oracle_attn.argtypes = [f32p, f32p, f32p, f64p, f64p,
-                                    ci, ci, ci, ci, ci, ci, cd, ci, ci]
+                                    ci, ci, ci, ci, ci, ci, cd, ci, ci, f64p, ci]
         lib.oracle_attn.restype = ci
         lib.oracle_attn_rows.argtypes = [f32p, f32p, f32p, f64p, f64p,
-                                         ci, ci, ci, ci, ci, ci, cd, ci,
+                                         ci, ci, ci, ci, ci, ci, cd, ci, ci, f64p,
                                          i64p, ci, ci]
         lib.oracle_attn_rows.restype = ci
         lib.oracle_decode_paged.argtypes = [f32p, u16p, u16p, i32p, i32p, f64p, f64p,
@@ -75,28 +75,45 @@ def _f32(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
 
 
-def attention(q, k, v, scale: float, causal: bool = False, nthreads: int | None = None):
+def _slopes(slopes, Hq):
+    if slopes is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(slopes, dtype=np.float64).reshape(-1))
+    if a.size != Hq:
+        raise ValueError("need one ALiBi slope per query head")
+    return a
+
+
+def _sp(a):
+    return None if a is None else _ptr(a, ctypes.c_double)
+
+
+def attention(q, k, v, scale: float, causal: bool = False, nthreads: int | None = None,
+              window: int = 0, alibi_slopes=None):
     """Standard attention in fp64.  q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (float32 values).
 
     Returns (O [B,Hq,Nq,d] float64, L [B,Hq,Nq] float64).  Causal: key j is
-    visible to query i iff j <= i.
+    visible to query i iff j <= i.  window W > 0 keeps keys with i - j < W;
+    alibi_slopes (one per query head) add slope_h * (j - i) to the scores.
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     B, Hq, Nq, d = q.shape
     _, Hkv, Nk, _ = k.shape
     o = np.zeros((B, Hq, Nq, d), dtype=np.float64)
     lse = np.zeros((B, Hq, Nq), dtype=np.float64)
+    sl = _slopes(alibi_slopes, Hq)
     rc = _load().oracle_attn(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
                              _ptr(v, ctypes.c_float), _ptr(o, ctypes.c_double),
                              _ptr(lse, ctypes.c_double), B, Hq, Hkv, Nq, Nk, d,
-                             float(scale), int(bool(causal)),
+                             float(scale), int(bool(causal)), int(window), _sp(sl),
                              int(nthreads or max_threads()))
     if rc != 0:
         raise ValueError("oracle_attn failed with code %d" % rc)
     return o, lse
 
 
-def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | None = None):
+def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | None = None,
+                   window: int = 0, alibi_slopes=None):
     """The same definition for selected rows; rows[r] = (b*Hq + h)*Nq + i."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     B, Hq, Nq, d = q.shape
@@ -104,10 +121,11 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | No
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     o = np.zeros((rows.size, d), dtype=np.float64)
     lse = np.zeros((rows.size,), dtype=np.float64)
+    sl = _slopes(alibi_slopes, Hq)
     rc = _load().oracle_attn_rows(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
                                   _ptr(v, ctypes.c_float), _ptr(o, ctypes.c_double),
                                   _ptr(lse, ctypes.c_double), B, Hq, Hkv, Nq, Nk, d,
-                                  float(scale), int(bool(causal)),
+                                  float(scale), int(bool(causal)), int(window), _sp(sl),
                                   _ptr(rows, ctypes.c_int64), int(rows.size),
                                   int(nthreads or max_threads()))
     if rc != 0:

@@ -16,8 +16,14 @@
  *   For each batch b and query head h, with key/value head g = h / (Hq/Hkv)
  *   (grouped-query sharing, screna.ai MHA/MQA/GQA answer: heads are grouped and
  *   each group shares one K and V; contiguous groups):
- *     s_ij = scale * sum_c q[b,h,i,c] * k[b,g,j,c]      for j in V_i
- *     V_i  = { j : j <= i } when causal (Lab 01 step 4), else { 0 .. Nk-1 }
+ *     s_ij = scale * sum_c q[b,h,i,c] * k[b,g,j,c] + a_h * (j - i)   for j in V_i
+ *     V_i  = { j : j <= i } when causal (Lab 01 step 4), else { 0 .. Nk-1 },
+ *            further limited to { j : i - j < W } by a sliding window W > 0
+ *   The last two are the Lab 01 "Extensions" (sliding-window attention as in
+ *   Mistral, ALiBi bias), which the page only names; read plainly, a window of
+ *   W keeps the W most recent keys (i-W < j <= i) and ALiBi adds a per-head
+ *   linear bias a_h * (j - i) (slope a_h >= 0 given by the caller) to the
+ *   scaled score.  a_h = 0 and W = 0 give plain attention.
  *     m_i  = max_{j in V_i} s_ij
  *     l_i  = sum_{j in V_i} exp(s_ij - m_i)
  *     O_i  = sum_{j in V_i} exp(s_ij - m_i) / l_i * v[b,g,j,:]
@@ -81,16 +87,27 @@ static int check_dims(int B, int Hq, int Hkv, int Nq, int Nk, int d)
     return 0;
 }
 
+/* Visible key range [*lo, *hi) of query i. */
+static void visible_range(int i, int Nk, int causal, int window, int *lo, int *hi)
+{
+    *hi = causal ? ((i + 1 < Nk) ? i + 1 : Nk) : Nk;
+    *lo = (window > 0 && i - window + 1 > 0) ? i - window + 1 : 0;
+    if (*lo > *hi) *lo = *hi;
+}
+
 /* Full evaluation: q [B,Hq,Nq,d], k,v [B,Hkv,Nk,d] (float), o [B,Hq,Nq,d],
- * lse [B,Hq,Nq] (double).  Causal means key j is visible to query i iff j <= i. */
+ * lse [B,Hq,Nq] (double).  Causal means key j is visible to query i iff j <= i;
+ * window W > 0 additionally requires i - j < W; slopes (Hq values, or NULL)
+ * add the ALiBi bias slopes[h] * (j - i). */
 int oracle_attn(const float *q, const float *k, const float *v,
                 double *o, double *lse,
                 int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                double scale, int causal, int nthreads)
+                double scale, int causal, int window, const double *slopes,
+                int nthreads)
 {
     int b, h, G;
     double *S, *Kd, *Vd, *Qd;
-    if (check_dims(B, Hq, Hkv, Nq, Nk, d)) return -1;
+    if (check_dims(B, Hq, Hkv, Nq, Nk, d) || window < 0) return -1;
     if (!q || !k || !v || !o || !lse) return -1;
     G = Hq / Hkv;
     if (nthreads <= 0) nthreads = 1;
@@ -112,7 +129,7 @@ int oracle_attn(const float *q, const float *k, const float *v,
             for (i = 0; i < (long)Nq * d; ++i) Qd[i] = (double)qh[i];
             for (i = 0; i < (long)Nk * d; ++i) { Kd[i] = (double)kh[i]; Vd[i] = (double)vh[i]; }
 
-            /* S = scale * Q K^T, the whole Nq x Nk matrix of this head. */
+            /* S = scale * Q K^T (+ ALiBi bias), the whole Nq x Nk matrix of this head. */
             #pragma omp parallel for num_threads(nthreads) schedule(static)
             for (i = 0; i < Nq; ++i) {
                 int j, c;
@@ -120,14 +137,15 @@ int oracle_attn(const float *q, const float *k, const float *v,
                     double acc = 0.0;
                     for (c = 0; c < d; ++c) acc += Qd[(size_t)i * d + c] * Kd[(size_t)j * d + c];
                     S[(size_t)i * Nk + j] = scale * acc;
+                    if (slopes) S[(size_t)i * Nk + j] += slopes[h] * (double)(j - i);
                 }
             }
             /* Row-wise softmax over the visible keys, then P V and L. */
             #pragma omp parallel for num_threads(nthreads) schedule(static)
             for (i = 0; i < Nq; ++i) {
-                int n = Nk;
-                if (causal) n = (i + 1 < Nk) ? (int)(i + 1) : Nk;
-                softmax_row_times_v(S + (size_t)i * Nk, n, Vd, d,
+                int lo, hi;
+                visible_range((int)i, Nk, causal, window, &lo, &hi);
+                softmax_row_times_v(S + (size_t)i * Nk + lo, hi - lo, Vd + (size_t)lo * d, d,
                                     oh + (size_t)i * d, lh + i);
             }
         }
@@ -141,11 +159,11 @@ int oracle_attn(const float *q, const float *k, const float *v,
 int oracle_attn_rows(const float *q, const float *k, const float *v,
                      double *o_rows, double *lse_rows,
                      int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                     double scale, int causal,
+                     double scale, int causal, int window, const double *slopes,
                      const int64_t *rows, int nrows, int nthreads)
 {
     int G, r, bad = 0;
-    if (check_dims(B, Hq, Hkv, Nq, Nk, d)) return -1;
+    if (check_dims(B, Hq, Hkv, Nq, Nk, d) || window < 0) return -1;
     if (!q || !k || !v || !o_rows || !lse_rows || (!rows && nrows > 0) || nrows < 0) return -1;
     for (r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq * Nq) return -1;
@@ -158,19 +176,22 @@ int oracle_attn_rows(const float *q, const float *k, const float *v,
         int i = (int)(id % Nq);
         int bh = (int)(id / Nq);
         int h = bh % Hq, b = bh / Hq, g = h / G;
-        int n = causal ? ((i + 1 < Nk) ? i + 1 : Nk) : Nk;
+        int lo, hi, n;
         const float *qi = q + (((size_t)b * Hq + h) * Nq + i) * (size_t)d;
         const float *kh = k + ((size_t)b * Hkv + g) * (size_t)Nk * d;
         const float *vh = v + ((size_t)b * Hkv + g) * (size_t)Nk * d;
-        double *s = (double *)malloc(sizeof(double) * ((size_t)n + 1));
-        double *vd = (double *)malloc(sizeof(double) * ((size_t)n * d + 1));
+        double *s, *vd;
         int j, c;
+        visible_range(i, Nk, causal, window, &lo, &hi);
+        n = hi - lo;
+        s = (double *)malloc(sizeof(double) * ((size_t)n + 1));
+        vd = (double *)malloc(sizeof(double) * ((size_t)n * d + 1));
         if (!s || !vd) { free(s); free(vd); bad = 1; continue; }
-        for (j = 0; j < n; ++j) {
+        for (j = lo; j < hi; ++j) {
             double acc = 0.0;
             for (c = 0; c < d; ++c) acc += (double)qi[c] * (double)kh[(size_t)j * d + c];
-            s[j] = scale * acc;
-            for (c = 0; c < d; ++c) vd[(size_t)j * d + c] = (double)vh[(size_t)j * d + c];
+            s[j - lo] = scale * acc + (slopes ? slopes[h] * (double)(j - i) : 0.0);
+            for (c = 0; c < d; ++c) vd[(size_t)(j - lo) * d + c] = (double)vh[(size_t)j * d + c];
         }
         softmax_row_times_v(s, n, vd, d, o_rows + (size_t)r * d, lse_rows + r);
         free(s); free(vd);

@@ -152,7 +152,7 @@ def test_golden_decode(case):
 
 # ------------------------------------------------------ decimal brute force
 
-def _brute_decimal(q, k, v, scale, causal, G):
+def _brute_decimal(q, k, v, scale, causal, G, window=0, slopes=None):
     """Per-element evaluation in 50-digit decimals: p_ij = e^{s_ij} / sum_j e^{s_ij}."""
     ctx = decimal.Context(prec=50)
     D = lambda x: ctx.create_decimal_from_float(float(x))
@@ -165,9 +165,13 @@ def _brute_decimal(q, k, v, scale, causal, G):
             g = h // G
             for i in range(N):
                 js = range(i + 1) if causal else range(k.shape[2])
+                if window:
+                    js = [j for j in js if i - j < window]
                 e = {}
                 for j in js:
                     s = ctx.multiply(sc, sum((ctx.multiply(D(q[b, h, i, c]), D(k[b, g, j, c])) for c in range(d)), decimal.Decimal(0)))
+                    if slopes is not None:
+                        s = s + ctx.multiply(D(slopes[h]), decimal.Decimal(j - i))
                     e[j] = ctx.exp(s)
                 tot = sum(e.values(), decimal.Decimal(0))
                 for c in range(d):
@@ -187,6 +191,89 @@ def test_decimal_brute_force(N, d, Hq, Hkv, causal):
     ob, lb = _brute_decimal(q, k, v, 0.6, causal, Hq // Hkv)
     np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, lb, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window,use_alibi", [(1, False), (2, True), (3, False), (0, True)])
+def test_decimal_brute_force_window_alibi(window, use_alibi):
+    rng = np.random.default_rng(window * 10 + use_alibi)
+    Hq, Hkv, N, d = 4, 2, 7, 3
+    q, k, v = (rng.standard_normal(s).astype(np.float32) for s in
+               ((1, Hq, N, d), (1, Hkv, N, d), (1, Hkv, N, d)))
+    slopes = [0.5, 0.25, 0.125, 0.0625] if use_alibi else None
+    o, lse = oracle.attention(q, k, v, scale=0.6, causal=True, window=window, alibi_slopes=slopes)
+    ob, lb = _brute_decimal(q, k, v, 0.6, True, Hq // Hkv, window=window, slopes=slopes)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lb, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- sliding window, ALiBi
+
+def test_window_covering_everything_is_causal():
+    N = 21
+    q, k, v = rand(2, 4, N, 8), rand(2, 2, N, 8), rand(2, 2, N, 8)
+    o1, l1 = oracle.attention(q, k, v, scale=0.3, causal=True)
+    for w in (N, N + 5, 10 ** 6):
+        o2, l2 = oracle.attention(q, k, v, scale=0.3, causal=True, window=w)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+
+
+def test_window_of_one_returns_own_value():
+    q, k, v = rand(1, 3, 9, 4), rand(1, 3, 9, 4), rand(1, 3, 9, 4)
+    o, lse = oracle.attention(q, k, v, scale=0.45, causal=True, window=1)
+    np.testing.assert_allclose(o, v.astype(np.float64), rtol=0, atol=1e-15)
+    s = 0.45 * np.einsum("bhnd,bhnd->bhn", q.astype(np.float64), k.astype(np.float64))
+    np.testing.assert_allclose(lse, s, rtol=0, atol=1e-13)
+
+
+def test_window_rows_equal_attention_over_the_window():
+    N, d, W = 14, 4, 5
+    q, k, v = rand(1, 1, N, d), rand(1, 1, N, d), rand(1, 1, N, d)
+    o, lse = oracle.attention(q, k, v, scale=0.8, causal=True, window=W)
+    for i in range(N):
+        lo = max(0, i - W + 1)
+        oi, li = oracle.attention(q[:, :, i:i + 1], k[:, :, lo:i + 1], v[:, :, lo:i + 1], scale=0.8)
+        np.testing.assert_array_equal(o[0, 0, i], oi[0, 0, 0])
+        np.testing.assert_array_equal(lse[0, 0, i], li[0, 0, 0])
+
+
+def test_alibi_zero_slopes_is_plain():
+    q, k, v = rand(1, 2, 11, 8), rand(1, 2, 11, 8), rand(1, 2, 11, 8)
+    for causal in (False, True):
+        o1, l1 = oracle.attention(q, k, v, scale=0.2, causal=causal)
+        o2, l2 = oracle.attention(q, k, v, scale=0.2, causal=causal, alibi_slopes=[0.0, 0.0])
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_alibi_is_one_extra_dimension(causal):
+    # slope_h * (j - i) = (extra coordinate slope_h of q) * (extra coordinate j of
+    # k) - slope_h * i.  The last term is constant along a row, so O is that of
+    # plain attention on the augmented vectors and L is lower by slope_h * i.
+    B, Hq, Hkv, N, d = 1, 4, 2, 13, 5
+    q, k, v = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d)
+    slopes = np.array([0.5, 0.25, 0.125, 0.0625])
+    qa = np.concatenate([q, np.broadcast_to(slopes[None, :, None, None], (B, Hq, N, 1))], axis=3)
+    ka = np.concatenate([k, np.broadcast_to(np.arange(N)[None, None, :, None], (B, Hkv, N, 1))], axis=3)
+    o1, l1 = oracle.attention(q, k, v, scale=1.0, causal=causal, alibi_slopes=slopes)
+    # v must share d with q/k in the oracle: pad v with one zero column.
+    va = np.concatenate([v, np.zeros((B, Hkv, N, 1), np.float32)], axis=3)
+    o2, l2 = oracle.attention(qa.astype(np.float32), ka.astype(np.float32), va, scale=1.0, causal=causal)
+    np.testing.assert_allclose(o1, o2[..., :d], rtol=0, atol=1e-12)
+    shift = slopes[None, :, None] * np.arange(N)[None, None, :]
+    np.testing.assert_allclose(l1, l2 - shift, rtol=0, atol=1e-11)
+
+
+def test_rows_evaluator_window_alibi():
+    B, Hq, Hkv, N, d = 1, 4, 2, 40, 8
+    q, k, v = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d)
+    slopes = [0.3, 0.2, 0.1, 0.05]
+    o, lse = oracle.attention(q, k, v, scale=0.25, causal=True, window=9, alibi_slopes=slopes)
+    rows = RNG.choice(B * Hq * N, size=30, replace=False)
+    orow, lrow = oracle.attention_rows(q, k, v, 0.25, True, rows, window=9, alibi_slopes=slopes)
+    np.testing.assert_allclose(orow, o.reshape(-1, d)[rows], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lrow, lse.reshape(-1)[rows], rtol=0, atol=1e-14)
 
 
 # ------------------------------------------------------- online recurrence
@@ -352,8 +439,11 @@ MUTANTS = {
     "no_max_shift_sign": ("s[j] = exp(s[j] - m)", "s[j] = exp(m - s[j])"),
     "drop_normalisation": ("double p = s[j] / l;", "double p = s[j];"),
     "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
-    "causal_off_by_one": ("if (causal) n = (i + 1 < Nk) ? (int)(i + 1) : Nk;",
-                          "if (causal) n = (i < Nk) ? (int)(i) + (i == 0) : Nk;"),
+    "causal_off_by_one": ("*hi = causal ? ((i + 1 < Nk) ? i + 1 : Nk) : Nk;",
+                          "*hi = causal ? ((i < Nk) ? i + (i == 0) : Nk) : Nk;"),
+    "window_off_by_one": ("i - window + 1 > 0) ? i - window + 1 : 0;", "i - window > 0) ? i - window : 0;"),
+    "alibi_sign": ("S[(size_t)i * Nk + j] += slopes[h] * (double)(j - i);",
+                   "S[(size_t)i * Nk + j] += slopes[h] * (double)(i - j);"),
     "wrong_gqa_group": ("int g = h / G;\n            const float *qh", "int g = h % Hkv;\n            const float *qh"),
     "dropped_term": ("for (c = 0; c < d; ++c) acc += Qd", "for (c = 1; c < d; ++c) acc += Qd"),
     "log_base_two": ("*lse = m + log(l);", "*lse = m + log2(l);"),
@@ -379,7 +469,11 @@ def test_pins_catch_planted_mistakes(name, tmp_path):
         real_build = oracle.build
         oracle.build = lambda force=False: str(lib)
         failures = 0
-        checks = [test_single_key_returns_its_value, test_identical_keys_average_the_values,
+        checks = [test_window_of_one_returns_own_value,
+                  lambda: test_alibi_is_one_extra_dimension(True),
+                  lambda: test_decimal_brute_force_window_alibi(2, True),
+                  test_window_rows_equal_attention_over_the_window,
+                  test_single_key_returns_its_value, test_identical_keys_average_the_values,
                   lambda: test_weights_sum_to_one(True), test_causal_row_zero_sees_only_key_zero,
                   test_two_keys_logistic_weights, test_gqa_equals_mha_with_repeated_heads,
                   lambda: test_decimal_brute_force(5, 4, 2, 2, True),
