@@ -193,12 +193,21 @@ class Prefill:
         self.q, self.k, self.v = syn.prefill_inputs(cfg, device="cuda")
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(cfg.B, cfg.Hq, cfg.N, dtype=torch.float32, device="cuda")
+        self.slopes = torch.tensor(syn.alibi_slopes(cfg.Hq), dtype=torch.float32, device="cuda")
 
     def launch(self):
         c = self.cfg
-        rc = self.lib.attn_fwd(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
-                               self.o.data_ptr(), self.lse.data_ptr(), c.B, c.Hq, c.Hkv, c.N, c.d,
-                               c.scale, int(c.causal), torch.cuda.current_stream().cuda_stream)
+        if c.window or c.alibi:
+            rc = self.lib.attn_fwd_ext(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                       self.o.data_ptr(), self.lse.data_ptr(), c.B, c.Hq, c.Hkv,
+                                       c.N, c.d, c.scale, int(c.causal), c.window,
+                                       self.slopes.data_ptr() if c.alibi else None,
+                                       torch.cuda.current_stream().cuda_stream)
+        else:
+            rc = self.lib.attn_fwd(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                   self.o.data_ptr(), self.lse.data_ptr(), c.B, c.Hq, c.Hkv, c.N,
+                                   c.d, c.scale, int(c.causal),
+                                   torch.cuda.current_stream().cuda_stream)
         if rc != 0:
             raise RuntimeError("attn_fwd failed: %d" % rc)
         return 1  # kernels launched
@@ -407,7 +416,7 @@ def run_ours(args):
 
     if not args.skip_components:
         comps = {}
-        for cfg in (syn.CAUSAL, syn.GQA):
+        for cfg in (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI):
             it = Prefill(cfg, lib)
             timed_launches([it], flush, 3)
             t, _ = timed_launches([it], flush, args.component_reps)
@@ -453,7 +462,7 @@ def run_only(args):
     import exact_io_aware_101_b200 as ea
     torch.cuda.set_device(0)
     lib = ea.library()
-    table = {c.name: c for c in syn.MHA_SWEEP + (syn.CAUSAL, syn.GQA)}
+    table = {c.name: c for c in syn.MHA_SWEEP + (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI)}
     if args.only == syn.DECODE.name:
         it = Decode(syn.DECODE, lib)
     elif args.only in table:

@@ -26,7 +26,8 @@ __all__ = [
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
-EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_decode_workspace_bytes",
+EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ext", "attn_fwd_f32_ext",
+                    "attn_decode_workspace_bytes",
                     "attn_decode_paged", "attn_decode_paged_noalloc", "attn_device_status",
                     "attn_status_string", "attn_version")
 # Size of the library's fixed per-device scratch used by attn_decode_paged_noalloc.
@@ -57,6 +58,10 @@ def library() -> ctypes.CDLL:
         lib.attn_fwd.restype = ci
         lib.attn_fwd_f32.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
         lib.attn_fwd_f32.restype = ci
+        lib.attn_fwd_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
+        lib.attn_fwd_ext.restype = ci
+        lib.attn_fwd_f32_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
+        lib.attn_fwd_f32_ext.restype = ci
         lib.attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
@@ -105,7 +110,7 @@ def _raise(rc: int, what: str):
         raise AttnError(rc, what)
 
 
-def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype):
+def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype, window=0, alibi_slopes=None):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n, dtype, 4)
     B, Hq, N, d = q.shape
@@ -122,22 +127,40 @@ def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype):
     _check(lse, "lse", torch.float32, 3)
     if tuple(out.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, N):
         raise ValueError("out/lse shapes do not match q")
-    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-            B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _stream(q))
+    if window or alibi_slopes is not None:
+        slopes_ptr = None
+        if alibi_slopes is not None:
+            _check(alibi_slopes, "alibi_slopes", torch.float32, 1)
+            if alibi_slopes.numel() != Hq:
+                raise ValueError("alibi_slopes needs one value per query head")
+            slopes_ptr = alibi_slopes.data_ptr()
+        ext = getattr(library(), fn.__name__ + "_ext")
+        rc = ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                 B, Hq, Hkv, N, d, float(scale), int(bool(causal)), int(window), slopes_ptr,
+                 _stream(q))
+    else:
+        rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _stream(q))
     _raise(rc, what)
     return out, lse
 
 
-def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
-    """bf16 prefill: q [B,Hq,N,d], k/v [B,Hkv,N,d] -> (O bf16 [B,Hq,N,d], L fp32 [B,Hq,N])."""
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+             window: int = 0, alibi_slopes=None):
+    """bf16 prefill: q [B,Hq,N,d], k/v [B,Hkv,N,d] -> (O bf16 [B,Hq,N,d], L fp32 [B,Hq,N]).
+
+    window > 0 (with causal): keys with i - j >= window are masked.  alibi_slopes:
+    a CUDA float32 tensor [Hq]; slope_h * (j - i) is added to the scaled scores.
+    """
     return _prefill(library().attn_fwd, "attn_fwd", q, k, v, causal, scale, out, lse,
-                    torch.bfloat16)
+                    torch.bfloat16, window, alibi_slopes)
 
 
-def attn_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
-    """fp32 prefill with fp32 arithmetic throughout."""
+def attn_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+                 window: int = 0, alibi_slopes=None):
+    """fp32 prefill with fp32 arithmetic throughout (same options as attn_fwd)."""
     return _prefill(library().attn_fwd_f32, "attn_fwd_f32", q, k, v, causal, scale, out, lse,
-                    torch.float32)
+                    torch.float32, window, alibi_slopes)
 
 
 def decode_workspace_bytes(S: int, Hq: int, d: int, max_blocks: int, page_size: int = 16) -> int:

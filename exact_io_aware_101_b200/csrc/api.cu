@@ -65,30 +65,47 @@ using namespace exattn;
 
 extern "C" {
 
-attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
-                       int Hq, int Hkv, int N, int d, float scale, int causal,
-                       attn_stream_t stream) {
+attn_status_t attn_fwd_ext(const void *q, const void *k, const void *v, void *o, float *lse,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           int window, const float *alibi_slopes, attn_stream_t stream) {
   attn_status_t st = check_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
   if (st != ATTN_OK) return st;
+  if (window < 0 || (window > 0 && !causal) || (alibi_slopes && !aligned4(alibi_slopes)))
+    return ATTN_ERR_INVALID_ARG;
   unsigned *status = nullptr;
   bool sm100 = false;
   if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
   if (!sm100) return ATTN_ERR_UNSUPPORTED;
-  return launch_prefill_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal,
-                             reinterpret_cast<cudaStream_t>(stream), status);
+  return launch_prefill_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window,
+                             alibi_slopes, reinterpret_cast<cudaStream_t>(stream), status);
+}
+
+attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                       int Hq, int Hkv, int N, int d, float scale, int causal,
+                       attn_stream_t stream) {
+  return attn_fwd_ext(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, nullptr, stream);
+}
+
+attn_status_t attn_fwd_f32_ext(const float *q, const float *k, const float *v, float *o,
+                               float *lse, int B, int Hq, int Hkv, int N, int d, float scale,
+                               int causal, int window, const float *alibi_slopes,
+                               attn_stream_t stream) {
+  attn_status_t st = check_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
+  if (st != ATTN_OK) return st;
+  if (window < 0 || (window > 0 && !causal) || (alibi_slopes && !aligned4(alibi_slopes)))
+    return ATTN_ERR_INVALID_ARG;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_prefill_f32(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window,
+                            alibi_slopes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
                            int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                            attn_stream_t stream) {
-  attn_status_t st = check_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
-  if (st != ATTN_OK) return st;
-  unsigned *status = nullptr;
-  bool sm100 = false;
-  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
-  if (!sm100) return ATTN_ERR_UNSUPPORTED;
-  return launch_prefill_f32(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal,
-                            reinterpret_cast<cudaStream_t>(stream));
+  return attn_fwd_f32_ext(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, nullptr, stream);
 }
 
 size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_blocks, int page_size) {

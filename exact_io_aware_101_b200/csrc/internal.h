@@ -8,13 +8,16 @@
 
 namespace exattn {
 
+// window > 0: sliding window; slopes (device, one per query head) or nullptr: ALiBi.
 attn_status_t launch_prefill_bf16(const void *q, const void *k, const void *v, void *o, float *lse,
                                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-                                  cudaStream_t stream, unsigned *status);
+                                  int window, const float *slopes, cudaStream_t stream,
+                                  unsigned *status);
 
 attn_status_t launch_prefill_f32(const float *q, const float *k, const float *v, float *o,
                                  float *lse, int B, int Hq, int Hkv, int N, int d, float scale,
-                                 int causal, cudaStream_t stream);
+                                 int causal, int window, const float *slopes,
+                                 cudaStream_t stream);
 
 // Number of key chunks (pages per chunk fixed) a sequence of max_blocks pages
 // can be split into, and the workspace layout that follows from it.

@@ -4,7 +4,9 @@
 // bf16 tensor-core kernel ("Phase 08" page, Lab 01 steps 2-4 and the online
 // softmax recurrence of its talking points), in float32 arithmetic with the
 // accurate expf/logf, so that it meets the Lab 01 bar of 1e-4 against standard
-// attention.
+// attention.  It also takes the Lab 01 extensions: a sliding window (key j
+// visible only if i - j < window) and per-head ALiBi slopes (bias
+// slope * (j - i) added to the scaled score).
 //
 // A CTA owns 16 query rows of one (batch, head); each of its 4 warps keeps 4
 // rows' running max m, sum l and output accumulator (d/32 columns per lane).
@@ -38,7 +40,8 @@ template <int D>
 __global__ void __launch_bounds__(128)
     prefill_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
                        const float *__restrict__ v, float *__restrict__ o,
-                       float *__restrict__ lse, int Hq, int Hkv, int N, float scale, int causal) {
+                       float *__restrict__ lse, int Hq, int Hkv, int N, float scale, int causal,
+                       int window, const float *__restrict__ slopes) {
   constexpr int DPL = D / 32;  // output columns per lane
   __shared__ float sQ[kRows][D];
   __shared__ float sK[kKeys][D + 1];  // +1: lane j reads row j without bank conflicts
@@ -68,7 +71,9 @@ __global__ void __launch_bounds__(128)
   }
 
   const int kv_end = causal ? min(N, row0 + kRows) : N;
-  for (int kt = 0; kt < kv_end; kt += kKeys) {
+  const int kv_begin = window > 0 ? (max(0, row0 - window + 1) / kKeys) * kKeys : 0;
+  const float slope = slopes ? slopes[h] : 0.f;
+  for (int kt = kv_begin; kt < kv_end; kt += kKeys) {
     __syncthreads();
     for (int idx = threadIdx.x; idx < kKeys * D; idx += blockDim.x) {
       const int j = idx / D, c = idx % D;
@@ -85,8 +90,8 @@ __global__ void __launch_bounds__(128)
       float s = 0.f;
 #pragma unroll 8
       for (int c = 0; c < D; ++c) s = fmaf(sQ[lr][c], sK[lane][c], s);
-      s *= scale;
-      const bool vis = (j < N) && (!causal || j <= i);
+      s = s * scale + slope * static_cast<float>(j - i);
+      const bool vis = (j < N) && (!causal || j <= i) && (window <= 0 || i - j < window);
       s = vis ? s : -INFINITY;
       const float tmax = warp_max(s);
       const float m_new = fmaxf(m[rr], tmax);
@@ -121,14 +126,17 @@ __global__ void __launch_bounds__(128)
 
 attn_status_t launch_prefill_f32(const float *q, const float *k, const float *v, float *o,
                                  float *lse, int B, int Hq, int Hkv, int N, int d, float scale,
-                                 int causal, cudaStream_t stream) {
+                                 int causal, int window, const float *slopes,
+                                 cudaStream_t stream) {
   const long long bh = static_cast<long long>(B) * Hq;
   if (bh > 65535) return ATTN_ERR_UNSUPPORTED;
   dim3 grid((N + kRows - 1) / kRows, static_cast<unsigned>(bh));
   if (d == 128)
-    prefill_f32_kernel<128><<<grid, 128, 0, stream>>>(q, k, v, o, lse, Hq, Hkv, N, scale, causal);
+    prefill_f32_kernel<128><<<grid, 128, 0, stream>>>(q, k, v, o, lse, Hq, Hkv, N, scale, causal,
+                                                      window, slopes);
   else if (d == 64)
-    prefill_f32_kernel<64><<<grid, 128, 0, stream>>>(q, k, v, o, lse, Hq, Hkv, N, scale, causal);
+    prefill_f32_kernel<64><<<grid, 128, 0, stream>>>(q, k, v, o, lse, Hq, Hkv, N, scale, causal,
+                                                     window, slopes);
   else
     return ATTN_ERR_UNSUPPORTED;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -91,6 +91,8 @@ struct Params {
   int pairs;  // ceil(N / 256)
   float scale_log2;
   int causal;
+  int window;            // > 0: key j visible to query i only if i - j < window
+  const float *slopes;   // ALiBi slope per query head (kernel variant with the bias)
 };
 
 // One thread's 128-column score row -> P (bf16 pairs in TMEM at s_addr) and
@@ -122,7 +124,7 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float c, flo
   return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
 }
 
-template <int D>
+template <int D, bool kAlibi>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -164,9 +166,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int hkv = hq / (p.Hq / p.Hkv);
   const int row0 = pair * 2 * BM;
   const int nkv = (p.N + BN - 1) / BN;
-  const int n0 = p.causal ? min(2 * pair + 1, nkv) : nkv;
-  const int n1 = (row0 + BM < p.N) ? (p.causal ? min(2 * pair + 2, nkv) : nkv) : 0;
-  const int n = max(n0, n1);
+  // KV tiles [js_t, je_t) of each Q tile: the causal diagonal caps the end,
+  // a sliding window moves the start; a Q tile past N has none.
+  // (Scalars, not arrays: the issuing thread reads them every iteration.)
+  const bool rows1 = row0 + BM < p.N;
+  const int je0 = p.causal ? min(row0 / BN + 1, nkv) : nkv;
+  const int je1 = !rows1 ? 0 : (p.causal ? min((row0 + BM) / BN + 1, nkv) : nkv);
+  const int js0 = p.window > 0 ? max(0, row0 - p.window + 1) / BN : 0;
+  const int js1 = (!rows1 || p.window <= 0) ? 0 : max(0, row0 + BM - p.window + 1) / BN;
+  const int jlo = js0;
+  const int jhi = max(je0, je1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -210,7 +219,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
                       row0 + t * BM, zq);
       int issued = 0;
-      for (int i = 0; i < 2 * n; ++i) {
+      for (int i = 0; i < 2 * (jhi - jlo); ++i) {
         const int slot = i % C::NST;
         const int round = i / C::NST;
         if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status))
@@ -219,7 +228,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
         for (int c = 0; c < C::CH; ++c)
           tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
-                      64 * c, (i >> 1) * BN, zkv);
+                      64 * c, (jlo + (i >> 1)) * BN, zkv);
         issued = i + 1;
       }
       // Drain: no copy may still be writing shared memory when the CTA exits.
@@ -265,50 +274,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                  (acc || ks > 0) ? 1u : 0u);
       };
 
+      // K/V tile j of this CTA sits at ring index 2*(j - jlo) (K) and +1 (V).
+      auto has = [&](int t, int j) {
+        return t == 0 ? (j >= js0 && j < je0) : (j >= js1 && j < je1);
+      };
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.status);
       ok = ok && wait_full(0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        tc_commit(&bars->s_full[0]);
-        if (n1 > 0) {
-          issue_s(1, 0);
-          tc_commit(&bars->s_full[1]);
-        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (has(t, jlo)) {
+            issue_s(t, 0);
+            tc_commit(&bars->s_full[t]);
+          }
         tc_commit(&bars->empty[slot_of(0)]);
       }
-      for (int j = 0; ok && j < n; ++j) {
-        const uint32_t ph = j & 1;
+      for (int j = jlo; ok && j < jhi; ++j) {
+        const int rj = j - jlo;
         bool v_ready = false;
-        if (j < n0) {
-          if (!(ok = mbar_wait(&bars->p_full[0], ph, abort_flag, p.status) && wait_full(2 * j + 1)))
+        if (has(0, j)) {
+          if (!(ok = mbar_wait(&bars->p_full[0], (j - js0) & 1, abort_flag, p.status) &&
+                     wait_full(2 * rj + 1)))
             break;
           v_ready = true;
           tc_fence_after();
-          issue_pv(0, 2 * j + 1, j > 0);
+          issue_pv(0, 2 * rj + 1, j > js0);
           tc_commit(&bars->o_full[0]);
         }
-        if (j + 1 < n && !(ok = wait_full(2 * j + 2))) break;
-        if (j + 1 < n0) {
+        if (j + 1 < jhi && !(ok = wait_full(2 * rj + 2))) break;
+        if (has(0, j + 1)) {
           // P0(j) aliases S0.  tcgen05.mma ops issued by one thread execute in
           // order, so S0(j+1) overwrites the P0(j) columns only after PV0(j),
           // issued just before, has consumed them: no completion wait needed.
-          issue_s(0, 2 * j + 2);
+          issue_s(0, 2 * rj + 2);
           tc_commit(&bars->s_full[0]);
         }
-        if (j < n1) {
-          if (!(ok = mbar_wait(&bars->p_full[1], ph, abort_flag, p.status))) break;
-          if (!v_ready && !(ok = wait_full(2 * j + 1))) break;
+        if (has(1, j)) {
+          if (!(ok = mbar_wait(&bars->p_full[1], (j - js1) & 1, abort_flag, p.status))) break;
+          if (!v_ready && !(ok = wait_full(2 * rj + 1))) break;
           tc_fence_after();
-          issue_pv(1, 2 * j + 1, j > 0);
+          issue_pv(1, 2 * rj + 1, j > js1);
           tc_commit(&bars->o_full[1]);
         }
-        tc_commit(&bars->empty[slot_of(2 * j + 1)]);  // V(j) no longer needed
-        if (j + 1 < n1) {
-          issue_s(1, 2 * j + 2);  // in order after PV1(j), as for tile 0
+        tc_commit(&bars->empty[slot_of(2 * rj + 1)]);  // V(j) no longer needed
+        if (has(1, j + 1)) {
+          issue_s(1, 2 * rj + 2);  // in order after PV1(j), as for tile 0
           tc_commit(&bars->s_full[1]);
         }
-        if (j + 1 < n) tc_commit(&bars->empty[slot_of(2 * j + 2)]);  // K(j+1) done
+        if (j + 1 < jhi) tc_commit(&bars->empty[slot_of(2 * rj + 2)]);  // K(j+1) done
       }
       // Every MMA issued above must finish before TMEM is released.
       tc_commit(&bars->mma_done);
@@ -324,32 +338,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = quarter * 32 + lane;    // row within the Q tile
     const int qtile = 2 * pair + t;
     const int row = qtile * BM + r;
-    const int nt = t == 0 ? n0 : n1;
+    const int jst = t == 0 ? js0 : js1, jen = t == 0 ? je0 : je1;
+    const int nt = jen - jst;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + t * 128;
     const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
     const float c = p.scale_log2;
+    // ALiBi slope in log2 units; the bias slope * (key - query) joins the score
+    // before the row max.
+    const float slope2 = kAlibi ? p.slopes[hq] * 1.4426950408889634f : 0.f;
     float m = -INFINITY;  // reference max, in log2 units of scaled scores
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      ok = mbar_wait(&bars->s_full[t], j & 1, abort_flag, p.status);
+    for (int j = jst; j < jen; ++j) {
+      ok = mbar_wait(&bars->s_full[t], (j - jst) & 1, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      int limit = min(BN, p.N - j * BN);
-      if (p.causal && j == qtile) limit = min(limit, r + 1);
+      // Visible columns [lo, hi) of this row in KV tile j: the end of the keys,
+      // the causal diagonal and the sliding window.
+      int hi = min(BN, p.N - j * BN);
+      if (p.causal) hi = min(hi, row - j * BN + 1);
+      // (Rows past N take the last real row's window so that they never force
+      // the masked path on a warp whose real rows need none.)
+      const int lo = p.window > 0 ? min(row, p.N - 1) - p.window + 1 - j * BN : 0;
       // The whole 128-column score row of this thread, in one TMEM load.
       uint32_t sv[128];
       tmem_ld128(s_addr, sv);
       tmem_ld_wait128(sv);
-      // Only diagonal and last tiles carry masked columns; elsewhere the warp
-      // takes the branch-free path.
-      const bool masked = !__all_sync(0xffffffffu, limit == BN);
+      float cx = c;  // factor still to apply to sv in the exponent
+      if (kAlibi) {
+        const float rb = slope2 * static_cast<float>(j * BN - row);
+        const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2), rb2 = make_float2(rb, rb);
+#pragma unroll
+        for (int i = 0; i < 128; i += 2) {
+          const float2 bias = fma2(sl2, make_float2(static_cast<float>(i), static_cast<float>(i + 1)), rb2);
+          const float2 x = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, bias);
+          sv[i] = __float_as_uint(x.x);
+          sv[i + 1] = __float_as_uint(x.y);
+        }
+        cx = 1.0f;
+      }
+      // Only diagonal, window-edge and last tiles carry masked columns;
+      // elsewhere the warp takes the branch-free path.
+      const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= BN);
       if (masked) {
 #pragma unroll
         for (int i = 0; i < 128; ++i)
-          if (i >= limit) sv[i] = 0xff800000u;  // -inf
+          if (i < lo || i >= hi) sv[i] = 0xff800000u;  // -inf
       }
       float mx;
       {
@@ -363,19 +399,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         mx = fmax3(m0, m1, fmaxf(m2, m3));
       }
-      const float m_new = fmaxf(m, mx * c);
+      const float m_new = fmaxf(m, mx * cx);
       const bool resc = m_new > m + 8.0f;
       const float alpha = resc ? ex2(m - m_new) : 1.0f;
       if (resc) m = m_new;
       l *= alpha;
+      // A row that has seen no visible key yet (a window edge) keeps m = -inf;
+      // its masked scores must still give P = 0, not -inf - (-inf).
+      const float m_use = (m == -INFINITY) ? 0.f : m;
       // P = 2^(s*c - m), rounded to bf16 and written over the (already read) S
       // columns; the row sum stays in fp32.  Unmasked tiles compute one pair in
       // four with the FMA-pipe polynomial to unload the special-function unit.
       if (masked)
-        l += exp_row<false>(sv, c, m, s_addr);
+        l += exp_row<false>(sv, cx, m_use, s_addr);
       else
-        l += exp_row<true>(sv, c, m, s_addr);
-      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        l += exp_row<true>(sv, cx, m_use, s_addr);
+      if (j > jst && __any_sync(0xffffffffu, resc)) {
         // Lazy rescale of O (rare once the max settles).  O is stable here:
         // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
 #pragma unroll
@@ -463,15 +502,15 @@ bool make_map(CUtensorMap *map, const void *base, int D, int N, int BH) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kAlibi>
 attn_status_t launch(const void *q, const void *k, const void *v, void *o, float *lse, int B,
-                     int Hq, int Hkv, int N, float scale, int causal, cudaStream_t stream,
-                     unsigned *status) {
+                     int Hq, int Hkv, int N, float scale, int causal, int window,
+                     const float *slopes, cudaStream_t stream, unsigned *status) {
   using C = Cfg<D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D>,
+    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D, kAlibi>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
@@ -490,9 +529,11 @@ attn_status_t launch(const void *q, const void *k, const void *v, void *o, float
   prm.pairs = (N + 2 * BM - 1) / (2 * BM);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.causal = causal ? 1 : 0;
+  prm.window = window;
+  prm.slopes = slopes;
   const long long ctas = static_cast<long long>(prm.pairs) * B * Hq;
   if (ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  prefill_bf16_kernel<D><<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(
+  prefill_bf16_kernel<D, kAlibi><<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(
       mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -501,9 +542,19 @@ attn_status_t launch(const void *q, const void *k, const void *v, void *o, float
 
 attn_status_t launch_prefill_bf16(const void *q, const void *k, const void *v, void *o, float *lse,
                                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-                                  cudaStream_t stream, unsigned *status) {
-  if (d == 128) return launch<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, stream, status);
-  if (d == 64) return launch<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, stream, status);
+                                  int window, const float *slopes, cudaStream_t stream,
+                                  unsigned *status) {
+  const bool alibi = slopes != nullptr;
+  if (d == 128)
+    return alibi ? launch<128, true>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, window, slopes,
+                                     stream, status)
+                 : launch<128, false>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, window,
+                                      nullptr, stream, status);
+  if (d == 64)
+    return alibi ? launch<64, true>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, window, slopes,
+                                    stream, status)
+                 : launch<64, false>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, window,
+                                     nullptr, stream, status);
   return ATTN_ERR_UNSUPPORTED;
 }
 

@@ -40,6 +40,8 @@ class Prefill:
     causal: bool
     dtype: str  # "bf16" or "f32"
     seed: int
+    window: int = 0      # sliding window (with causal): keys with i - j >= window masked
+    alibi: bool = False  # ALiBi bias with the geometric slopes of alibi_slopes(Hq)
 
     @property
     def scale(self) -> float:
@@ -47,7 +49,12 @@ class Prefill:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs, 4*B*Hq*N^2*d, halved when causal."""
+        """Algorithmic FLOPs: 4*d per visible (query, key) pair -- 4*B*Hq*N^2*d,
+        halved when causal (the workloads' convention), fewer with a window."""
+        if self.window > 0:
+            n, w = self.N, min(self.window, self.N)
+            pairs = w * (w + 1) / 2.0 + (n - w) * w
+            return 4.0 * self.B * self.Hq * pairs * self.d
         f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
         return f / 2.0 if self.causal else f
 
@@ -85,6 +92,15 @@ MHA_SWEEP = tuple(Prefill("mha_n%d" % n, 2, 16, 16, n, 128, False, "bf16", 1000 
 CAUSAL = Prefill("causal_n8192", 1, 32, 32, 8192, 128, True, "bf16", 2)
 GQA = Prefill("gqa_causal_n4096", 4, 32, 8, 4096, 128, True, "bf16", 3)
 DECODE = Decode()
+# Lab 01 extensions: a Mistral-style window of 4096 keys and ALiBi, both causal,
+# on the causal workload's shape.
+WINDOW = Prefill("window4096_causal_n8192", 1, 32, 32, 8192, 128, True, "bf16", 5, window=4096)
+ALIBI = Prefill("alibi_causal_n8192", 1, 32, 32, 8192, 128, True, "bf16", 6, alibi=True)
+
+
+def alibi_slopes(H: int) -> list:
+    """The geometric ALiBi slopes 2^(-8 (h+1) / H), h = 0..H-1 (Press et al.)."""
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
 
 
 def _gen(device, seed: int) -> torch.Generator:

@@ -94,6 +94,30 @@ EXATTN_API attn_status_t attn_fwd_f32(const float *q, const float *k, const floa
                            int causal, attn_stream_t stream);
 
 /*
+ * attn_fwd_ext / attn_fwd_f32_ext -- attn_fwd / attn_fwd_f32 with the two
+ * variants the Phase 08 page lists among the Lab 01 extensions: sliding-window
+ * attention (as in Mistral) and ALiBi bias.  The page only names them; this
+ * library reads them plainly:
+ *   window > 0      key j is visible to query i only if i - j < window, on top
+ *                   of causal masking (window > 0 requires causal != 0);
+ *                   window == 0 means no window.
+ *   alibi_slopes    NULL, or a DEVICE array of Hq floats a_h: the bias
+ *                   a_h * (j - i) is added to scale * q_i . k_j before the
+ *                   softmax (a_h >= 0 makes older keys weigh less); L includes it.
+ * Other arguments, layouts and errors as for attn_fwd / attn_fwd_f32;
+ * window < 0, a window without causal, or a misaligned slopes pointer give
+ * ATTN_ERR_INVALID_ARG.
+ */
+EXATTN_API attn_status_t attn_fwd_ext(const void *q, const void *k, const void *v, void *o,
+                                      float *lse, int B, int Hq, int Hkv, int N, int d,
+                                      float scale, int causal, int window,
+                                      const float *alibi_slopes, attn_stream_t stream);
+EXATTN_API attn_status_t attn_fwd_f32_ext(const float *q, const float *k, const float *v,
+                                          float *o, float *lse, int B, int Hq, int Hkv, int N,
+                                          int d, float scale, int causal, int window,
+                                          const float *alibi_slopes, attn_stream_t stream);
+
+/*
  * attn_decode_workspace_bytes -- bytes of device workspace attn_decode_paged
  * needs for S sequences, Hq query heads, head dim d and at most max_blocks
  * pages per sequence.  Returns 0 for invalid sizes.

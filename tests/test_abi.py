@@ -83,6 +83,13 @@ def test_prefill_argument_checks(lib, kw, code):
                             kw.get("d", 128), kw.get("scale", 0.1), 0, None) == code
 
 
+@pytest.mark.parametrize("window,causal,slopes,code", [
+    (-1, 1, None, INVALID), (8, 0, None, INVALID), (0, 1, A + 2, INVALID), (8, 1, A + 1, INVALID)])
+def test_window_alibi_argument_checks(lib, window, causal, slopes, code):
+    for fn in (lib.attn_fwd_ext, lib.attn_fwd_f32_ext):
+        assert fn(A, A, A, A, A, 1, 2, 1, 16, 128, 0.1, causal, window, slopes, None) == code
+
+
 def test_decode_workspace_size(lib):
     # 512 pages of 16 tokens in chunks of 32 pages -> 16 chunks per sequence.
     n = ea.decode_workspace_bytes(64, 32, 128, 512)

@@ -157,3 +157,77 @@ def test_full_size_mha(cfg):
 @pytest.mark.parametrize("cfg", [syn.CAUSAL, syn.GQA], ids=lambda c: c.name)
 def test_full_size_causal_and_gqa(cfg):
     full_size_check(cfg)
+
+
+# ------------------------------------------------ sliding window and ALiBi
+
+EXT_SMALL = [
+    # B, Hq, Hkv, N, d, window, alibi
+    (1, 2, 2, 300, 128, 1, False),
+    (1, 2, 1, 300, 128, 17, True),
+    (1, 4, 2, 513, 128, 128, False),
+    (2, 2, 2, 700, 64, 200, True),
+    (1, 2, 2, 1000, 128, 129, False),
+    (1, 2, 2, 1000, 128, 0, True),
+    (1, 2, 2, 640, 128, 5000, True),   # window wider than the sequence
+    (1, 8, 2, 900, 128, 300, True),    # GQA
+]
+
+
+def slopes_for(Hq):
+    return torch.tensor(syn.alibi_slopes(Hq), dtype=torch.float32)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,window,alibi", EXT_SMALL)
+def test_bf16_window_alibi_small(B, Hq, Hkv, N, d, window, alibi):
+    q, k, v = syn.random_qkv(B, Hq, Hkv, N, d, seed=300 + N + window)
+    scale = 1.0 / math.sqrt(d)
+    sl = slopes_for(Hq) if alibi else None
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=scale, causal=True, window=window,
+                                    alibi_slopes=None if sl is None else sl.numpy())
+    out = torch.full_like(q, float("nan"), device=DEV)
+    lse = torch.full((B, Hq, N), float("nan"), device=DEV)
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=scale, out=out,
+                       lse=lse, window=window, alibi_slopes=None if sl is None else sl.to(DEV))
+    torch.cuda.synchronize()
+    assert_bf16_parity(o, l, o_ref, l_ref, (B, Hq, Hkv, N, d, window, alibi))
+    assert ea.device_status() == 0
+
+
+@pytest.mark.parametrize("window,alibi", [(1, False), (37, True), (200, False), (0, True)])
+def test_fp32_window_alibi(window, alibi):
+    B, Hq, Hkv, N, d = 1, 4, 2, 260, 64
+    q, k, v = syn.random_qkv(B, Hq, Hkv, N, d, seed=40 + window, dtype=torch.float32)
+    sl = slopes_for(Hq) if alibi else None
+    o_ref, l_ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale=0.125, causal=True,
+                                    window=window, alibi_slopes=None if sl is None else sl.numpy())
+    o, l = ea.attn_fwd_f32(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=0.125,
+                           window=window, alibi_slopes=None if sl is None else sl.to(DEV))
+    torch.cuda.synchronize()
+    assert_f32_parity(o, l, o_ref, l_ref, (window, alibi))
+
+
+def test_window_wider_than_sequence_equals_causal_bitwise():
+    q, k, v = (t.to(DEV) for t in syn.random_qkv(1, 4, 2, 777, 128, seed=9))
+    o1, l1 = ea.attn_fwd(q, k, v, causal=True)
+    o2, l2 = ea.attn_fwd(q, k, v, causal=True, window=777)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("cfg", [syn.WINDOW, syn.ALIBI], ids=lambda c: c.name)
+def test_full_size_window_and_alibi(cfg):
+    q, k, v = syn.prefill_inputs(cfg, device=DEV)
+    sl = slopes_for(cfg.Hq).to(DEV) if cfg.alibi else None
+    o, l = ea.attn_fwd(q, k, v, causal=True, scale=cfg.scale, window=cfg.window, alibi_slopes=sl)
+    torch.cuda.synchronize()
+    assert ea.device_status() == 0
+    assert torch.isfinite(o.float()).all() and torch.isfinite(l).all()
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.N, 64, cfg.seed)
+    o_ref, l_ref = oracle.attention_rows(q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                         v.float().cpu().numpy(), cfg.scale, True, rows,
+                                         window=cfg.window,
+                                         alibi_slopes=None if sl is None else sl.cpu().numpy())
+    idx = torch.from_numpy(rows).to(DEV)
+    assert_bf16_parity(o.reshape(-1, cfg.d)[idx], l.reshape(-1)[idx], o_ref, l_ref, cfg.name)
