@@ -57,6 +57,13 @@ def _load():
                                             ci, ci, ci, ci, ci, ci, ci, cd,
                                             i32p, ci, ci]
         lib.oracle_decode_paged.restype = ci
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.oracle_decode_paged_q8.argtypes = [f32p, u8p, u8p, f32p, f32p, i32p, i32p, f64p,
+                                               f64p, ci, ci, ci, ci, ci, ci, ci, cd, ci,
+                                               i32p, ci, ci]
+        lib.oracle_decode_paged_q8.restype = ci
+        lib.oracle_e4m3_to_double.argtypes = [ci]
+        lib.oracle_e4m3_to_double.restype = cd
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ci
         _lib = lib
@@ -165,4 +172,53 @@ def decode_paged(q, k_pages_bf16_bits, v_pages_bf16_bits, block_table, seq_lens,
                                      int(nthreads or max_threads()))
     if rc != 0:
         raise ValueError("oracle_decode_paged failed with code %d" % rc)
+    return o, lse
+
+
+def e4m3_to_double(byte: int) -> float:
+    """The oracle's decoding of one FP8 E4M3 byte."""
+    return float(_load().oracle_e4m3_to_double(int(byte)))
+
+
+KV_FORMATS = {"e4m3": 0, "int8": 1}
+
+
+def _bytes(a) -> np.ndarray:
+    a = np.asarray(a)
+    return np.ascontiguousarray(a.view(np.uint8) if a.dtype == np.int8 else a.astype(np.uint8, copy=False))
+
+
+def decode_paged_q8(q, k_pages_u8, v_pages_u8, k_scales, v_scales, block_table, seq_lens,
+                    scale: float, fmt: str = "e4m3", seq_ids=None, nthreads: int | None = None):
+    """Decode over an 8-bit paged cache with one scale per (page, kv head).
+
+    k/v pages [num_pages,Hkv,page_size,d] uint8 holding E4M3 (fmt "e4m3") or
+    two's-complement INT8 (fmt "int8") bytes; k/v scales [num_pages,Hkv]
+    float32; element = scale * decoded byte.  Returns (O [nseq,Hq,d],
+    L [nseq,Hq]) in float64.
+    """
+    q = _f32(q)
+    kp, vp = _bytes(k_pages_u8), _bytes(v_pages_u8)
+    ks = _f32(k_scales)
+    vs = _f32(v_scales)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    S, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = kp.shape
+    if d2 != d or vp.shape != kp.shape or ks.shape != (num_pages, Hkv) or vs.shape != ks.shape:
+        raise ValueError("page pool / scale shape mismatch")
+    max_blocks = bt.shape[1]
+    if seq_ids is None:
+        seq_ids = np.arange(S, dtype=np.int32)
+    seq_ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32))
+    o = np.zeros((seq_ids.size, Hq, d), dtype=np.float64)
+    lse = np.zeros((seq_ids.size, Hq), dtype=np.float64)
+    rc = _load().oracle_decode_paged_q8(
+        _ptr(q, ctypes.c_float), _ptr(kp, ctypes.c_uint8), _ptr(vp, ctypes.c_uint8),
+        _ptr(ks, ctypes.c_float), _ptr(vs, ctypes.c_float), _ptr(bt, ctypes.c_int32),
+        _ptr(sl, ctypes.c_int32), _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+        S, Hq, Hkv, d, page_size, max_blocks, num_pages, float(scale), KV_FORMATS[fmt],
+        _ptr(seq_ids, ctypes.c_int32), int(seq_ids.size), int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_decode_paged_q8 failed with code %d" % rc)
     return o, lse

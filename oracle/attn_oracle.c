@@ -37,6 +37,8 @@
  * oracle_decode_paged gathers a sequence's keys and values from the page pool
  * through the block table (Lab 03 step 4: pages reached through an
  * indirection table), then evaluates the same definition for its one query.
+ * oracle_decode_paged_q8 is the same over 8-bit pages (E4M3 or INT8) with one
+ * scale per (page, kv head): each element is dequantised to fp64 first.
  *
  * Inputs are float (the exact values the GPU sees: fp32, or bf16 upcast) or,
  * for the page pool, raw bf16 bit patterns; arithmetic is double throughout.
@@ -264,6 +266,97 @@ int oracle_decode_paged(const float *q, const uint16_t *k_pages, const uint16_t 
     }
     return bad ? -2 : 0;
 }
+
+/* An OCP FP8 E4M3 ("e4m3fn") byte: 1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN; there
+ * is no infinity.  Written from the format's definition. */
+static double e4m3_to_double(uint8_t b)
+{
+    int sign = (b >> 7) & 1, e = (b >> 3) & 0xF, m = b & 7;
+    double v;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* One 8-bit cache element: fmt 0 = FP8 E4M3, fmt 1 = INT8 (two's complement). */
+static double q8_to_double(uint8_t b, int fmt)
+{
+    return fmt == 0 ? e4m3_to_double(b) : (double)(int8_t)b;
+}
+
+/* Decode over an 8-bit paged KV cache: the KV-cache quantisation answer of the
+ * screna.ai page (8-bit storage halves the cache against 16-bit; INT8 is the
+ * safe default, NVIDIA's FP8 the hardware format; group-wise scales keep
+ * accuracy).  Read plainly: each (page, kv head) slice of K and of V is one
+ * group with one fp32 scale, k = k_scales[p*Hkv+g] * q8(byte), likewise v;
+ * the bytes are E4M3 (fmt 0) or INT8 (fmt 1).  Everything else is exactly
+ * oracle_decode_paged. */
+int oracle_decode_paged_q8(const float *q, const uint8_t *k_pages, const uint8_t *v_pages,
+                           const float *k_scales, const float *v_scales,
+                           const int32_t *block_table, const int32_t *seq_lens,
+                           double *o, double *lse,
+                           int S, int Hq, int Hkv, int d, int page_size, int max_blocks,
+                           int num_pages, double scale, int fmt,
+                           const int32_t *seq_ids, int nseq, int nthreads)
+{
+    int G, r, bad = 0;
+    if (S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || page_size <= 0 || max_blocks <= 0 ||
+        num_pages <= 0 || Hq % Hkv != 0 || nseq < 0 || (fmt != 0 && fmt != 1)) return -1;
+    if (!q || !k_pages || !v_pages || !k_scales || !v_scales || !block_table || !seq_lens ||
+        !o || !lse || (!seq_ids && nseq > 0)) return -1;
+    G = Hq / Hkv;
+    for (r = 0; r < nseq; ++r) {
+        int s = seq_ids[r], t, len;
+        if (s < 0 || s >= S) return -1;
+        len = seq_lens[s];
+        if (len < 0 || len > max_blocks * page_size) return -1;
+        for (t = 0; t < len; t += page_size) {
+            int32_t p = block_table[(size_t)s * max_blocks + t / page_size];
+            if (p < 0 || p >= num_pages) return -1;
+        }
+    }
+    if (nthreads <= 0) nthreads = 1;
+
+    #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) reduction(|:bad)
+    for (r = 0; r < nseq * Hkv; ++r) {
+        int s = seq_ids[r / Hkv], g = r % Hkv;
+        int len = seq_lens[s];
+        int t, c, hh;
+        double *kd = (double *)malloc(sizeof(double) * ((size_t)len * d + 1));
+        double *vd = (double *)malloc(sizeof(double) * ((size_t)len * d + 1));
+        double *sc = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+        if (!kd || !vd || !sc) { free(kd); free(vd); free(sc); bad = 1; continue; }
+        for (t = 0; t < len; ++t) {
+            int32_t p = block_table[(size_t)s * max_blocks + t / page_size];
+            size_t base = (((size_t)p * Hkv + g) * page_size + (t % page_size)) * (size_t)d;
+            double ks = (double)k_scales[(size_t)p * Hkv + g];
+            double vs = (double)v_scales[(size_t)p * Hkv + g];
+            for (c = 0; c < d; ++c) {
+                kd[(size_t)t * d + c] = ks * q8_to_double(k_pages[base + c], fmt);
+                vd[(size_t)t * d + c] = vs * q8_to_double(v_pages[base + c], fmt);
+            }
+        }
+        for (hh = 0; hh < G; ++hh) {
+            int h = g * G + hh;
+            const float *qs = q + ((size_t)s * Hq + h) * (size_t)d;
+            for (t = 0; t < len; ++t) {
+                double acc = 0.0;
+                for (c = 0; c < d; ++c) acc += (double)qs[c] * kd[(size_t)t * d + c];
+                sc[t] = scale * acc;
+            }
+            softmax_row_times_v(sc, len, vd, d,
+                                o + ((size_t)(r / Hkv) * Hq + h) * (size_t)d,
+                                lse + (size_t)(r / Hkv) * Hq + h);
+        }
+        free(kd); free(vd); free(sc);
+    }
+    return bad ? -2 : 0;
+}
+
+/* Exposed for the pins: the e4m3 decode of one byte. */
+double oracle_e4m3_to_double(int byte) { return e4m3_to_double((uint8_t)byte); }
 
 int oracle_max_threads(void)
 {

@@ -13,6 +13,11 @@ the mathematics fix, independently of the oracle's own code:
 * structural invariants: GQA equals MHA with repeated K/V heads, key/value
   permutation invariance, shift invariance under large offsets, causal rows
   equal non-causal attention over the prefix, paged equals contiguous;
+* 8-bit KV cache: all 256 E4M3 codes against torch's float8_e4m3fn
+  converter and the format's fixed points; E4M3 / INT8 decode with
+  power-of-two scales equals the bf16 paged decode of the dequantised cache
+  exactly; scale linearity (V's scale multiplies O, K's acts as the softmax
+  scale);
 * mutation checks: plausible one-token mistakes planted in a copy of the
   oracle's C source are each caught by at least one pin.
 """
@@ -433,6 +438,127 @@ def test_decode_rejects_bad_page_ids():
                             np.array([[0, 5]], np.int32), np.array([3], np.int32), scale=1.0)
 
 
+# ------------------------------------------------------- FP8 (e4m3) KV cache
+
+
+def _e4m3_table():
+    """All 256 E4M3 bytes decoded by torch's float8_e4m3fn conversion (an
+    implementation independent of the oracle), as float64."""
+    import torch
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    return codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_decoding_matches_format():
+    # The format's fixed points: 1.0 = 0.0111.000, the largest finite value 448
+    # = 0.1111.110, the smallest normal 2^-6, the smallest subnormal 2^-9,
+    # NaN at S.1111.111, sign-magnitude negatives; then all 256 codes against
+    # torch's converter.
+    assert oracle.e4m3_to_double(0x38) == 1.0
+    assert oracle.e4m3_to_double(0x7E) == 448.0
+    assert oracle.e4m3_to_double(0x08) == 2.0 ** -6
+    assert oracle.e4m3_to_double(0x01) == 2.0 ** -9
+    assert oracle.e4m3_to_double(0x07) == 7 * 2.0 ** -9
+    assert oracle.e4m3_to_double(0x3C) == 1.5
+    assert oracle.e4m3_to_double(0xC0) == -2.0
+    assert math.isnan(oracle.e4m3_to_double(0x7F)) and math.isnan(oracle.e4m3_to_double(0xFF))
+    assert math.copysign(1.0, oracle.e4m3_to_double(0x80)) == -1.0
+    ref = _e4m3_table()
+    got = np.array([oracle.e4m3_to_double(b) for b in range(256)])
+    finite = ~np.isnan(ref)
+    np.testing.assert_array_equal(np.isnan(got), ~finite)
+    np.testing.assert_array_equal(got[finite], ref[finite])
+
+
+def _q8_cache(rng, P, Hkv, ps, d, scale_exps, fmt):
+    """Random finite 8-bit codes (E4M3 NaN codes excluded) and power-of-two scales."""
+    kb = rng.integers(0, 256, size=(P, Hkv, ps, d)).astype(np.uint8)
+    vb = rng.integers(0, 256, size=(P, Hkv, ps, d)).astype(np.uint8)
+    if fmt == "e4m3":
+        for a in (kb, vb):
+            a[(a & 0x7F) == 0x7F] = 0x3A
+    ks = (2.0 ** rng.choice(scale_exps, size=(P, Hkv))).astype(np.float32)
+    vs = (2.0 ** rng.choice(scale_exps, size=(P, Hkv))).astype(np.float32)
+    return kb, vb, ks, vs
+
+
+def _q8_values(codes, fmt):
+    """Decoded codes, by torch's e4m3 converter or numpy's int8 view."""
+    if fmt == "e4m3":
+        return _e4m3_table()[codes]
+    return codes.view(np.int8).astype(np.float64)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "int8"])
+def test_q8_decode_equals_decode_of_dequantised_cache(fmt):
+    # With per-(page, head) scales, each cached element is scale * code.
+    # Dequantise in the test (torch's e4m3 table or numpy's int8 view); with
+    # power-of-two scales every value is exactly representable in bf16 (at
+    # most 8 significant bits), so the pinned bf16 paged decode sees the same
+    # numbers and must agree exactly.
+    rng = np.random.default_rng(77)
+    S, Hq, Hkv, d, ps, P, maxb = 4, 8, 2, 16, 4, 24, 5
+    exps = [-6, -5, -4, -3] if fmt == "e4m3" else [-9, -8, -7]
+    kb, vb, ks, vs = _q8_cache(rng, P, Hkv, ps, d, exps, fmt)
+    lens = np.array([1, 7, 20, 0], dtype=np.int32)
+    bt = np.full((S, maxb), -1, dtype=np.int32)
+    perm = rng.permutation(P).astype(np.int32)
+    nxt = 0
+    for s in range(S):
+        n = -(-int(lens[s]) // ps)
+        bt[s, :n] = perm[nxt:nxt + n]
+        nxt += n
+    q = _bits_to_f32(_bf16_bits(rand(S, Hq, d, rng=rng)))
+    kd = _q8_values(kb, fmt) * ks[:, :, None, None].astype(np.float64)
+    vd = _q8_values(vb, fmt) * vs[:, :, None, None].astype(np.float64)
+    kbits, vbits = _bf16_bits(kd.astype(np.float32)), _bf16_bits(vd.astype(np.float32))
+    np.testing.assert_array_equal(_bits_to_f32(kbits).astype(np.float64), kd)
+    np.testing.assert_array_equal(_bits_to_f32(vbits).astype(np.float64), vd)
+    o8, l8 = oracle.decode_paged_q8(q, kb, vb, ks, vs, bt, lens, scale=0.3, fmt=fmt)
+    ob, lb = oracle.decode_paged(q, kbits, vbits, bt, lens, scale=0.3)
+    np.testing.assert_array_equal(o8, ob)
+    np.testing.assert_array_equal(l8, lb)
+    # and directly against contiguous attention over the dequantised tokens
+    for s in range(S):
+        if lens[s] == 0:
+            continue
+        n = int(lens[s])
+        kc = np.stack([kd[bt[s, t // ps], :, t % ps] for t in range(n)], axis=1)
+        vc = np.stack([vd[bt[s, t // ps], :, t % ps] for t in range(n)], axis=1)
+        oc, lc = oracle.attention(q[s][None, :, None, :], kc[None], vc[None], scale=0.3)
+        np.testing.assert_allclose(o8[s], oc[0, :, 0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l8[s], lc[0, :, 0], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "int8"])
+def test_q8_scale_linearity(fmt):
+    # V's scale multiplies the output and leaves L alone; K's scale multiplies
+    # every score, i.e. acts like the softmax scale.
+    rng = np.random.default_rng(78)
+    S, Hq, Hkv, d, ps, P, maxb = 2, 4, 2, 8, 4, 6, 3
+    kb, vb, _, _ = _q8_cache(rng, P, Hkv, ps, d, [0], fmt)
+    one = np.ones((P, Hkv), np.float32)
+    bt = np.array([[0, 1, 2], [3, 4, 5]], dtype=np.int32)
+    lens = np.array([9, 12], dtype=np.int32)
+    q = rand(S, Hq, d, rng=rng) * (0.05 if fmt == "e4m3" else 0.002)
+    o1, l1 = oracle.decode_paged_q8(q, kb, vb, one, one, bt, lens, scale=0.5, fmt=fmt)
+    o2, l2 = oracle.decode_paged_q8(q, kb, vb, one, 3.0 * one, bt, lens, scale=0.5, fmt=fmt)
+    np.testing.assert_allclose(o2, 3.0 * o1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(l2, l1)
+    o3, l3 = oracle.decode_paged_q8(q, kb, vb, 0.25 * one, one, bt, lens, scale=0.5, fmt=fmt)
+    o4, l4 = oracle.decode_paged_q8(q, kb, vb, one, one, bt, lens, scale=0.125, fmt=fmt)
+    np.testing.assert_allclose(o3, o4, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l3, l4, rtol=0, atol=1e-12)
+
+
+def test_q8_decode_rejects_bad_page_ids():
+    kp = np.zeros((2, 1, 2, 1), dtype=np.uint8)
+    sc = np.ones((2, 1), np.float32)
+    with pytest.raises(ValueError):
+        oracle.decode_paged_q8(np.ones((1, 1, 1), np.float32), kp, kp, sc, sc,
+                               np.array([[0, 5]], np.int32), np.array([3], np.int32), scale=1.0)
+
+
 # ------------------------------------------------------------- mutations
 
 MUTANTS = {
@@ -449,6 +575,57 @@ MUTANTS = {
     "log_base_two": ("*lse = m + log(l);", "*lse = m + log2(l);"),
     "scale_dropped": ("S[(size_t)i * Nk + j] = scale * acc;", "S[(size_t)i * Nk + j] = acc;"),
 }
+
+
+Q8_MUTANTS = {
+    "e4m3_bias": ("else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                  "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_subnormal_exponent": ("if (e == 0) v = ldexp((double)m / 8.0, -6);",
+                                "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
+    "e4m3_mantissa_width": ("else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                            "else v = ldexp(1.0 + (double)m / 16.0, e - 7);"),
+    "q8_scales_swapped": ("double ks = (double)k_scales[(size_t)p * Hkv + g];",
+                          "double ks = (double)v_scales[(size_t)p * Hkv + g];"),
+    "q8_scale_index": ("double vs = (double)v_scales[(size_t)p * Hkv + g];",
+                       "double vs = (double)v_scales[(size_t)g * Hkv + p % Hkv];"),
+    "int8_unsigned": ("fmt == 0 ? e4m3_to_double(b) : (double)(int8_t)b;",
+                      "fmt == 0 ? e4m3_to_double(b) : (double)b;"),
+}
+
+
+def _run_mutant(src_old, src_new, tmp_path, checks):
+    src = open(os.path.join(ROOT, "oracle", "attn_oracle.c")).read()
+    assert src_old in src
+    mutated = src.replace(src_old, src_new, 1)
+    cpath = tmp_path / "mut.c"
+    cpath.write_text(mutated)
+    lib = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(lib), str(cpath), "-lm"])
+    saved = oracle._lib
+    real_build = oracle.build
+    try:
+        oracle._lib = None
+        oracle.build = lambda force=False: str(lib)
+        failures = 0
+        for chk in checks:
+            try:
+                chk()
+            except (AssertionError, ValueError, FloatingPointError):
+                failures += 1
+        return failures
+    finally:
+        oracle.build = real_build
+        oracle._lib = saved
+
+
+@pytest.mark.parametrize("name", sorted(Q8_MUTANTS))
+def test_q8_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = Q8_MUTANTS[name]
+    checks = [test_e4m3_decoding_matches_format]
+    for fmt in ("e4m3", "int8"):
+        checks += [lambda f=fmt: test_q8_decode_equals_decode_of_dequantised_cache(f),
+                   lambda f=fmt: test_q8_scale_linearity(f)]
+    assert _run_mutant(old, new, tmp_path, checks) > 0, "mutant %s survived every pin" % name
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
