@@ -9,8 +9,9 @@ per-launch CUDA-event pairs that give the kernel time.
 The JSON line also carries, measured in the same run:
   * ``components``: causal N=8192 (H=32), GQA causal N=4096 (B=4, Hq=32,
     Hkv=8) prefill TFLOP/s, and the paged GQA decode (64 sequences, context
-    U[512, 8192], 16-token pages) in HBM GB/s, each as a fraction of the
-    measured peak;
+    U[512, 8192], 16-token pages) in HBM GB/s over a bf16 cache and over 8-bit
+    (E4M3, INT8) caches of the same shape, each as a fraction of the measured
+    peak;
   * ``roofline`` for the prefill kernel (tensor-bound);
   * ``e2e``: the same sweep through the public API with pinned host buffers,
     host->device and device->host copies inside the timed region;
@@ -238,6 +239,34 @@ class Decode:
         return 2  # split + combine
 
 
+class DecodeQ8:
+    """The decode workload over an 8-bit cache (same q, lengths and placement)."""
+
+    def __init__(self, cfg, lib, fmt):
+        import exact_io_aware_101_b200 as ea
+        self.cfg, self.lib, self.fmt = cfg, lib, fmt
+        self.code = ea.KV_FORMATS[fmt]
+        self.inp = syn.decode_inputs_q8(cfg, fmt=fmt, device="cuda")
+        self.o = torch.empty_like(self.inp["q"])
+        self.lse = torch.empty(cfg.S, cfg.Hq, dtype=torch.float32, device="cuda")
+        self.ws_bytes = ea.decode_workspace_bytes(cfg.S, cfg.Hq, cfg.d, cfg.max_blocks)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.bytes = syn.decode_bytes(self.inp["seq_lens"].cpu().tolist(), cfg.Hkv, cfg.d, cfg.Hq,
+                                      cfg.page_size, kv_elem_bytes=1)
+
+    def launch(self):
+        c, i = self.cfg, self.inp
+        rc = self.lib.attn_decode_paged_q8(
+            i["q"].data_ptr(), i["k_pages"].data_ptr(), i["v_pages"].data_ptr(),
+            i["k_scales"].data_ptr(), i["v_scales"].data_ptr(), self.code,
+            i["block_table"].data_ptr(), i["seq_lens"].data_ptr(), self.o.data_ptr(),
+            self.lse.data_ptr(), c.S, c.Hq, c.Hkv, c.d, c.page_size, c.max_blocks, c.num_pages,
+            c.scale, self.ws.data_ptr(), self.ws_bytes, torch.cuda.current_stream().cuda_stream)
+        if rc != 0:
+            raise RuntimeError("attn_decode_paged_q8 failed: %d" % rc)
+        return 2  # split + combine
+
+
 def timed_launches(items, flush, reps):
     """Per-item list of CUDA-event durations (ms), L2 flushed before each launch."""
     times = [[] for _ in items]
@@ -435,10 +464,21 @@ def run_ours(args):
                                      "traffic": profiled_traffic("decode_paged_gqa.md",
                                                                  "decode_paged.cu"),
                                      "bound": "hbm"}
+        del dec
+        for fmt in ("e4m3", "int8"):
+            dq = DecodeQ8(syn.DECODE, lib, fmt)
+            timed_launches([dq], flush, 3)
+            t, _ = timed_launches([dq], flush, args.component_reps)
+            sec = sum(t[0]) / len(t[0]) / 1e3
+            gbs = dq.bytes / sec / 1e9
+            comps["decode_paged_gqa_" + fmt] = {
+                "gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3,
+                "algorithmic_bytes": dq.bytes, "peak_gbs": peak_hbm,
+                "traffic": profiled_traffic("decode_q8_gqa.md", "decode_q8.cu"), "bound": "hbm"}
+            del dq
         if ea.device_status() != 0:
             raise RuntimeError("device status word set in the component runs")
         line["components"] = comps
-        del dec
 
     if not args.skip_e2e:
         ms, h2d, d2h = e2e_sweep(sweep, max(1, min(args.steps, 5)))
@@ -463,12 +503,16 @@ def run_only(args):
     torch.cuda.set_device(0)
     lib = ea.library()
     table = {c.name: c for c in syn.MHA_SWEEP + (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI)}
+    q8 = {syn.DECODE.name + "_" + f: f for f in ("e4m3", "int8")}
     if args.only == syn.DECODE.name:
         it = Decode(syn.DECODE, lib)
+    elif args.only in q8:
+        it = DecodeQ8(syn.DECODE, lib, q8[args.only])
     elif args.only in table:
         it = Prefill(table[args.only], lib)
     else:
-        raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table) + [syn.DECODE.name]))
+        raise SystemExit("unknown workload %r; one of %s"
+                         % (args.only, sorted(table) + [syn.DECODE.name] + sorted(q8)))
     for _ in range(args.reps):
         it.launch()
     torch.cuda.synchronize()

@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "attn_fwd", "attn_fwd_f32", "attn_decode_paged", "attn_decode_paged_noalloc",
-    "decode_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
+    "attn_decode_paged_q8", "KV_FORMATS", "decode_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
     "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
     "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "AttnError",
 ]
@@ -28,12 +28,16 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ext", "attn_fwd_f32_ext",
                     "attn_decode_workspace_bytes",
-                    "attn_decode_paged", "attn_decode_paged_noalloc", "attn_device_status",
+                    "attn_decode_paged", "attn_decode_paged_noalloc", "attn_decode_paged_q8",
+                    "attn_device_status",
                     "attn_status_string", "attn_version")
 # Size of the library's fixed per-device scratch used by attn_decode_paged_noalloc.
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 ATTN_DEV_BAD_PAGE = 0x1
 ATTN_DEV_TIMEOUT = 0x2
+# kv_format codes of attn_decode_paged_q8 and the torch dtypes accepted for each.
+KV_FORMATS = {"e4m3": 0, "int8": 1}
+_KV_DTYPES = {"e4m3": (torch.float8_e4m3fn, torch.uint8), "int8": (torch.int8,)}
 _STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_CUDA"}
 
 _lib = None
@@ -70,6 +74,9 @@ def library() -> ctypes.CDLL:
         lib.attn_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
                                                   ci, ci, cf, vp]
         lib.attn_decode_paged_noalloc.restype = ci
+        lib.attn_decode_paged_q8.argtypes = [vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, ci, ci, ci,
+                                             ci, ci, ci, ci, cf, vp, ctypes.c_size_t, vp]
+        lib.attn_decode_paged_q8.restype = ci
         lib.attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
         lib.attn_device_status.restype = ci
         lib.attn_status_string.argtypes = [ci]
@@ -206,6 +213,59 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float |
                                      num_pages, float(scale), workspace.data_ptr(),
                                      workspace.numel(), _stream(q))
     _raise(rc, "attn_decode_paged")
+    return out, lse
+
+
+def attn_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, block_table, seq_lens,
+                         kv_format: str = "e4m3", scale: float | None = None, out=None, lse=None,
+                         workspace=None):
+    """Paged single-token decode over an 8-bit KV cache.
+
+    k_pages/v_pages [num_pages,Hkv,page_size,d]: E4M3 codes (torch.float8_e4m3fn,
+    or their bytes as uint8) for kv_format "e4m3", torch.int8 for "int8";
+    k_scales/v_scales [num_pages,Hkv] float32, one per (page, K/V head): the
+    element is scale * code.  Everything else as attn_decode_paged.
+    """
+    if kv_format not in KV_FORMATS:
+        raise ValueError("kv_format must be one of %s" % sorted(KV_FORMATS))
+    _check(q, "q", torch.bfloat16, 3)
+    for name, t in (("k_pages", k_pages), ("v_pages", v_pages)):
+        if not isinstance(t, torch.Tensor) or t.dtype not in _KV_DTYPES[kv_format]:
+            raise TypeError("%s must be one of %s for kv_format %r"
+                            % (name, _KV_DTYPES[kv_format], kv_format))
+        _check(t, name, t.dtype, 4)
+    _check(k_scales, "k_scales", torch.float32, 2)
+    _check(v_scales, "v_scales", torch.float32, 2)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    S, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = k_pages.shape
+    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("page pools must be [num_pages, Hkv, page_size, d]")
+    if tuple(k_scales.shape) != (num_pages, Hkv) or tuple(v_scales.shape) != (num_pages, Hkv):
+        raise ValueError("scales must be [num_pages, Hkv]")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table/seq_lens must have S rows")
+    max_blocks = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 3)
+    _check(lse, "lse", torch.float32, 2)
+    need = decode_workspace_bytes(S, Hq, d, max_blocks, page_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace", torch.uint8, 1)
+    rc = library().attn_decode_paged_q8(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                        k_scales.data_ptr(), v_scales.data_ptr(),
+                                        KV_FORMATS[kv_format], block_table.data_ptr(),
+                                        seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), S,
+                                        Hq, Hkv, d, page_size, max_blocks, num_pages, float(scale),
+                                        workspace.data_ptr(), workspace.numel(), _stream(q))
+    _raise(rc, "attn_decode_paged_q8")
     return out, lse
 
 

@@ -136,6 +136,33 @@ attn_status_t attn_decode_paged(const void *q, const void *k_pages, const void *
                              reinterpret_cast<cudaStream_t>(stream), status);
 }
 
+attn_status_t attn_decode_paged_q8(const void *q, const void *k_pages, const void *v_pages,
+                                   const float *k_scales, const float *v_scales, int kv_format,
+                                   const int32_t *block_table, const int32_t *seq_lens, void *o,
+                                   float *lse, int S, int Hq, int Hkv, int d, int page_size,
+                                   int max_blocks, int num_pages, float scale, void *workspace,
+                                   size_t workspace_bytes, attn_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned4(k_scales) ||
+      !aligned4(v_scales) || !aligned4(block_table) || !aligned4(seq_lens) || !aligned16(o) ||
+      !aligned4(lse) || !aligned16(workspace))
+    return ATTN_ERR_INVALID_ARG;
+  if (S <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || page_size <= 0 ||
+      max_blocks <= 0 || num_pages <= 0 || !good_scale(scale) ||
+      (kv_format != ATTN_KV_E4M3 && kv_format != ATTN_KV_INT8))
+    return ATTN_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || page_size != 16) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks) * page_size > (1LL << 30)) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_pages) * Hkv >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < decode_workspace_bytes(S, Hq, d, max_blocks)) return ATTN_ERR_INVALID_ARG;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, kv_format, block_table,
+                                seq_lens, o, lse, S, Hq, Hkv, d, max_blocks, num_pages, scale,
+                                workspace, reinterpret_cast<cudaStream_t>(stream), status);
+}
+
 // The workspace-free decode: same checks and kernels as attn_decode_paged, with
 // the library's fixed per-device scratch array standing in for the workspace.
 attn_status_t attn_decode_paged_noalloc(const void *q, const void *k_pages, const void *v_pages,

@@ -314,7 +314,8 @@ template <int D>
 __global__ void __launch_bounds__(128)
     decode_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ l2_part,
                           const int *__restrict__ seq_lens, __nv_bfloat16 *__restrict__ o,
-                          float *__restrict__ lse, int S, int Hq, int max_blocks, int nsplit) {
+                          float *__restrict__ lse, int S, int Hq, int max_blocks, int nsplit,
+                          int pages_per_split) {
   constexpr int DPL = D / 32;
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(128)
     return;
   }
   const int nparts =
-      bad_len ? 0 : ((len + kPageSize - 1) / kPageSize + kPagesPerSplit - 1) / kPagesPerSplit;
+      bad_len ? 0 : ((len + kPageSize - 1) / kPageSize + pages_per_split - 1) / pages_per_split;
   const float *lp = l2_part + head * nsplit;
   bool bad = bad_len;
   float M = -INFINITY;
@@ -457,16 +458,25 @@ attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void
   else
     return ATTN_ERR_UNSUPPORTED;
   if (!ok) return ATTN_ERR_UNSUPPORTED;
+  return launch_decode_combine(o_part, l2_part, seq_lens, o, lse, S, Hq, d, max_blocks, nsplit,
+                               kPagesPerSplit, stream);
+}
+
+attn_status_t launch_decode_combine(const float *o_part, const float *l2_part, const int *seq_lens,
+                                    void *o, float *lse, int S, int Hq, int d, int max_blocks,
+                                    int nsplit, int pages_per_split, cudaStream_t stream) {
   const int heads = S * Hq;
   const int blocks = (heads + 3) / 4;
   if (d == 128)
     decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(o_part, l2_part, seq_lens,
                                                            static_cast<__nv_bfloat16 *>(o), lse, S,
-                                                           Hq, max_blocks, nsplit);
-  else
+                                                           Hq, max_blocks, nsplit, pages_per_split);
+  else if (d == 64)
     decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(o_part, l2_part, seq_lens,
                                                           static_cast<__nv_bfloat16 *>(o), lse, S,
-                                                          Hq, max_blocks, nsplit);
+                                                          Hq, max_blocks, nsplit, pages_per_split);
+  else
+    return ATTN_ERR_UNSUPPORTED;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -1,0 +1,550 @@
+// decode_q8.cu -- single-token attention over an 8-bit paged KV cache.
+//
+// What it computes: the paged decode of decode_paged.cu ("Phase 08" page,
+// Concepts: KV cache and paged attention; Lab 03 step 4) over a cache whose K
+// and V pages hold 8-bit codes -- FP8 E4M3 or INT8 -- with one fp32 scale per
+// (page, K/V head) for K and one for V: the KV-cache quantisation answer of the
+// screna.ai interview page (8-bit storage halves the cache against 16 bits;
+// group-wise scales; INT8 the safe default, FP8 the hardware format).  The
+// element a kernel works with is scale * code, exactly as the fp64 oracle
+// dequantises it.
+//
+// Why it is shaped this way.  The decode reads every cached byte once, so it is
+// bound by HBM bandwidth; at one byte per element the bytes halve, and the
+// CUDA-core work of the 16-bit kernel (per element: decode, and one FMA per
+// query head of the group for q.k and again for p.v) would no longer hide under
+// the copy.  So the two contractions of a page run as warp-level m16n8k16 MMAs
+// on f16 operands with f32 accumulation, with a page's 16 tokens as the M (or
+// K) extent of one tile:
+//   S^T[16 tok x 8 heads] = K_page[16 x d] . Q^T[d x 8]          (d/16 MMAs)
+//   O^T[d x 8 heads]     += V_page^T[d x 16 tok] . P^T[16 x 8]   (d/16 MMAs)
+// E4M3 and INT8 codes convert to f16 exactly (cvt.rn.f16x2.e4m3x2; for INT8
+// the byte goes into the mantissa of 1024 and 1152 is subtracted), so the only
+// roundings are Q's (bf16 -> f16 after a per-head power-of-two normalisation,
+// exact for every element within 2^28 of the head's largest), P's (f16) and
+// the f32 accumulations.  The page scales are applied in f32: the K scale to
+// the scores, the V scale when the page's P.V is added to the accumulator.
+//
+// Data movement.  One CTA per (chunk of kPagesPerSplit pages, K/V head, head
+// chunk, sequence); warp 4 is the producer: it TMA-loads each page's K and V
+// slices (16 rows x d bytes, 128-byte swizzle for d = 128, 64-byte for d = 64)
+// into a kStages-deep ring.  The swizzle makes both fragment patterns
+// conflict-free: K rows read along d, and V read across token rows at one
+// column.  Warps 0..3 take pages round-robin, keep a running max / sum per
+// head (online softmax, lazily rescaled), and the CTA merges them into one
+// normalised partial per head; the combine kernel of decode_paged.cu merges
+// the chunks exactly as for the 16-bit cache.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace exattn {
+namespace {
+
+constexpr int kPage = 16;
+constexpr int kPagesPerSplitQ8 = 32;  // must equal the 16-bit kernel's (shared workspace)
+constexpr int kWarpsQ8 = 4;
+constexpr int kStagesQ8 = 8;
+constexpr float kRescaleLog2 = 8.f;  // lazy rescale: move the max only when it grows by > 2^8
+
+template <int D>
+constexpr int tile_bytes() { return kPage * D; }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Two E4M3 codes in the low 16 bits (element 0 in bits 0-7) -> f16x2 (element 0
+// in the low half).  Exact: every E4M3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t w) {
+  uint32_t r;
+  const uint16_t h = static_cast<uint16_t>(w & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
+  return r;
+}
+
+// [u0, 0x64, u1, 0x64] is the f16x2 pair (1024 + u0, 1024 + u1); with
+// u = code + 128 (the code's sign bit flipped) subtracting 1152 leaves the
+// signed code, exactly.
+__device__ __forceinline__ uint32_t biased_f16x2_to_int(uint32_t x) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64806480u));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset of logical offset o inside a TMA-swizzled tile (tile base aligned
+// to the swizzle span): 128-byte swizzle for 128-byte rows, 64-byte for 64.
+template <int D>
+__device__ __forceinline__ uint32_t swz(uint32_t o) {
+  if constexpr (D == 128) return o ^ (((o >> 7) & 7u) << 4);
+  else return o ^ (((o >> 7) & 3u) << 4);
+}
+
+// The pair of codes (lo = element 0) at bits [16h, 16h+16) of a word -> f16x2.
+template <int FMT>
+__device__ __forceinline__ uint32_t codes_f16x2(uint32_t w, int h) {
+  if constexpr (FMT == ATTN_KV_E4M3) {
+    return e4m3x2_f16x2(h ? (w >> 16) : w);
+  } else {
+    const uint32_t x = w ^ 0x80808080u;
+    return biased_f16x2_to_int(prmt(x, 0x64646464u, h ? 0x4342u : 0x4140u));
+  }
+}
+
+// V^T fragment pair from two token rows' words A (token t) and B (token t+1):
+// element e of each (e = 0..3) gives the pair (A_e, B_e).
+template <int FMT>
+__device__ __forceinline__ void vpairs(uint32_t A, uint32_t B, uint32_t (&p)[4]) {
+  if constexpr (FMT == ATTN_KV_E4M3) {
+    const uint32_t lo = prmt(A, B, 0x5140u), hi = prmt(A, B, 0x7362u);
+    p[0] = e4m3x2_f16x2(lo);
+    p[1] = e4m3x2_f16x2(lo >> 16);
+    p[2] = e4m3x2_f16x2(hi);
+    p[3] = e4m3x2_f16x2(hi >> 16);
+  } else {
+    const uint32_t a = A ^ 0x80808080u, b = B ^ 0x80808080u;
+    const uint32_t lo = prmt(a, b, 0x5140u), hi = prmt(a, b, 0x7362u);
+    p[0] = biased_f16x2_to_int(prmt(lo, 0x64646464u, 0x4140u));
+    p[1] = biased_f16x2_to_int(prmt(lo, 0x64646464u, 0x4342u));
+    p[2] = biased_f16x2_to_int(prmt(hi, 0x64646464u, 0x4140u));
+    p[3] = biased_f16x2_to_int(prmt(hi, 0x64646464u, 0x4342u));
+  }
+}
+
+template <int D>
+struct VRow;  // one thread's slice of a V row: D/8 bytes
+template <>
+struct VRow<128> {
+  uint32_t w[4];
+};
+template <>
+struct VRow<64> {
+  uint32_t w[2];
+};
+
+template <int D>
+__device__ __forceinline__ VRow<D> load_vrow(const uint8_t *tile, int row, int g, bool live) {
+  VRow<D> r;
+  const uint8_t *p = tile + swz<D>(static_cast<uint32_t>(row * D + (D / 8) * g));
+  if constexpr (D == 128) {
+    const uint4 u = live ? *reinterpret_cast<const uint4 *>(p) : make_uint4(0, 0, 0, 0);
+    r.w[0] = u.x; r.w[1] = u.y; r.w[2] = u.z; r.w[3] = u.w;
+  } else {
+    const uint2 u = live ? *reinterpret_cast<const uint2 *>(p) : make_uint2(0, 0);
+    r.w[0] = u.x; r.w[1] = u.y;
+  }
+  return r;
+}
+
+// Workspace and partial layout as in decode_paged.cu: o_part [S][Hq][nsplit][D]
+// f32 (normalised), l2_part [S][Hq][nsplit] f32 (log2-sum-exp; NaN marks a bad
+// sequence).
+template <int D, int GB, int FMT>
+__global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
+    decode_q8_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const __nv_bfloat16 *__restrict__ q, const float *__restrict__ k_scales,
+                           const float *__restrict__ v_scales,
+                           const int *__restrict__ block_table, const int *__restrict__ seq_lens,
+                           float *__restrict__ o_part, float *__restrict__ l2_part, int Hq,
+                           int Hkv, int max_blocks, int num_pages, float scale_log2, int nsplit,
+                           int head_chunks, unsigned *status) {
+  constexpr int KS = D / 16;   // k-steps of the q.k MMA = M-tiles of the p.v MMA
+  constexpr int KCH = D / 64;  // 16-byte chunks of a K row held by one thread
+  constexpr int TILE = tile_bytes<D>();
+  constexpr int STAGE = 2 * TILE;
+  static_assert(GB >= 1 && GB <= 8, "one n8 tile of heads per CTA");
+  static_assert(kPagesPerSplitQ8 <= 32 && kPagesPerSplitQ8 / kWarpsQ8 <= 32, "one lane per page");
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y / head_chunks;
+  const int h0 = kvh * (Hq / Hkv) + (blockIdx.y % head_chunks) * GB;
+  const int s = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;  // MMA fragment coordinates
+
+  const int len = seq_lens[s];
+  const bool bad_len = len < 0 || len > max_blocks * kPage;
+  const int page_begin = split * kPagesPerSplitQ8;
+  const int n_pages = bad_len ? 0 : (len + kPage - 1) / kPage;
+  if (!bad_len && page_begin >= n_pages) return;  // chunk past the end: nothing to do
+  const int npg = bad_len ? 0 : min(n_pages, page_begin + kPagesPerSplitQ8) - page_begin;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *ring = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ uint64_t full[kStagesQ8], empty[kStagesQ8];
+  __shared__ int stage_ntok[kStagesQ8];
+  __shared__ int sm_pid[kPagesPerSplitQ8];
+  __shared__ float sm_m[kWarpsQ8][GB], sm_l[kWarpsQ8][GB];
+  __shared__ float sm_acc[kWarpsQ8][GB][D];
+  __shared__ int sm_bad, sm_abort;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesQ8; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    sm_bad = bad_len ? 1 : 0;
+    sm_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpsQ8 && lane < npg)
+    sm_pid[lane] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + lane];
+  __syncthreads();
+
+  if (warp == kWarpsQ8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < npg; ++i) {
+        const int st = i % kStagesQ8;
+        if (i >= kStagesQ8 &&
+            !mbar_wait(&empty[st], ((i / kStagesQ8) - 1) & 1, &sm_abort, status))
+          break;
+        const int pid = sm_pid[i];
+        if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
+          sm_bad = 1;
+          stage_ntok[st] = 0;
+          mbar_arrive(&full[st]);
+        } else {
+          stage_ntok[st] = min(kPage, len - (page_begin + i) * kPage);
+          uint8_t *dst = ring + st * STAGE;
+          const int z = pid * Hkv + kvh;
+          mbar_arrive_expect_tx(&full[st], STAGE);
+          tma_load_3d(dst, &tm_k, &full[st], 0, 0, z);
+          tma_load_3d(dst + TILE, &tm_v, &full[st], 0, 0, z);
+        }
+        issued = i + 1;
+      }
+      // Let every copy land before the CTA (and its shared memory) goes away.
+      for (int i = max(0, issued - kStagesQ8); i < issued; ++i)
+        mbar_wait_drain(&full[i % kStagesQ8], (i / kStagesQ8) & 1, status);
+    }
+  } else {
+    // ------------------------------------------------------------ compute
+    // Q^T fragments (the B operand of the q.k MMA) for head n = g: k-step t
+    // takes d = (D/4)c + 4t + {0,1} and {2,3}, the same permutation of d the
+    // K fragments use.  Each head is scaled by a power of two 2^e (its largest
+    // |q| lands in [2^14, 2^15)) before rounding to f16; the scores get
+    // scale*log2(e)*2^-e back in f32.
+    uint32_t qb[KS][2];
+    float sq_own;
+    {
+      float qv[D / 4];
+      const bool live = g < GB;
+      const __nv_bfloat16 *qp = q + (static_cast<size_t>(s) * Hq + h0 + (live ? g : 0)) * D +
+                                (D / 4) * c;
+#pragma unroll
+      for (int u = 0; u < D / 32; ++u) {
+        const uint4 w = live ? *reinterpret_cast<const uint4 *>(qp + 8 * u) : make_uint4(0, 0, 0, 0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          qv[8 * u + 2 * e] = __uint_as_float(ww[e] << 16);
+          qv[8 * u + 2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u);
+        }
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < D / 4; ++e) amax = fmaxf(amax, fabsf(qv[e]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      int ex = 0;
+      if (amax > 0.f && amax <= 3.4028235e38f) {
+        int fe;
+        frexpf(amax, &fe);  // amax in [2^(fe-1), 2^fe)
+        ex = min(100, max(-120, 15 - fe));
+      }
+#pragma unroll
+      for (int t = 0; t < KS; ++t) {
+        qb[t][0] = pack_f16x2(ldexpf(qv[4 * t], ex), ldexpf(qv[4 * t + 1], ex));
+        qb[t][1] = pack_f16x2(ldexpf(qv[4 * t + 2], ex), ldexpf(qv[4 * t + 3], ex));
+      }
+      sq_own = ldexpf(scale_log2, -ex);
+    }
+    // Score multipliers of this thread's two accumulator columns (heads 2c, 2c+1).
+    const float sq0 = __shfl_sync(0xffffffffu, sq_own, 8 * c);
+    const float sq1 = __shfl_sync(0xffffffffu, sq_own, 8 * c + 4);
+
+    // Page scales of this warp's pages: lane j holds those of its j-th page.
+    float ks_r = 0.f, vs_r = 0.f;
+    {
+      const int i = warp + kWarpsQ8 * lane;
+      if (lane < (kPagesPerSplitQ8 + kWarpsQ8 - 1) / kWarpsQ8 && i < npg) {
+        const int pid = sm_pid[i];
+        if (pid >= 0 && pid < num_pages) {
+          ks_r = k_scales[static_cast<size_t>(pid) * Hkv + kvh];
+          vs_r = v_scales[static_cast<size_t>(pid) * Hkv + kvh];
+        }
+      }
+    }
+
+    float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2c, 2c+1 (log2 units)
+    float l0 = 0.f, l1 = 0.f;              // this thread's share of the running sums
+    float acc[KS][4];                      // O^T: rows d = (D/8)g + 2i (+1), cols 2c, 2c+1
+#pragma unroll
+    for (int i = 0; i < KS; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+    // Source lanes of the P^T fragment: tokens 2c and 2c+1 of head g.
+    const int src0 = 8 * c + (g >> 1), src1 = src0 + 4;
+    const uint32_t psel = (g & 1) ? 0x7632u : 0x5410u;
+
+    for (int j = 0, i = warp; i < npg; ++j, i += kWarpsQ8) {
+      const int st = i % kStagesQ8;
+      const bool ok = mbar_wait(&full[st], (i / kStagesQ8) & 1, &sm_abort, status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int ntok = stage_ntok[st];
+      const float ks = __shfl_sync(0xffffffffu, ks_r, j);
+      const float vs = __shfl_sync(0xffffffffu, vs_r, j);
+      if (ntok > 0) {
+        const uint8_t *kt = ring + st * (2 * TILE);
+        const uint8_t *vt = kt + TILE;
+        // ---- S^T = K . Q^T for tokens g and g+8.
+        uint4 ka[KCH], kb[KCH];
+#pragma unroll
+        for (int h = 0; h < KCH; ++h) {
+          const uint32_t col = static_cast<uint32_t>((D / 4) * c + 16 * h);
+          ka[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>(g * D + col));
+          kb[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>((g + 8) * D + col));
+        }
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < KS; ++t) {
+          const uint4 &A = ka[t / 4], &B = kb[t / 4];
+          const uint32_t wa = (t % 4 == 0) ? A.x : (t % 4 == 1) ? A.y : (t % 4 == 2) ? A.z : A.w;
+          const uint32_t wb = (t % 4 == 0) ? B.x : (t % 4 == 1) ? B.y : (t % 4 == 2) ? B.z : B.w;
+          mma_f16(sc, codes_f16x2<FMT>(wa, 0), codes_f16x2<FMT>(wb, 0), codes_f16x2<FMT>(wa, 1),
+                  codes_f16x2<FMT>(wb, 1), qb[t][0], qb[t][1]);
+        }
+        const float kq0 = ks * sq0, kq1 = ks * sq1;
+        float s0 = sc[0] * kq0, s1 = sc[1] * kq1, s2 = sc[2] * kq0, s3 = sc[3] * kq1;
+        if (ntok < kPage) {
+          if (g >= ntok) s0 = s1 = -INFINITY;
+          if (g + 8 >= ntok) s2 = s3 = -INFINITY;
+        }
+        // ---- online softmax per head (column), over the page's 16 tokens.
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const bool grow = (mx0 > m0 + kRescaleLog2) || (mx1 > m1 + kRescaleLog2);
+        if (__any_sync(0xffffffffu, grow)) {
+          const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+          const float a0 = ex2(m0 - n0), a1 = ex2(m1 - n1);
+          m0 = n0;
+          m1 = n1;
+          l0 *= a0;
+          l1 *= a1;
+#pragma unroll
+          for (int i2 = 0; i2 < KS; ++i2) {
+            acc[i2][0] *= a0;
+            acc[i2][1] *= a1;
+            acc[i2][2] *= a0;
+            acc[i2][3] *= a1;
+          }
+        }
+        const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        // ---- P^T fragment: (P[head g][tok 2c], [2c+1]) and tokens 2c+8, 2c+9.
+        const uint32_t P01 = pack_f16x2(p0, p1), P23 = pack_f16x2(p2, p3);
+        const uint32_t x0 = __shfl_sync(0xffffffffu, P01, src0);
+        const uint32_t x1 = __shfl_sync(0xffffffffu, P01, src1);
+        const uint32_t y0 = __shfl_sync(0xffffffffu, P23, src0);
+        const uint32_t y1 = __shfl_sync(0xffffffffu, P23, src1);
+        const uint32_t pb0 = prmt(x0, x1, psel), pb1 = prmt(y0, y1, psel);
+        // ---- O^T += V^T . P^T.  Rows past the sequence end read as zero.
+        const VRow<D> va = load_vrow<D>(vt, 2 * c, g, 2 * c < ntok);
+        const VRow<D> vb = load_vrow<D>(vt, 2 * c + 1, g, 2 * c + 1 < ntok);
+        const VRow<D> vc = load_vrow<D>(vt, 2 * c + 8, g, 2 * c + 8 < ntok);
+        const VRow<D> vd = load_vrow<D>(vt, 2 * c + 9, g, 2 * c + 9 < ntok);
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) {
+          uint32_t lo[4], hi[4];
+          vpairs<FMT>(va.w[w], vb.w[w], lo);
+          vpairs<FMT>(vc.w[w], vd.w[w], hi);
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            float t4[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_f16(t4, lo[2 * e2], lo[2 * e2 + 1], hi[2 * e2], hi[2 * e2 + 1], pb0, pb1);
+            float(&a)[4] = acc[2 * w + e2];
+            a[0] = fmaf(t4[0], vs, a[0]);
+            a[1] = fmaf(t4[1], vs, a[1]);
+            a[2] = fmaf(t4[2], vs, a[2]);
+            a[3] = fmaf(t4[3], vs, a[3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
+    }
+
+    // Sums over the warp's tokens (lanes sharing c hold the same heads).
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    const int hA = 2 * c, hB = 2 * c + 1;
+#pragma unroll
+    for (int i = 0; i < KS; ++i) {
+      const int d0 = (D / 8) * g + 2 * i;
+      if (hA < GB) {
+        sm_acc[warp][hA][d0] = acc[i][0];
+        sm_acc[warp][hA][d0 + 1] = acc[i][2];
+      }
+      if (hB < GB) {
+        sm_acc[warp][hB][d0] = acc[i][1];
+        sm_acc[warp][hB][d0 + 1] = acc[i][3];
+      }
+    }
+    if (g == 0) {
+      if (hA < GB) {
+        sm_m[warp][hA] = m0;
+        sm_l[warp][hA] = l0;
+      }
+      if (hB < GB) {
+        sm_m[warp][hB] = m1;
+        sm_l[warp][hB] = l1;
+      }
+    }
+  }
+  __syncthreads();
+
+  // Merge the warps and write this chunk's normalised partial per head.
+  const bool bad = sm_bad != 0 || sm_abort != 0;
+  if (bad && threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
+  for (int idx = threadIdx.x; idx < GB * D; idx += blockDim.x) {
+    const int hh = idx / D, col = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarpsQ8; ++w) M = fmaxf(M, sm_m[w][hh]);
+    float wsum = 0.f, num = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarpsQ8; ++w) {
+      const float wt = (sm_m[w][hh] == -INFINITY) ? 0.f : ex2(sm_m[w][hh] - M);
+      wsum += wt * sm_l[w][hh];
+      num += wt * sm_acc[w][hh][col];
+    }
+    const size_t slot = (static_cast<size_t>(s) * Hq + h0 + hh) * nsplit + split;
+    o_part[slot * D + col] = bad ? NAN : num / wsum;
+    if (col == 0) l2_part[slot] = bad ? NAN : M + log2f(wsum);
+  }
+}
+
+// Page pool [num_pages][Hkv][16][D] bytes as a 3-D tensor (D, 16, num_pages*Hkv);
+// one box is one page slice of one K/V head.
+bool make_page_map(CUtensorMap *map, const void *base, int D, long long slices) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(kPage),
+                        static_cast<cuuint64_t>(slices)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(kPage) * D};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(kPage), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int GB, int FMT>
+attn_status_t launch_split_q8(dim3 grid, cudaStream_t st, const CUtensorMap &mk,
+                              const CUtensorMap &mv, const void *q, const float *ks,
+                              const float *vs, const int *bt, const int *sl, float *op, float *lp,
+                              int Hq, int Hkv, int maxb, int npages, float sl2, int nsplit, int hc,
+                              unsigned *status) {
+  constexpr int kSmem = kStagesQ8 * 2 * tile_bytes<D>() + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(decode_q8_split_kernel<D, GB, FMT>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  decode_q8_split_kernel<D, GB, FMT><<<grid, (kWarpsQ8 + 1) * 32, kSmem, st>>>(
+      mk, mv, static_cast<const __nv_bfloat16 *>(q), ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages,
+      sl2, nsplit, hc, status);
+  return ATTN_OK;
+}
+
+template <int D, int FMT>
+attn_status_t dispatch_q8(int GB, dim3 grid, cudaStream_t st, const CUtensorMap &mk,
+                          const CUtensorMap &mv, const void *q, const float *ks, const float *vs,
+                          const int *bt, const int *sl, float *op, float *lp, int Hq, int Hkv,
+                          int maxb, int npages, float sl2, int nsplit, int hc, unsigned *status) {
+  switch (GB) {
+    case 8: return launch_split_q8<D, 8, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 4: return launch_split_q8<D, 4, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 2: return launch_split_q8<D, 2, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 1: return launch_split_q8<D, 1, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+  }
+  return ATTN_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+attn_status_t launch_decode_paged_q8(const void *q, const void *k_pages, const void *v_pages,
+                                     const float *k_scales, const float *v_scales, int kv_format,
+                                     const int *block_table, const int *seq_lens, void *o,
+                                     float *lse, int S, int Hq, int Hkv, int d, int max_blocks,
+                                     int num_pages, float scale, void *workspace,
+                                     cudaStream_t stream, unsigned *status) {
+  const int G = Hq / Hkv;
+  const int GB = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+  const int head_chunks = G / GB;
+  const int nsplit = (max_blocks + kPagesPerSplitQ8 - 1) / kPagesPerSplitQ8;
+  const size_t parts = static_cast<size_t>(S) * Hq * nsplit;
+  float *o_part = static_cast<float *>(workspace);
+  float *l2_part = reinterpret_cast<float *>(
+      static_cast<uint8_t *>(workspace) +
+      ((parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+  if (static_cast<long long>(Hkv) * head_chunks > 65535 || S > 65535) return ATTN_ERR_UNSUPPORTED;
+  CUtensorMap mk, mv;
+  const long long slices = static_cast<long long>(num_pages) * Hkv;
+  if (!make_page_map(&mk, k_pages, d, slices) || !make_page_map(&mv, v_pages, d, slices))
+    return ATTN_ERR_CUDA;
+  dim3 grid(nsplit, Hkv * head_chunks, S);
+  const float sl2 = scale * 1.4426950408889634f;
+  attn_status_t st;
+  if (d == 128 && kv_format == ATTN_KV_E4M3)
+    st = dispatch_q8<128, ATTN_KV_E4M3>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+  else if (d == 128 && kv_format == ATTN_KV_INT8)
+    st = dispatch_q8<128, ATTN_KV_INT8>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+  else if (d == 64 && kv_format == ATTN_KV_E4M3)
+    st = dispatch_q8<64, ATTN_KV_E4M3>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+  else if (d == 64 && kv_format == ATTN_KV_INT8)
+    st = dispatch_q8<64, ATTN_KV_INT8>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+  else
+    return ATTN_ERR_UNSUPPORTED;
+  if (st != ATTN_OK) return st;
+  return launch_decode_combine(o_part, l2_part, seq_lens, o, lse, S, Hq, d, max_blocks, nsplit,
+                               kPagesPerSplitQ8, stream);
+}
+
+}  // namespace exattn

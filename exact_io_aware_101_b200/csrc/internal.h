@@ -1,6 +1,8 @@
 // internal.h -- launchers shared between the kernel files and the C ABI layer.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -29,6 +31,24 @@ attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void
                                   int S, int Hq, int Hkv, int d, int max_blocks, int num_pages,
                                   float scale, void *workspace, cudaStream_t stream,
                                   unsigned *status);
+
+// Merge the chunk partials of a split decode (workspace layout of
+// decode_workspace_bytes) into O (bf16) and L; chunks hold pages_per_split pages.
+attn_status_t launch_decode_combine(const float *o_part, const float *l2_part, const int *seq_lens,
+                                    void *o, float *lse, int S, int Hq, int d, int max_blocks,
+                                    int nsplit, int pages_per_split, cudaStream_t stream);
+
+// The same decode over 8-bit pages (kv_format ATTN_KV_E4M3 or ATTN_KV_INT8) with
+// per-(page, K/V head) fp32 scales; same workspace.
+attn_status_t launch_decode_paged_q8(const void *q, const void *k_pages, const void *v_pages,
+                                     const float *k_scales, const float *v_scales, int kv_format,
+                                     const int *block_table, const int *seq_lens, void *o,
+                                     float *lse, int S, int Hq, int Hkv, int d, int max_blocks,
+                                     int num_pages, float scale, void *workspace,
+                                     cudaStream_t stream, unsigned *status);
+
+// cuTensorMapEncodeTiled, or nullptr if the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 
 // Device address of the fixed scratch array used by attn_decode_paged_noalloc
 // (ATTN_DECODE_NOALLOC_SCRATCH_BYTES bytes) on the current device.

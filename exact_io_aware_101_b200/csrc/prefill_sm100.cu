@@ -473,6 +473,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // --------------------------------------------------------------- host side
+}  // namespace
+
+// cuTensorMapEncodeTiled from the driver, looked up once (no link-time libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -486,6 +489,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   });
   return fn;
 }
+
+namespace {
 
 // [BH][N][D] bf16 viewed as a 3-D tensor; boxes of 64 x 128 x 1, 128B swizzle.
 bool make_map(CUtensorMap *map, const void *base, int D, int N, int BH) {

@@ -16,6 +16,8 @@ causal, grouped-query and paged-decode extensions):
 * ``DECODE``  bf16 paged decode, 64 sequences, Hq=32, Hkv=8, d=128,
   lengths uniform in [512, 8192], 16-token pages from a 40000-page pool placed
   by a random permutation                                        seed 4
+  The 8-bit cache variants (E4M3, INT8) quantise the same pools per
+  (page, K/V head) slice with scale = amax / qmax (quantize_pages).
 
 Generation order for a prefill workload: q, k, v from one generator.  For the
 decode workload: seq_lens (randint, CPU), the page permutation (randperm, CPU),
@@ -166,17 +168,65 @@ def decode_inputs(cfg: Decode = DECODE, device="cpu", seq_lens=None):
                 block_table=table.to(device), seq_lens=seq_lens.to(device))
 
 
-def decode_bytes(seq_lens, Hkv: int, d: int, Hq: int, page_size: int = 16) -> int:
+def decode_bytes(seq_lens, Hkv: int, d: int, Hq: int, page_size: int = 16,
+                 kv_elem_bytes: int = 2) -> int:
     """Algorithmic HBM bytes of one decode call.
 
-    K and V of every visible token (bf16), q and o (bf16), L (fp32) and the
-    block-table entries the call follows.  A partly filled last page counts only
-    its visible tokens.
+    K and V of every visible token (kv_elem_bytes per element: 2 for bf16, 1 for
+    an 8-bit cache), q and o (bf16), L (fp32) and the block-table entries the
+    call follows.  A partly filled last page counts only its visible tokens.
+    An 8-bit cache adds its two fp32 scales per (visited page, K/V head).
     """
     lens = [int(x) for x in seq_lens]
-    kv = sum(lens) * Hkv * d * 2 * 2
+    kv = sum(lens) * Hkv * d * 2 * kv_elem_bytes
     S = len(lens)
     qo = 2 * S * Hq * d * 2
     lse = S * Hq * 4
-    bt = 4 * sum((n + page_size - 1) // page_size for n in lens)
-    return kv + qo + lse + bt
+    pages = sum((n + page_size - 1) // page_size for n in lens)
+    bt = 4 * pages
+    scales = 2 * 4 * pages * Hkv if kv_elem_bytes == 1 else 0
+    return kv + qo + lse + bt + scales
+
+
+# Largest code magnitude of each 8-bit cache format.
+KV_QMAX = {"e4m3": 448.0, "int8": 127.0}
+
+
+def quantize_pages(pages: torch.Tensor, fmt: str, chunk: int = 4096):
+    """8-bit codes and per-(page, K/V head) fp32 scales for a page pool.
+
+    pages [P, Hkv, page_size, d] (any float dtype).  scale = amax / qmax over the
+    slice (1 for an all-zero slice); codes = x / scale rounded to the format
+    (E4M3 by torch's float8_e4m3fn conversion, INT8 by round-half-even and a
+    clamp to [-127, 127]).  This is how the synthetic cache is written; the
+    decode only reads it.  Returns (codes, scales) with codes of dtype
+    float8_e4m3fn or int8.
+    """
+    P, Hkv = pages.shape[0], pages.shape[1]
+    out_dtype = torch.float8_e4m3fn if fmt == "e4m3" else torch.int8
+    codes = torch.empty(pages.shape, dtype=out_dtype, device=pages.device)
+    scales = torch.empty((P, Hkv), dtype=torch.float32, device=pages.device)
+    for p0 in range(0, P, chunk):
+        x = pages[p0:p0 + chunk].float()
+        amax = x.abs().amax(dim=(2, 3))
+        sc = torch.where(amax > 0, amax / KV_QMAX[fmt], torch.ones_like(amax))
+        y = x / sc[:, :, None, None]
+        if fmt == "e4m3":
+            codes[p0:p0 + chunk] = y.to(torch.float8_e4m3fn)
+        else:
+            codes[p0:p0 + chunk] = torch.round(y).clamp(-127, 127).to(torch.int8)
+        scales[p0:p0 + chunk] = sc
+    return codes, scales
+
+
+def decode_inputs_q8(cfg: Decode = DECODE, fmt: str = "e4m3", device="cpu", seq_lens=None):
+    """decode_inputs with the K/V pools quantised to an 8-bit cache.
+
+    dict(q, k_pages/v_pages (codes), k_scales/v_scales [P,Hkv] fp32, block_table,
+    seq_lens): the same q, lengths and placement as decode_inputs(cfg).
+    """
+    inp = decode_inputs(cfg, device=device, seq_lens=seq_lens)
+    kc, ks = quantize_pages(inp.pop("k_pages"), fmt)
+    vc, vs = quantize_pages(inp.pop("v_pages"), fmt)
+    inp.update(k_pages=kc, v_pages=vc, k_scales=ks, v_scales=vs)
+    return inp

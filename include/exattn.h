@@ -154,6 +154,40 @@ EXATTN_API attn_status_t attn_decode_paged(const void *q, const void *k_pages, c
                                 attn_stream_t stream);
 
 /*
+ * attn_decode_paged_q8 -- attn_decode_paged over an 8-bit KV cache.  The
+ * KV-cache quantisation answer of the screna.ai interview page: 8-bit storage
+ * halves the cache against 16 bits, INT8 is the safe default and NVIDIA's FP8
+ * the hardware format, and group-wise scales keep accuracy.  Here the group is
+ * one (page, K/V head) slice: the element the attention uses is
+ *   k = k_scales[p * Hkv + g] * code(k_pages[p, g, slot, c])     (v likewise)
+ * with code() the E4M3 value (kv_format ATTN_KV_E4M3: sign, 4 exponent bits of
+ * bias 7, 3 mantissa bits, S.1111.111 = NaN, no infinities) or the two's-
+ * complement integer (ATTN_KV_INT8).  Everything else -- block table, lengths,
+ * outputs, workspace (attn_decode_workspace_bytes), bad-page handling -- is as
+ * for attn_decode_paged.
+ *
+ *   q                  [S, Hq, d] bf16
+ *   k_pages, v_pages   [num_pages, Hkv, page_size, d] one byte per element,
+ *                      16-byte aligned
+ *   k_scales, v_scales [num_pages, Hkv] float32 (device); only the entries of
+ *                      pages a sequence reaches are read
+ * num_pages * Hkv < 2^31.  The query is rounded to f16 inside the kernel after
+ * a per-head power-of-two normalisation and P is rounded to f16 before the P.V
+ * product; scores, sums and outputs accumulate in float32.
+ */
+#define ATTN_KV_E4M3 0
+#define ATTN_KV_INT8 1
+EXATTN_API attn_status_t attn_decode_paged_q8(const void *q, const void *k_pages,
+                                              const void *v_pages, const float *k_scales,
+                                              const float *v_scales, int kv_format,
+                                              const int32_t *block_table,
+                                              const int32_t *seq_lens, void *o, float *lse,
+                                              int S, int Hq, int Hkv, int d, int page_size,
+                                              int max_blocks, int num_pages, float scale,
+                                              void *workspace, size_t workspace_bytes,
+                                              attn_stream_t stream);
+
+/*
  * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot
  * allocate device memory.  The pages have no counterpart to this entry point; it
  * exists for how the library is used, not for the method.
