@@ -48,9 +48,15 @@ namespace exattn {
 namespace {
 
 constexpr int kPage = 16;
-constexpr int kPagesPerSplitQ8 = 32;  // must equal the 16-bit kernel's (shared workspace)
+// 64 pages (1024 tokens) per chunk: at one byte per element a chunk holds as
+// many bytes as the 16-bit kernel's 32-page chunk, so start-up (block table,
+// first copies) is amortised as well; the workspace of the 32-page chunking
+// is larger than this one needs.
+constexpr int kPagesPerSplitQ8 = 64;
 constexpr int kWarpsQ8 = 4;
-constexpr int kStagesQ8 = 8;
+// 16 stages of 4 KiB (d = 128): the same bytes in flight per CTA as the 16-bit
+// kernel's 8 stages of 8 KiB.
+constexpr int kStagesQ8 = 16;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale: move the max only when it grows by > 2^8
 
 template <int D>
@@ -176,7 +182,10 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
   constexpr int TILE = tile_bytes<D>();
   constexpr int STAGE = 2 * TILE;
   static_assert(GB >= 1 && GB <= 8, "one n8 tile of heads per CTA");
-  static_assert(kPagesPerSplitQ8 <= 32 && kPagesPerSplitQ8 / kWarpsQ8 <= 32, "one lane per page");
+  static_assert(kPagesPerSplitQ8 <= 64 && kPagesPerSplitQ8 / kWarpsQ8 <= 32,
+                "two block-table entries per producer lane, one page per consumer lane");
+  static_assert(kWarpsQ8 * GB * D * 4 + 2 * kWarpsQ8 * GB * 4 <= kStagesQ8 * STAGE,
+                "the merge scratch fits in the ring");
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / head_chunks;
   const int h0 = kvh * (Hq / Hkv) + (blockIdx.y % head_chunks) * GB;
@@ -197,9 +206,11 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
   __shared__ uint64_t full[kStagesQ8], empty[kStagesQ8];
   __shared__ int stage_ntok[kStagesQ8];
   __shared__ int sm_pid[kPagesPerSplitQ8];
-  __shared__ float sm_m[kWarpsQ8][GB], sm_l[kWarpsQ8][GB];
-  __shared__ float sm_acc[kWarpsQ8][GB][D];
   __shared__ int sm_bad, sm_abort;
+  // Merge scratch, over the ring once every page has been consumed.
+  float(*sm_acc)[GB][D] = reinterpret_cast<float(*)[GB][D]>(ring);
+  float(*sm_m)[GB] = reinterpret_cast<float(*)[GB]>(ring + kWarpsQ8 * GB * D * 4);
+  float(*sm_l)[GB] = reinterpret_cast<float(*)[GB]>(ring + kWarpsQ8 * GB * D * 4 + kWarpsQ8 * GB * 4);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStagesQ8; ++i) {
       mbar_init(&full[i], 1);
@@ -209,8 +220,10 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
     sm_abort = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpsQ8 && lane < npg)
-    sm_pid[lane] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + lane];
+  if (warp == kWarpsQ8) {
+    for (int i = lane; i < npg; i += 32)
+      sm_pid[i] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + i];
+  }
   __syncthreads();
 
   if (warp == kWarpsQ8) {
@@ -270,18 +283,21 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
       for (int e = 0; e < D / 4; ++e) amax = fmaxf(amax, fabsf(qv[e]));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // ex = 15 - (exponent of amax + 1), so amax * 2^ex lies in [2^14, 2^15);
+      // clamped so that 2^ex and 2^-ex are normal floats (exact multipliers).
       int ex = 0;
       if (amax > 0.f && amax <= 3.4028235e38f) {
-        int fe;
-        frexpf(amax, &fe);  // amax in [2^(fe-1), 2^fe)
-        ex = min(100, max(-120, 15 - fe));
+        const int e_amax = static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127;
+        ex = min(100, max(-113, 14 - e_amax));  // subnormal amax: e_amax = -127, clamped
       }
+      const float up = __uint_as_float(static_cast<uint32_t>(127 + ex) << 23);
+      const float down = __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
 #pragma unroll
       for (int t = 0; t < KS; ++t) {
-        qb[t][0] = pack_f16x2(ldexpf(qv[4 * t], ex), ldexpf(qv[4 * t + 1], ex));
-        qb[t][1] = pack_f16x2(ldexpf(qv[4 * t + 2], ex), ldexpf(qv[4 * t + 3], ex));
+        qb[t][0] = pack_f16x2(qv[4 * t] * up, qv[4 * t + 1] * up);
+        qb[t][1] = pack_f16x2(qv[4 * t + 2] * up, qv[4 * t + 3] * up);
       }
-      sq_own = ldexpf(scale_log2, -ex);
+      sq_own = scale_log2 * down;
     }
     // Score multipliers of this thread's two accumulator columns (heads 2c, 2c+1).
     const float sq0 = __shfl_sync(0xffffffffu, sq_own, 8 * c);
@@ -291,7 +307,7 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
     float ks_r = 0.f, vs_r = 0.f;
     {
       const int i = warp + kWarpsQ8 * lane;
-      if (lane < (kPagesPerSplitQ8 + kWarpsQ8 - 1) / kWarpsQ8 && i < npg) {
+      if (lane < kPagesPerSplitQ8 / kWarpsQ8 && i < npg) {
         const int pid = sm_pid[i];
         if (pid >= 0 && pid < num_pages) {
           ks_r = k_scales[static_cast<size_t>(pid) * Hkv + kvh];
@@ -329,15 +345,18 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
           ka[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>(g * D + col));
           kb[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>((g + 8) * D + col));
         }
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        // Two accumulator chains (even / odd k-steps) halve the MMA latency chain.
+        float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int t = 0; t < KS; ++t) {
           const uint4 &A = ka[t / 4], &B = kb[t / 4];
           const uint32_t wa = (t % 4 == 0) ? A.x : (t % 4 == 1) ? A.y : (t % 4 == 2) ? A.z : A.w;
           const uint32_t wb = (t % 4 == 0) ? B.x : (t % 4 == 1) ? B.y : (t % 4 == 2) ? B.z : B.w;
-          mma_f16(sc, codes_f16x2<FMT>(wa, 0), codes_f16x2<FMT>(wb, 0), codes_f16x2<FMT>(wa, 1),
-                  codes_f16x2<FMT>(wb, 1), qb[t][0], qb[t][1]);
+          mma_f16((t & 1) ? sd : sc, codes_f16x2<FMT>(wa, 0), codes_f16x2<FMT>(wb, 0),
+                  codes_f16x2<FMT>(wa, 1), codes_f16x2<FMT>(wb, 1), qb[t][0], qb[t][1]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[e] += sd[e];
         const float kq0 = ks * sq0, kq1 = ks * sq1;
         float s0 = sc[0] * kq0, s1 = sc[1] * kq1, s2 = sc[2] * kq0, s3 = sc[3] * kq1;
         if (ntok < kPage) {
@@ -409,6 +428,8 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
+    // The merge scratch lives in the ring: wait until every warp is done with it.
+    asm volatile("bar.sync 1, %0;" ::"n"(kWarpsQ8 * 32) : "memory");
     const int hA = 2 * c, hB = 2 * c + 1;
 #pragma unroll
     for (int i = 0; i < KS; ++i) {

@@ -62,6 +62,7 @@ CASES = [
     ([1025, 96], 32, 1, 64),        # MQA with 32 query heads (4 head chunks)
     ([250, 17, 48], 6, 2, 128),     # group of 3
     ([129, 40], 16, 8, 64),         # group of 2
+    ([1023, 1024, 1025, 2049], 16, 4, 128),  # around the 1024-token chunk boundary
 ]
 
 
