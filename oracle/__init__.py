@@ -6,7 +6,9 @@ package and shares no code with it; the two meet only through the seeded input
 generators, which hold none of the method's arithmetic.
 
 The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP); this module
-compiles it with gcc on first use and marshals numpy arrays to it.  The
+compiles it with gcc on first use and marshals numpy arrays to it.  It covers
+the forward (full and sampled rows), the paged decode over 16-bit and 8-bit
+caches, and the backward (full, sampled dQ rows, sampled dK/dV keys).  The
 definition it evaluates is standard attention (Phase 08 page, Lab 01 step 1;
 screna.ai FlashAttention answer): S = scale * Q K^T over the visible keys,
 P = softmax(S) row-wise, O = P V, L = m + ln(sum exp(s - m)).
@@ -64,6 +66,15 @@ def _load():
         lib.oracle_decode_paged_q8.restype = ci
         lib.oracle_e4m3_to_double.argtypes = [ci]
         lib.oracle_e4m3_to_double.restype = cd
+        lib.oracle_attn_bwd.argtypes = [f32p, f32p, f32p, f32p, f64p, f64p, f64p,
+                                        ci, ci, ci, ci, ci, cd, ci, ci, f64p, ci]
+        lib.oracle_attn_bwd.restype = ci
+        lib.oracle_attn_bwd_dq_rows.argtypes = [f32p, f32p, f32p, f32p, f64p, ci, ci, ci, ci, ci,
+                                                cd, ci, ci, f64p, i64p, ci, ci]
+        lib.oracle_attn_bwd_dq_rows.restype = ci
+        lib.oracle_attn_bwd_dkv_rows.argtypes = [f32p, f32p, f32p, f32p, f64p, f64p, ci, ci, ci,
+                                                 ci, ci, cd, ci, ci, f64p, i64p, ci, ci]
+        lib.oracle_attn_bwd_dkv_rows.restype = ci
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ci
         _lib = lib
@@ -138,6 +149,74 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | No
     if rc != 0:
         raise ValueError("oracle_attn_rows failed with code %d" % rc)
     return o, lse
+
+
+def attention_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0,
+                  alibi_slopes=None, nthreads: int | None = None):
+    """Gradients of attention in fp64: q, do [B,Hq,N,d], k, v [B,Hkv,N,d].
+
+    Returns (dQ [B,Hq,N,d], dK [B,Hkv,N,d], dV [B,Hkv,N,d]) in float64, the
+    derivatives of sum(do * O) with O = attention(q, k, v, ...).
+    """
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, Hq, N, d = q.shape
+    _, Hkv, N2, _ = k.shape
+    if N2 != N or do.shape != q.shape or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    dq = np.zeros((B, Hq, N, d), dtype=np.float64)
+    dk = np.zeros((B, Hkv, N, d), dtype=np.float64)
+    dv = np.zeros((B, Hkv, N, d), dtype=np.float64)
+    sl = _slopes(alibi_slopes, Hq)
+    rc = _load().oracle_attn_bwd(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                 _ptr(v, ctypes.c_float), _ptr(do, ctypes.c_float),
+                                 _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                                 _ptr(dv, ctypes.c_double), B, Hq, Hkv, N, d, float(scale),
+                                 int(bool(causal)), int(window), _sp(sl),
+                                 int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd failed with code %d" % rc)
+    return dq, dk, dv
+
+
+def attention_bwd_dq_rows(q, k, v, do, scale: float, causal: bool, rows, window: int = 0,
+                          alibi_slopes=None, nthreads: int | None = None):
+    """dQ of selected rows; rows[r] = (b*Hq + h)*N + i.  Returns [len(rows), d]."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((rows.size, d), dtype=np.float64)
+    sl = _slopes(alibi_slopes, Hq)
+    rc = _load().oracle_attn_bwd_dq_rows(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                         _ptr(v, ctypes.c_float), _ptr(do, ctypes.c_float),
+                                         _ptr(out, ctypes.c_double), B, Hq, Hkv, N, d,
+                                         float(scale), int(bool(causal)), int(window), _sp(sl),
+                                         _ptr(rows, ctypes.c_int64), int(rows.size),
+                                         int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd_dq_rows failed with code %d" % rc)
+    return out
+
+
+def attention_bwd_dkv_rows(q, k, v, do, scale: float, causal: bool, keys, window: int = 0,
+                           alibi_slopes=None, nthreads: int | None = None):
+    """dK and dV of selected keys; keys[r] = (b*Hkv + g)*N + j.  Returns two [len(keys), d]."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
+    dk = np.zeros((keys.size, d), dtype=np.float64)
+    dv = np.zeros((keys.size, d), dtype=np.float64)
+    sl = _slopes(alibi_slopes, Hq)
+    rc = _load().oracle_attn_bwd_dkv_rows(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                          _ptr(v, ctypes.c_float), _ptr(do, ctypes.c_float),
+                                          _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double),
+                                          B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                                          int(window), _sp(sl), _ptr(keys, ctypes.c_int64),
+                                          int(keys.size), int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd_dkv_rows failed with code %d" % rc)
+    return dk, dv
 
 
 def decode_paged(q, k_pages_bf16_bits, v_pages_bf16_bits, block_table, seq_lens,

@@ -39,6 +39,8 @@
  * indirection table), then evaluates the same definition for its one query.
  * oracle_decode_paged_q8 is the same over 8-bit pages (E4M3 or INT8) with one
  * scale per (page, kv head): each element is dequantised to fp64 first.
+ * oracle_attn_bwd (and its sampled forms _dq_rows, _dkv_rows) evaluates the
+ * gradients of the same definition with respect to Q, K and V.
  *
  * Inputs are float (the exact values the GPU sees: fp32, or bf16 upcast) or,
  * for the page pool, raw bf16 bit patterns; arithmetic is double throughout.
@@ -278,6 +280,268 @@ static double e4m3_to_double(uint8_t b)
     if (e == 0) v = ldexp((double)m / 8.0, -6);
     else v = ldexp(1.0 + (double)m / 8.0, e - 7);
     return sign ? -v : v;
+}
+
+/* ------------------------------------------------------------------ backward
+ *
+ * The gradients of the attention of one head with respect to its inputs, given
+ * the output gradient dO ("Phase 08" page, Concepts: FlashAttention backward;
+ * Lab 01 step 6: a backward pass that keeps only O and L; quiz question on
+ * recomputation).  They follow from the chain rule on the definition above:
+ *   P_ij  = exp(s_ij - L_i) for j in V_i, 0 elsewhere
+ *   dV_j  = sum_i P_ij dO_i                       (O = P V)
+ *   dP_ij = dO_i . v_j
+ *   D_i   = sum_j P_ij dP_ij                      (= dO_i . O_i)
+ *   dS_ij = P_ij (dP_ij - D_i)                    (softmax Jacobian)
+ *   dQ_i  = scale * sum_j dS_ij k_j,   dK_j = scale * sum_i dS_ij q_i
+ * The ALiBi bias does not depend on Q or K and drops out of the chain.  With
+ * grouped heads, dK and dV of a K/V head sum the contributions of every query
+ * head of its group.  Nq = Nk = N (self-attention prefill).
+ */
+
+/* Scores of query i (q row qi) against keys [lo, hi) into s[j - lo]; returns
+ * the row's logsumexp. */
+static double score_row(const double *qi, const double *Kd, int lo, int hi, int d, double scale,
+                        double slope, int i, double *s)
+{
+    int j, c;
+    double m = -INFINITY, l = 0.0;
+    for (j = lo; j < hi; ++j) {
+        double acc = 0.0;
+        for (c = 0; c < d; ++c) acc += qi[c] * Kd[(size_t)j * d + c];
+        s[j - lo] = scale * acc + slope * (double)(j - i);
+        if (s[j - lo] > m) m = s[j - lo];
+    }
+    if (hi <= lo) return -INFINITY;
+    for (j = lo; j < hi; ++j) l += exp(s[j - lo] - m);
+    return m + log(l);
+}
+
+/* Full backward: q, dout [B,Hq,N,d], k, v [B,Hkv,N,d] (float); dq [B,Hq,N,d],
+ * dk, dv [B,Hkv,N,d] (double, written).  Materialises P and dS of one head at a
+ * time (N x N doubles each). */
+int oracle_attn_bwd(const float *q, const float *k, const float *v, const float *dout,
+                    double *dq, double *dk, double *dv,
+                    int B, int Hq, int Hkv, int N, int d,
+                    double scale, int causal, int window, const double *slopes,
+                    int nthreads)
+{
+    int b, h, G;
+    double *P, *dS, *Qd, *Kd, *Vd, *dOd;
+    if (check_dims(B, Hq, Hkv, N, N, d) || window < 0) return -1;
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    G = Hq / Hkv;
+    if (nthreads <= 0) nthreads = 1;
+    P = (double *)malloc(sizeof(double) * ((size_t)N * N + 1));
+    dS = (double *)malloc(sizeof(double) * ((size_t)N * N + 1));
+    Qd = (double *)malloc(sizeof(double) * ((size_t)N * d + 1));
+    Kd = (double *)malloc(sizeof(double) * ((size_t)N * d + 1));
+    Vd = (double *)malloc(sizeof(double) * ((size_t)N * d + 1));
+    dOd = (double *)malloc(sizeof(double) * ((size_t)N * d + 1));
+    if (!P || !dS || !Qd || !Kd || !Vd || !dOd) {
+        free(P); free(dS); free(Qd); free(Kd); free(Vd); free(dOd);
+        return -2;
+    }
+    memset(dk, 0, sizeof(double) * (size_t)B * Hkv * N * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * Hkv * N * d);
+
+    for (b = 0; b < B; ++b) {
+        for (h = 0; h < Hq; ++h) {
+            int g = h / G;
+            const size_t qoff = ((size_t)b * Hq + h) * (size_t)N * d;
+            const size_t koff = ((size_t)b * Hkv + g) * (size_t)N * d;
+            const double slope = slopes ? slopes[h] : 0.0;
+            long i;
+            for (i = 0; i < (long)N * d; ++i) {
+                Qd[i] = (double)q[qoff + i];
+                dOd[i] = (double)dout[qoff + i];
+                Kd[i] = (double)k[koff + i];
+                Vd[i] = (double)v[koff + i];
+            }
+            /* Rows: P, dS and dQ. */
+            #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 4)
+            for (i = 0; i < N; ++i) {
+                int j, c, lo, hi;
+                double L, D = 0.0;
+                double *Pi = P + (size_t)i * N, *dSi = dS + (size_t)i * N;
+                double *dqi = dq + qoff + (size_t)i * d;
+                visible_range((int)i, N, causal, window, &lo, &hi);
+                for (j = 0; j < N; ++j) { Pi[j] = 0.0; dSi[j] = 0.0; }
+                L = score_row(Qd + (size_t)i * d, Kd, lo, hi, d, scale, slope, (int)i, Pi + lo);
+                for (j = lo; j < hi; ++j) Pi[j] = exp(Pi[j] - L);
+                for (j = lo; j < hi; ++j) {
+                    double dp = 0.0;
+                    for (c = 0; c < d; ++c) dp += dOd[(size_t)i * d + c] * Vd[(size_t)j * d + c];
+                    dSi[j] = dp;                     /* dP for now */
+                    D += Pi[j] * dp;
+                }
+                for (j = lo; j < hi; ++j) dSi[j] = Pi[j] * (dSi[j] - D);
+                for (c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (j = lo; j < hi; ++j) acc += dSi[j] * Kd[(size_t)j * d + c];
+                    dqi[c] = scale * acc;
+                }
+            }
+            /* Columns: dK and dV of the K/V head, summed over its query heads. */
+            #pragma omp parallel for num_threads(nthreads) schedule(static)
+            for (i = 0; i < N; ++i) {      /* i is the key index here */
+                int r, c;
+                double *dkj = dk + koff + (size_t)i * d, *dvj = dv + koff + (size_t)i * d;
+                for (c = 0; c < d; ++c) {
+                    double ak = 0.0, av = 0.0;
+                    for (r = 0; r < N; ++r) {
+                        ak += dS[(size_t)r * N + i] * Qd[(size_t)r * d + c];
+                        av += P[(size_t)r * N + i] * dOd[(size_t)r * d + c];
+                    }
+                    dkj[c] += scale * ak;
+                    dvj[c] += av;
+                }
+            }
+        }
+    }
+    free(P); free(dS); free(Qd); free(Kd); free(Vd); free(dOd);
+    return 0;
+}
+
+/* dQ for selected rows (rows[r] = (b*Hq + h)*N + i), one row at a time. */
+int oracle_attn_bwd_dq_rows(const float *q, const float *k, const float *v, const float *dout,
+                            double *dq_rows, int B, int Hq, int Hkv, int N, int d,
+                            double scale, int causal, int window, const double *slopes,
+                            const int64_t *rows, int nrows, int nthreads)
+{
+    int r, G, bad = 0;
+    if (check_dims(B, Hq, Hkv, N, N, d) || window < 0 || nrows < 0) return -1;
+    if (!q || !k || !v || !dout || !dq_rows || (!rows && nrows > 0)) return -1;
+    for (r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq * N) return -1;
+    G = Hq / Hkv;
+    if (nthreads <= 0) nthreads = 1;
+    #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) reduction(|:bad)
+    for (r = 0; r < nrows; ++r) {
+        int64_t bh = rows[r] / N;
+        int i = (int)(rows[r] % N), b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+        int j, c, lo, hi;
+        const float *qi = q + (size_t)rows[r] * d, *doi = dout + (size_t)rows[r] * d;
+        const float *kh = k + ((size_t)b * Hkv + g) * (size_t)N * d;
+        const float *vh = v + ((size_t)b * Hkv + g) * (size_t)N * d;
+        double *Kd = (double *)malloc(sizeof(double) * ((size_t)N * d + 1));
+        double *s = (double *)malloc(sizeof(double) * ((size_t)N + 1));
+        double *dp = (double *)malloc(sizeof(double) * ((size_t)N + 1));
+        double qd[512], L, D = 0.0;
+        if (!Kd || !s || !dp || d > 512) { free(Kd); free(s); free(dp); bad = 1; continue; }
+        for (c = 0; c < d; ++c) qd[c] = (double)qi[c];
+        visible_range(i, N, causal, window, &lo, &hi);
+        for (j = lo; j < hi; ++j)
+            for (c = 0; c < d; ++c) Kd[(size_t)j * d + c] = (double)kh[(size_t)j * d + c];
+        L = score_row(qd, Kd, lo, hi, d, scale, slopes ? slopes[h] : 0.0, i, s);
+        for (j = lo; j < hi; ++j) {
+            double acc = 0.0;
+            s[j - lo] = exp(s[j - lo] - L);
+            for (c = 0; c < d; ++c) acc += (double)doi[c] * (double)vh[(size_t)j * d + c];
+            dp[j - lo] = acc;
+            D += s[j - lo] * acc;
+        }
+        for (c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (j = lo; j < hi; ++j) acc += s[j - lo] * (dp[j - lo] - D) * Kd[(size_t)j * d + c];
+            dq_rows[(size_t)r * d + c] = scale * acc;
+        }
+        free(Kd); free(s); free(dp);
+    }
+    return bad ? -2 : 0;
+}
+
+/* dK and dV for selected keys (keys[r] = (b*Hkv + g)*N + j).  Every query row
+ * of the K/V head's group needs its L_i and D_i, computed here from their
+ * definitions for each (b, g) the request touches. */
+int oracle_attn_bwd_dkv_rows(const float *q, const float *k, const float *v, const float *dout,
+                             double *dk_rows, double *dv_rows, int B, int Hq, int Hkv, int N,
+                             int d, double scale, int causal, int window, const double *slopes,
+                             const int64_t *keys, int nkeys, int nthreads)
+{
+    int r, G, bg;
+    double *L, *D;
+    if (check_dims(B, Hq, Hkv, N, N, d) || window < 0 || nkeys < 0) return -1;
+    if (!q || !k || !v || !dout || !dk_rows || !dv_rows || (!keys && nkeys > 0)) return -1;
+    for (r = 0; r < nkeys; ++r)
+        if (keys[r] < 0 || keys[r] >= (int64_t)B * Hkv * N) return -1;
+    G = Hq / Hkv;
+    if (nthreads <= 0) nthreads = 1;
+    L = (double *)malloc(sizeof(double) * ((size_t)G * N + 1));
+    D = (double *)malloc(sizeof(double) * ((size_t)G * N + 1));
+    if (!L || !D) { free(L); free(D); return -2; }
+    for (bg = 0; bg < B * Hkv; ++bg) {
+        int b = bg / Hkv, g = bg % Hkv, need = 0, bad = 0;
+        long t;
+        const float *kh = k + (size_t)bg * N * d, *vh = v + (size_t)bg * N * d;
+        for (r = 0; r < nkeys; ++r) if (keys[r] / N == bg) need = 1;
+        if (!need) continue;
+        /* L_i and D_i of every row of the group's query heads. */
+        #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 8) reduction(|:bad)
+        for (t = 0; t < (long)G * N; ++t) {
+            int hh = (int)(t / N), i = (int)(t % N), h = g * G + hh, j, c, lo, hi;
+            const float *qi = q + (((size_t)b * Hq + h) * N + i) * d;
+            const float *doi = dout + (((size_t)b * Hq + h) * N + i) * d;
+            double *s = (double *)malloc(sizeof(double) * ((size_t)N + 1));
+            double m = -INFINITY, l = 0.0, acc;
+            if (!s) { bad = 1; continue; }
+            visible_range(i, N, causal, window, &lo, &hi);
+            for (j = lo; j < hi; ++j) {
+                acc = 0.0;
+                for (c = 0; c < d; ++c) acc += (double)qi[c] * (double)kh[(size_t)j * d + c];
+                s[j - lo] = scale * acc + (slopes ? slopes[h] : 0.0) * (double)(j - i);
+                if (s[j - lo] > m) m = s[j - lo];
+            }
+            for (j = lo; j < hi; ++j) l += exp(s[j - lo] - m);
+            L[t] = (hi > lo) ? m + log(l) : -INFINITY;
+            D[t] = 0.0;
+            for (j = lo; j < hi; ++j) {
+                acc = 0.0;
+                for (c = 0; c < d; ++c) acc += (double)doi[c] * (double)vh[(size_t)j * d + c];
+                D[t] += exp(s[j - lo] - L[t]) * acc;
+            }
+            free(s);
+        }
+        if (bad) { free(L); free(D); return -2; }
+        #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+        for (r = 0; r < nkeys; ++r) {
+            int j, hh, i, c;
+            double kj[512], vj[512], ak[512], av[512];
+            if (keys[r] / N != bg || d > 512) continue;
+            j = (int)(keys[r] % N);
+            for (c = 0; c < d; ++c) {
+                kj[c] = (double)kh[(size_t)j * d + c];
+                vj[c] = (double)vh[(size_t)j * d + c];
+                ak[c] = 0.0; av[c] = 0.0;
+            }
+            for (hh = 0; hh < G; ++hh) {
+                int h = g * G + hh;
+                for (i = 0; i < N; ++i) {
+                    int lo, hi;
+                    const float *qi = q + (((size_t)b * Hq + h) * N + i) * d;
+                    const float *doi = dout + (((size_t)b * Hq + h) * N + i) * d;
+                    double sc = 0.0, dp = 0.0, p;
+                    visible_range(i, N, causal, window, &lo, &hi);
+                    if (j < lo || j >= hi) continue;
+                    for (c = 0; c < d; ++c) {
+                        sc += (double)qi[c] * kj[c];
+                        dp += (double)doi[c] * vj[c];
+                    }
+                    p = exp(scale * sc + (slopes ? slopes[h] : 0.0) * (double)(j - i) - L[(size_t)hh * N + i]);
+                    for (c = 0; c < d; ++c) {
+                        ak[c] += p * (dp - D[(size_t)hh * N + i]) * (double)qi[c];
+                        av[c] += p * (double)doi[c];
+                    }
+                }
+            }
+            for (c = 0; c < d; ++c) {
+                dk_rows[(size_t)r * d + c] = scale * ak[c];
+                dv_rows[(size_t)r * d + c] = av[c];
+            }
+        }
+    }
+    free(L); free(D);
+    return 0;
 }
 
 /* One 8-bit cache element: fmt 0 = FP8 E4M3, fmt 1 = INT8 (two's complement). */

@@ -18,6 +18,11 @@ the mathematics fix, independently of the oracle's own code:
   power-of-two scales equals the bf16 paged decode of the dequantised cache
   exactly; scale linearity (V's scale multiplies O, K's acts as the softmax
   scale);
+* backward: gradients equal a 4-point central-difference derivative of the
+  forward oracle (inputs on a 2^-10 grid so every perturbed value is exact in
+  float32); the two-key closed form; invariants (dK of a head sums to zero,
+  dV sums to the dO sum, constant V gives dQ = dK = 0); GQA equals MHA with
+  the group's gradients summed; the sampled evaluators equal the full one;
 * mutation checks: plausible one-token mistakes planted in a copy of the
   oracle's C source are each caught by at least one pin.
 """
@@ -559,6 +564,137 @@ def test_q8_decode_rejects_bad_page_ids():
                                np.array([[0, 5]], np.int32), np.array([3], np.int32), scale=1.0)
 
 
+# ------------------------------------------------------------------ backward
+
+
+def _grid_values(rng, shape, denom=1024):
+    """Values k/denom with |k| < denom/2: exact in float32, and so is x +- 2h for
+    h = 2^-12, which the finite-difference stencil below needs."""
+    return (rng.integers(-denom // 2, denom // 2, shape) / denom).astype(np.float32)
+
+
+def _fd_grads(q, k, v, do, scale, causal=False, window=0, alibi_slopes=None):
+    """Gradients of sum(do * O) by the 4-point central stencil (error O(h^4)),
+    from forward evaluations only."""
+    h = 2.0 ** -12
+    dod = do.astype(np.float64)
+
+    def f(a):
+        o, _ = oracle.attention(a[0], a[1], a[2], scale=scale, causal=causal, window=window,
+                                alibi_slopes=alibi_slopes)
+        return float((o * dod).sum())
+
+    out = []
+    for which in range(3):
+        base = [q, k, v]
+        g = np.zeros(base[which].shape)
+        for idx in np.ndindex(base[which].shape):
+            def ev(delta):
+                a = [x.copy() for x in base]
+                a[which][idx] += np.float32(delta)
+                return f(a)
+            g[idx] = (8 * (ev(h) - ev(-h)) - (ev(2 * h) - ev(-2 * h))) / (12 * h)
+        out.append(g)
+    return out
+
+
+@pytest.mark.parametrize("causal,window,alibi,Hq,Hkv", [
+    (False, 0, False, 1, 1), (True, 0, False, 2, 1), (True, 3, True, 2, 2), (False, 0, True, 4, 2)])
+def test_bwd_matches_finite_differences(causal, window, alibi, Hq, Hkv):
+    # The backward is the derivative of the forward: compare with a numerical
+    # derivative of the (separately pinned) forward oracle.
+    rng = np.random.default_rng(31 + Hq + window)
+    B, N, d = 1, 6, 3
+    q, k, v = (_grid_values(rng, (B, Hq, N, d)), _grid_values(rng, (B, Hkv, N, d)),
+               _grid_values(rng, (B, Hkv, N, d)))
+    do = _grid_values(rng, (B, Hq, N, d))
+    slopes = [0.5 * (h + 1) for h in range(Hq)] if alibi else None
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, scale=0.7, causal=causal, window=window,
+                                      alibi_slopes=slopes)
+    fq, fk, fv = _fd_grads(q, k, v, do, 0.7, causal, window, slopes)
+    for got, ref in ((dq, fq), (dk, fk), (dv, fv)):
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-10)
+
+
+def test_bwd_two_keys_closed_form():
+    # One query, two keys: P = (sig, 1 - sig) with sig the logistic of s0 - s1,
+    # dV_j = P_j dO, dS_0 = -dS_1 = sig (1 - sig) dO.(v0 - v1),
+    # dQ = scale dS_0 (k0 - k1), dK_0 = -dK_1 = scale dS_0 q.
+    q = np.array([[[[0.5, -0.25]]]], np.float32)
+    k = np.array([[[[1.0, 0.5], [-0.5, 0.25]]]], np.float32)
+    v = np.array([[[[2.0, 0.0], [0.0, -1.0]]]], np.float32)
+    # a second query row that sees both keys too (non-causal), with zero dO
+    q2 = np.concatenate([q, np.zeros_like(q)], axis=2)
+    do = np.array([[[[1.0, 3.0], [0.0, 0.0]]]], np.float32)
+    scale = 0.8
+    dq, dk, dv = oracle.attention_bwd(q2, k, v, do, scale=scale)
+    s0 = scale * float(q[0, 0, 0] @ k[0, 0, 0]); s1 = scale * float(q[0, 0, 0] @ k[0, 0, 1])
+    sig = 1.0 / (1.0 + math.exp(-(s0 - s1)))
+    dO = do[0, 0, 0].astype(np.float64)
+    ds0 = sig * (1 - sig) * float(dO @ (v[0, 0, 0] - v[0, 0, 1]))
+    np.testing.assert_allclose(dv[0, 0, 0], sig * dO, atol=1e-15)
+    np.testing.assert_allclose(dv[0, 0, 1], (1 - sig) * dO, atol=1e-15)
+    np.testing.assert_allclose(dq[0, 0, 0], scale * ds0 * (k[0, 0, 0] - k[0, 0, 1]), atol=1e-15)
+    np.testing.assert_allclose(dk[0, 0, 0], scale * ds0 * q[0, 0, 0], atol=1e-15)
+    np.testing.assert_allclose(dk[0, 0, 1], -scale * ds0 * q[0, 0, 0], atol=1e-15)
+    assert np.all(dq[0, 0, 1] == 0)
+
+
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 5)])
+def test_bwd_invariants(causal, window):
+    # Adding one vector to every key shifts each score row by a constant, so the
+    # dK of a head sum to zero; every P row sums to one, so the dV sum to the
+    # dO sum; with all values equal, O is constant and dQ = dK = 0.
+    rng = np.random.default_rng(41)
+    B, Hq, Hkv, N, d = 2, 4, 2, 19, 8
+    q, k, v = rand(B, Hq, N, d, rng=rng), rand(B, Hkv, N, d, rng=rng), rand(B, Hkv, N, d, rng=rng)
+    do = rand(B, Hq, N, d, rng=rng)
+    slopes = [0.1 * (h + 1) for h in range(Hq)]
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, scale=0.3, causal=causal, window=window,
+                                      alibi_slopes=slopes)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    G = Hq // Hkv
+    dosum = do.astype(np.float64).reshape(B, Hkv, G, N, d).sum(axis=(2, 3))
+    np.testing.assert_allclose(dv.sum(axis=2), dosum, atol=1e-11)
+    vc = np.broadcast_to(rand(B, Hkv, 1, d, rng=rng), v.shape).copy()
+    dq2, dk2, _ = oracle.attention_bwd(q, k, vc, do, scale=0.3, causal=causal, window=window)
+    assert np.abs(dq2).max() < 1e-13 and np.abs(dk2).max() < 1e-13
+
+
+def test_bwd_gqa_equals_mha_with_summed_heads():
+    rng = np.random.default_rng(42)
+    B, Hq, Hkv, N, d = 1, 6, 2, 11, 4
+    q, k, v = rand(B, Hq, N, d, rng=rng), rand(B, Hkv, N, d, rng=rng), rand(B, Hkv, N, d, rng=rng)
+    do = rand(B, Hq, N, d, rng=rng)
+    G = Hq // Hkv
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, scale=0.4, causal=True)
+    kr, vr = np.repeat(k, G, axis=1), np.repeat(v, G, axis=1)
+    dq2, dk2, dv2 = oracle.attention_bwd(q, kr, vr, do, scale=0.4, causal=True)
+    np.testing.assert_allclose(dq, dq2, atol=1e-14)
+    np.testing.assert_allclose(dk, dk2.reshape(B, Hkv, G, N, d).sum(axis=2), atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, G, N, d).sum(axis=2), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal,window,alibi", [(False, 0, False), (True, 0, False), (True, 7, True)])
+def test_bwd_sampled_evaluators_match_full(causal, window, alibi):
+    rng = np.random.default_rng(43)
+    B, Hq, Hkv, N, d = 2, 4, 2, 37, 16
+    q, k, v = rand(B, Hq, N, d, rng=rng), rand(B, Hkv, N, d, rng=rng), rand(B, Hkv, N, d, rng=rng)
+    do = rand(B, Hq, N, d, rng=rng)
+    slopes = [0.05 * (h + 1) for h in range(Hq)] if alibi else None
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, scale=0.25, causal=causal, window=window,
+                                      alibi_slopes=slopes)
+    rows = np.array([0, 1, 36, 37, 80, B * Hq * N - 1])
+    got = oracle.attention_bwd_dq_rows(q, k, v, do, 0.25, causal, rows, window=window,
+                                       alibi_slopes=slopes)
+    np.testing.assert_allclose(got, dq.reshape(-1, d)[rows], rtol=0, atol=1e-13)
+    keys = np.array([0, 5, 36, 37, 74, B * Hkv * N - 1])
+    gk, gv = oracle.attention_bwd_dkv_rows(q, k, v, do, 0.25, causal, keys, window=window,
+                                           alibi_slopes=slopes)
+    np.testing.assert_allclose(gk, dk.reshape(-1, d)[keys], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gv, dv.reshape(-1, d)[keys], rtol=0, atol=1e-12)
+
+
 # ------------------------------------------------------------- mutations
 
 MUTANTS = {
@@ -616,6 +752,34 @@ def _run_mutant(src_old, src_new, tmp_path, checks):
     finally:
         oracle.build = real_build
         oracle._lib = saved
+
+
+BWD_MUTANTS = {
+    "bwd_drop_D": ("for (j = lo; j < hi; ++j) dSi[j] = Pi[j] * (dSi[j] - D);",
+                   "for (j = lo; j < hi; ++j) dSi[j] = Pi[j] * dSi[j];"),
+    "bwd_dq_unscaled": ("dqi[c] = scale * acc;", "dqi[c] = acc;"),
+    "bwd_dk_uses_P": ("ak += dS[(size_t)r * N + i] * Qd[(size_t)r * d + c];",
+                      "ak += P[(size_t)r * N + i] * Qd[(size_t)r * d + c];"),
+    "bwd_dv_transposed": ("av += P[(size_t)r * N + i] * dOd[(size_t)r * d + c];",
+                          "av += P[(size_t)i * N + r] * dOd[(size_t)r * d + c];"),
+    "bwd_dk_not_summed_over_group": ("dkj[c] += scale * ak;", "dkj[c] = scale * ak;"),
+    "bwd_rows_sign": ("acc += s[j - lo] * (dp[j - lo] - D) * Kd[(size_t)j * d + c];",
+                      "acc += s[j - lo] * (D - dp[j - lo]) * Kd[(size_t)j * d + c];"),
+    "bwd_keys_missing_alibi": ("p = exp(scale * sc + (slopes ? slopes[h] : 0.0) * (double)(j - i) - L[(size_t)hh * N + i]);",
+                               "p = exp(scale * sc - L[(size_t)hh * N + i]);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_bwd_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = BWD_MUTANTS[name]
+    checks = [lambda: test_bwd_matches_finite_differences(True, 3, True, 2, 2),
+              lambda: test_bwd_matches_finite_differences(False, 0, False, 1, 1),
+              lambda: test_bwd_matches_finite_differences(False, 0, True, 4, 2),
+              test_bwd_two_keys_closed_form, test_bwd_gqa_equals_mha_with_summed_heads,
+              lambda: test_bwd_sampled_evaluators_match_full(True, 7, True),
+              lambda: test_bwd_invariants(True, 0)]
+    assert _run_mutant(old, new, tmp_path, checks) > 0, "mutant %s survived every pin" % name
 
 
 @pytest.mark.parametrize("name", sorted(Q8_MUTANTS))
