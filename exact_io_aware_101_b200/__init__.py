@@ -20,13 +20,15 @@ import torch
 
 __all__ = [
     "attn_fwd", "attn_fwd_f32", "attn_decode_paged", "attn_decode_paged_noalloc",
-    "attn_decode_paged_q8", "KV_FORMATS", "decode_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
+    "attn_decode_paged_q8", "KV_FORMATS", "decode_workspace_bytes", "attn_bwd",
+    "bwd_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
     "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
     "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "AttnError",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ext", "attn_fwd_f32_ext",
+                    "attn_bwd_workspace_bytes", "attn_bwd",
                     "attn_decode_workspace_bytes",
                     "attn_decode_paged", "attn_decode_paged_noalloc", "attn_decode_paged_q8",
                     "attn_device_status",
@@ -66,6 +68,11 @@ def library() -> ctypes.CDLL:
         lib.attn_fwd_ext.restype = ci
         lib.attn_fwd_f32_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
         lib.attn_fwd_f32_ext.restype = ci
+        lib.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci]
+        lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
+                                 vp, vp, ctypes.c_size_t, vp]
+        lib.attn_bwd.restype = ci
         lib.attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
@@ -168,6 +175,57 @@ def attn_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, out=
     """fp32 prefill with fp32 arithmetic throughout (same options as attn_fwd)."""
     return _prefill(library().attn_fwd_f32, "attn_fwd_f32", q, k, v, causal, scale, out, lse,
                     torch.float32, window, alibi_slopes)
+
+
+def bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:
+    return int(library().attn_bwd_workspace_bytes(B, Hq, N))
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+             window: int = 0, alibi_slopes=None, dq=None, dk=None, dv=None, workspace=None):
+    """Gradients (dQ, dK, dV) of sum(dout * O) for the bf16 attention.
+
+    q, o, dout [B,Hq,N,d] bf16; k, v [B,Hkv,N,d] bf16; lse [B,Hq,N] fp32 as
+    attn_fwd returned them for the same inputs and options.  Returns bf16
+    (dQ [B,Hq,N,d], dK [B,Hkv,N,d], dV [B,Hkv,N,d]).
+    """
+    for name, t in (("q", q), ("o", o), ("dout", dout)):
+        _check(t, name, torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must have q's shape")
+    if tuple(k.shape) != (B, Hkv, N, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, Hkv, N, d]")
+    if tuple(lse.shape) != (B, Hq, N):
+        raise ValueError("lse must be [B, Hq, N]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", torch.bfloat16, 4)
+    _check(dk, "dk", torch.bfloat16, 4)
+    _check(dv, "dv", torch.bfloat16, 4)
+    slopes_ptr = None
+    if alibi_slopes is not None:
+        alibi_slopes = torch.as_tensor(alibi_slopes, dtype=torch.float32, device=q.device).contiguous()
+        if alibi_slopes.numel() != Hq:
+            raise ValueError("need one ALiBi slope per query head")
+        slopes_ptr = alibi_slopes.data_ptr()
+    need = bwd_workspace_bytes(B, Hq, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace", torch.uint8, 1)
+    rc = library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq,
+                            Hkv, N, d, float(scale), int(bool(causal)), int(window), slopes_ptr,
+                            workspace.data_ptr(), workspace.numel(), _stream(q))
+    _raise(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def decode_workspace_bytes(S: int, Hq: int, d: int, max_blocks: int, page_size: int = 16) -> int:

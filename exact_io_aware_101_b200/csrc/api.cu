@@ -108,6 +108,34 @@ attn_status_t attn_fwd_f32(const float *q, const float *k, const float *v, float
   return attn_fwd_f32_ext(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, nullptr, stream);
 }
 
+size_t attn_bwd_workspace_bytes(int B, int Hq, int N) {
+  if (B <= 0 || Hq <= 0 || N <= 0) return 0;
+  return bwd_workspace_bytes(B, Hq, N);
+}
+
+attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                       const float *lse, const void *dout, void *dq, void *dk, void *dv, int B,
+                       int Hq, int Hkv, int N, int d, float scale, int causal, int window,
+                       const float *alibi_slopes, void *workspace, size_t workspace_bytes,
+                       attn_stream_t stream) {
+  attn_status_t st = check_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
+  if (st != ATTN_OK) return st;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return ATTN_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal) || (alibi_slopes && !aligned4(alibi_slopes)))
+    return ATTN_ERR_INVALID_ARG;
+  if (N <= 0) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(B, Hq, N)) return ATTN_ERR_INVALID_ARG;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal,
+                         window, alibi_slopes, workspace, reinterpret_cast<cudaStream_t>(stream),
+                         status);
+}
+
 size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_blocks, int page_size) {
   if (S <= 0 || Hq <= 0 || max_blocks <= 0 || page_size != 16 || (d != 64 && d != 128)) return 0;
   return decode_workspace_bytes(S, Hq, d, max_blocks);

@@ -1,0 +1,785 @@
+// bwd_sm100.cu -- bf16 exact attention backward on B200 tensor cores.
+//
+// What it computes: dQ, dK, dV of sum(dO * O) for O = softmax(scale*Q K^T
+// [+ mask, + ALiBi]) V, from Q, K, V, the forward's O and logsumexp L, and dO
+// ("Phase 08" page, Concepts: the FlashAttention backward needs only O and L;
+// Lab 01 step 6; quiz page: the backward recomputes the attention matrix tile
+// by tile instead of storing it).  With P = exp(S - L) recomputed per tile:
+//   D_i = rowsum(dO_i * O_i),  dP = dO V^T,  dS = P * (dP - D),
+//   dV = P^T dO,  dK = scale * dS^T Q,  dQ = scale * dS K.
+// The N x N matrices exist one tile at a time, in tensor memory.
+//
+// Three kernels, no atomics (the result does not depend on scheduling):
+//  * bwd_prep: per query row, D = rowsum(dO * O) and L*log2(e), written to a
+//    workspace padded to whole 128-row tiles (+inf / 0 past N, so padded rows
+//    get P = 0 without a mask).
+//  * bwd_dkdv: one CTA per 128-key tile of one (batch, K/V head).  K and V stay
+//    in shared memory; 64-row tiles of Q and dO (and their L, D) stream through
+//    a ring, for every query head of the group.  Per tile:
+//      S^T = K Q^T and dP^T = V dO^T      (128x64x16 MMAs, both K-major)
+//      P^T = 2^(S^T c - L2), dS^T = P^T (dP^T - D)   (CUDA cores, TMEM ld/st)
+//      dV += P^T dO, dK += dS^T Q          (A = P^T / dS^T from TMEM, B MN-major)
+//    S^T and dP^T are double-buffered in TMEM so the tensor pipe computes the
+//    next tile's scores while the current one is exponentiated.
+//  * bwd_dq: one CTA per 128-row Q tile of one (batch, query head); 64-key
+//    tiles of K and V stream through a ring.  S = Q K^T, dP = dO V^T,
+//    dS as above, dQ += dS K (A = dS from TMEM, B = K MN-major).
+// The recomputation costs two more tile products than a single kernel that
+// scatters dQ with atomic adds (7 instead of 5); the FLOP rate reported counts
+// the 5 of the algorithm.
+//
+// Warp roles (both GEMM kernels, 384 threads, as in the forward): warp 0 TMA
+// producer, warp 1 TMEM owner and MMA issuer, warps 4-7 and 8-11 two
+// elementwise warpgroups that split each tile's 64 columns in halves.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace exattn {
+namespace {
+
+constexpr int BT = 128;   // the resident tile: keys (dK/dV kernel) or query rows (dQ kernel)
+constexpr int BS = 64;    // the streamed tile: query rows (dK/dV) or keys (dQ)
+constexpr int NUM_THREADS = 384;
+constexpr int kRegsLow = 72;
+constexpr int kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= NUM_THREADS * 168 && kRegsLow % 8 == 0 &&
+                  kRegsHigh % 8 == 0,
+              "setmaxnreg split must fit the block's launch registers");
+constexpr int kHeadGroup = 8;
+constexpr int CHUNK_BIG = BT * 128;    // 128 rows x 128 bytes: one 64-column block of a resident tile
+constexpr int CHUNK_SMALL = BS * 128;  // 64 rows x 128 bytes: one 64-column block of a streamed tile
+
+// TMEM columns.  The elementwise warpgroup w reads columns [32w, 32w+32) of a
+// 64-column S / dP buffer and writes its bf16 result over the first 16 of them,
+// so the 64 bf16 values of a row sit at columns [0,16) and [32,48).
+__device__ __forceinline__ uint32_t col_s(int buf) { return static_cast<uint32_t>(buf) * 64; }
+__device__ __forceinline__ uint32_t col_dp(int buf) { return 128 + static_cast<uint32_t>(buf) * 64; }
+constexpr uint32_t kColAcc0 = 256;  // dV (dK/dV kernel) or dQ (dQ kernel)
+constexpr uint32_t kColAcc1 = 384;  // dK (dK/dV kernel)
+__device__ __forceinline__ uint32_t packed_col(int ks) {  // k-step of 16 -> 8 bf16 columns
+  return ks < 2 ? ks * 8 : 32 + (ks - 2) * 8;
+}
+
+template <int D>
+struct BCfg {
+  static constexpr int CH = D / 64;
+  static constexpr int BIG = BT * D * 2;
+  static constexpr int SMALL = BS * D * 2;
+  // dK/dV kernel: K, V resident; stages of {Q, dO, L2[64], D[64]}.
+  static constexpr int KV_NST = 4;
+  static constexpr int KV_STAGE = ((2 * SMALL + 2 * BS * 4) + 1023) / 1024 * 1024;
+  static constexpr int KV_RING_OFF = 2 * BIG;
+  static constexpr int KV_BAR_OFF = KV_RING_OFF + KV_NST * KV_STAGE;
+  // At least 116 KiB so that one CTA fills an SM: each CTA allocates all 512
+  // TMEM columns.
+  static constexpr int MIN_SMEM = 116 * 1024;
+  static constexpr int KV_SMEM = (KV_BAR_OFF + 2048 > MIN_SMEM) ? KV_BAR_OFF + 2048 : MIN_SMEM;
+  // dQ kernel: Q, dO resident; slots of one K or V tile.
+  static constexpr int Q_NST = (D == 64) ? 10 : 6;
+  static constexpr int Q_RING_OFF = 2 * BIG;
+  static constexpr int Q_BAR_OFF = Q_RING_OFF + Q_NST * SMALL;
+  static constexpr int Q_SMEM = (Q_BAR_OFF + 2048 > MIN_SMEM) ? Q_BAR_OFF + 2048 : MIN_SMEM;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BS, false, false);
+  static constexpr uint32_t IDESC_G = idesc_bf16_f32(BT, D, false, true);
+};
+
+struct BBars {
+  uint64_t full[10];
+  uint64_t empty[10];
+  uint64_t res_full;  // the resident tiles (K,V or Q,dO)
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct BwdParams {
+  void *dq, *dk, *dv;
+  const float *l2;    // [B*Hq][Npad]: L * log2(e), +inf past N
+  const float *dvec;  // [B*Hq][Npad]: rowsum(dO * O), 0 past N
+  unsigned *status;
+  int B, Hq, Hkv, N, Npad;
+  float scale, scale_log2;
+  int causal, window;
+  const float *slopes;  // per query head (ALiBi variant)
+};
+
+// Per row: D = rowsum(dO * O) (fp32 from the bf16 values) and L * log2(e); one
+// warp per row, rows past N padded.
+template <int D>
+__global__ void __launch_bounds__(256)
+    bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dout,
+                    const float *__restrict__ lse, float *__restrict__ l2,
+                    float *__restrict__ dvec, int BH, int N, int Npad) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(BH) * Npad) return;
+  const int bh = static_cast<int>(row / Npad), i = static_cast<int>(row % Npad);
+  if (i >= N) {
+    if (lane == 0) {
+      l2[row] = INFINITY;
+      dvec[row] = 0.f;
+    }
+    return;
+  }
+  const size_t src = (static_cast<size_t>(bh) * N + i) * D;
+  float acc = 0.f;
+  constexpr int EPL = D / 32;  // elements per lane: 4 (d=128) or 2 (d=64)
+  if constexpr (EPL == 4) {
+    const uint2 a = *reinterpret_cast<const uint2 *>(o + src + lane * 4);
+    const uint2 b = *reinterpret_cast<const uint2 *>(dout + src + lane * 4);
+    const uint32_t aw[2] = {a.x, a.y}, bw[2] = {b.x, b.y};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      acc = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(bw[e] & 0xffff0000u), acc);
+    }
+  } else {
+    const uint32_t a = *reinterpret_cast<const uint32_t *>(o + src + lane * 2);
+    const uint32_t b = *reinterpret_cast<const uint32_t *>(dout + src + lane * 2);
+    acc = fmaf(__uint_as_float(a << 16), __uint_as_float(b << 16), acc);
+    acc = fmaf(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u), acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    dvec[row] = acc;
+    l2[row] = lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f;
+  }
+}
+
+// 32 columns of one row: P = 2^(s*c + bias - l2), dS = P * (dp - dd), both
+// rounded to bf16 and packed in column pairs.  vis(i) masks a column.
+template <bool kAlibi, bool kMasked, bool kWantP, typename Vis>
+__device__ __forceinline__ void grad_cols(const uint32_t (&sv)[32], const uint32_t (&dpv)[32],
+                                          const float *l2c, const float *ddc, float l2s, float dds,
+                                          bool per_col, float c, float bias0, float bias_step,
+                                          Vis vis, uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    float p[2], ds[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float lv = per_col ? l2c[i + e] : l2s;
+      const float dv = per_col ? ddc[i + e] : dds;
+      float x = fmaf(__uint_as_float(sv[i + e]), c, -lv);
+      if (kAlibi) x = fmaf(bias_step, static_cast<float>(i + e), x + bias0);
+      float pe = ex2(x);
+      if (kMasked && !vis(i + e)) pe = 0.f;
+      p[e] = pe;
+      ds[e] = pe * (__uint_as_float(dpv[i + e]) - dv);
+    }
+    if (kWantP) pk[i >> 1] = pack_bf16x2(p[0], p[1]);
+    dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
+  }
+}
+
+// ------------------------------------------------------------------ dK / dV
+template <int D, bool kAlibi>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using C = BCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sK = smem;
+  uint8_t *sV = smem + C::BIG;
+  uint8_t *sRing = smem + C::KV_RING_OFF;
+  BBars *bars = reinterpret_cast<BBars *>(smem + C::KV_BAR_OFF);
+  volatile int *abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: 128-key tile kt of (batch, K/V head).  Causal: heaviest
+  // tiles (smallest kt: most query tiles) first within groups of heads.
+  const int nkt = (p.N + BT - 1) / BT;
+  const int BHk = p.B * p.Hkv;
+  int kt, bhk;
+  {
+    const int lin = static_cast<int>(blockIdx.x);
+    if (!p.causal) {
+      bhk = lin / nkt;
+      kt = lin % nkt;
+    } else {
+      const int grp = lin / (kHeadGroup * nkt);
+      const int first = grp * kHeadGroup;
+      const int hg = min(kHeadGroup, BHk - first);
+      const int rr = lin - grp * kHeadGroup * nkt;
+      kt = rr / hg;
+      bhk = first + rr % hg;
+    }
+  }
+  const int b = bhk / p.Hkv, g = bhk % p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  const int k0 = kt * BT;
+  const int nqt = (p.N + BS - 1) / BS;
+  // Query tiles [qs, qe) that can see a key of this tile.
+  const int qs = p.causal ? k0 / BS : 0;
+  const int qe = p.window > 0 ? min(nqt, (k0 + BT - 1 + p.window - 1) / BS + 1) : nqt;
+  const int nq = max(0, qe - qs);
+  const int n_items = G * nq;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::KV_NST; ++i) {
+      mbar_init(&bars->full[i], 1);
+      mbar_init(&bars->empty[i], 1);
+    }
+    mbar_init(&bars->res_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 256);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    regs_dec<kRegsLow>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(&bars->res_full, 2 * C::BIG);
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_3d(sK + c * CHUNK_BIG, &tm_k, &bars->res_full, 64 * c, k0, bhk);
+        tma_load_3d(sV + c * CHUNK_BIG, &tm_v, &bars->res_full, 64 * c, k0, bhk);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_items; ++it) {
+        const int slot = it % C::KV_NST, round = it / C::KV_NST;
+        if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status)) break;
+        const int hq = g * G + it / nq;
+        const int q0 = (qs + it % nq) * BS;
+        const int zq = b * p.Hq + hq;
+        uint8_t *st = sRing + slot * C::KV_STAGE;
+        mbar_arrive_expect_tx(&bars->full[slot], 2 * C::SMALL + 2 * BS * 4);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_3d(st + c * CHUNK_SMALL, &tm_q, &bars->full[slot], 64 * c, q0, zq);
+          tma_load_3d(st + C::SMALL + c * CHUNK_SMALL, &tm_do, &bars->full[slot], 64 * c, q0, zq);
+        }
+        const size_t vo = static_cast<size_t>(zq) * p.Npad + q0;
+        bulk_load(st + 2 * C::SMALL, p.l2 + vo, BS * 4, &bars->full[slot]);
+        bulk_load(st + 2 * C::SMALL + BS * 4, p.dvec + vo, BS * 4, &bars->full[slot]);
+        issued = it + 1;
+      }
+      mbar_wait_drain(&bars->res_full, 0, p.status);
+      for (int i = max(0, issued - C::KV_NST); i < issued; ++i)
+        mbar_wait_drain(&bars->full[i % C::KV_NST], (i / C::KV_NST) & 1, p.status);
+    }
+  } else if (warp == 1) {
+    // ================================================================== MMA
+    regs_dec<kRegsLow>();
+    if (lane == 0) {
+      const uint32_t ring = smem_u32(sRing);
+      const uint64_t kdesc = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t vdesc = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t qk0 = sdesc_sw128(ring, 16, 1024);                    // Q, K-major
+      const uint64_t dok0 = sdesc_sw128(ring + C::SMALL, 16, 1024);        // dO, K-major
+      const uint64_t qmn0 = sdesc_sw128(ring, CHUNK_SMALL, 1024);          // Q, MN-major
+      const uint64_t domn0 = sdesc_sw128(ring + C::SMALL, CHUNK_SMALL, 1024);  // dO, MN-major
+      auto wait_full = [&](int it) {
+        return mbar_wait(&bars->full[it % C::KV_NST], (it / C::KV_NST) & 1, abort_flag, p.status);
+      };
+      auto issue_st = [&](int buf, int it) {  // S^T = K Q^T, dP^T = V dO^T
+        const uint64_t so = static_cast<uint64_t>((it % C::KV_NST) * C::KV_STAGE) >> 4;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t oa = ((ks >> 2) * CHUNK_BIG + (ks & 3) * 32) >> 4;
+          const uint64_t ob = ((ks >> 2) * CHUNK_SMALL + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + col_s(buf), kdesc + oa, qk0 + so + ob, C::IDESC_S, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t oa = ((ks >> 2) * CHUNK_BIG + (ks & 3) * 32) >> 4;
+          const uint64_t ob = ((ks >> 2) * CHUNK_SMALL + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + col_dp(buf), vdesc + oa, dok0 + so + ob, C::IDESC_S, ks > 0);
+        }
+      };
+      auto issue_grad = [&](int buf, int it) {  // dV += P^T dO, dK += dS^T Q
+        const uint64_t so = static_cast<uint64_t>((it % C::KV_NST) * C::KV_STAGE) >> 4;
+#pragma unroll
+        for (int ks = 0; ks < BS / 16; ++ks)
+          mma_ts(tmem + kColAcc0, tmem + col_s(buf) + packed_col(ks), domn0 + so + ((ks * 2048) >> 4),
+                 C::IDESC_G, (it > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < BS / 16; ++ks)
+          mma_ts(tmem + kColAcc1, tmem + col_dp(buf) + packed_col(ks), qmn0 + so + ((ks * 2048) >> 4),
+                 C::IDESC_G, (it > 0 || ks > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&bars->res_full, 0, abort_flag, p.status);
+      for (int it = 0; ok && it < 2 && it < n_items; ++it) {
+        if (!(ok = wait_full(it))) break;
+        tc_fence_after();
+        issue_st(it, it);
+        tc_commit(&bars->s_full[it]);
+      }
+      for (int it = 0; ok && it < n_items; ++it) {
+        const int buf = it & 1;
+        if (!(ok = mbar_wait(&bars->p_full[buf], (it >> 1) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_grad(buf, it);
+        tc_commit(&bars->empty[it % C::KV_NST]);  // Q/dO stage consumed
+        if (it + 2 < n_items) {
+          if (!(ok = wait_full(it + 2))) break;
+          tc_fence_after();
+          // In order after the gradient MMAs above, which read P^T / dS^T from
+          // these columns: no completion wait needed.
+          issue_st(buf, it + 2);
+          tc_commit(&bars->s_full[buf]);
+        }
+      }
+      tc_commit(&bars->mma_done);
+      mbar_wait_drain(&bars->mma_done, 0, p.status);
+    }
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();
+  } else {
+    // ============================================================ elementwise
+    regs_inc<kRegsHigh>();
+    const int wg = (warp - 4) >> 2;      // column half of each tile
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;   // key row in the tile
+    const int key = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_items; ++it) {
+      const int buf = it & 1;
+      ok = mbar_wait(&bars->s_full[buf], (it >> 1) & 1, abort_flag, p.status) &&
+           mbar_wait(&bars->full[it % C::KV_NST], (it / C::KV_NST) & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int hq = g * G + it / nq;
+      const int qb = (qs + it % nq) * BS + 32 * wg;  // first query of this thread's 32 columns
+      const uint8_t *st = sRing + (it % C::KV_NST) * C::KV_STAGE;
+      const float *l2c = reinterpret_cast<const float *>(st + 2 * C::SMALL) + 32 * wg;
+      const float *ddc = l2c + BS;
+      uint32_t sv[32], dpv[32];
+      tmem_ld32(tmem + lane_off + col_s(buf) + 32 * wg, sv);
+      tmem_ld32(tmem + lane_off + col_dp(buf) + 32 * wg, dpv);
+      tmem_ld_wait(sv);
+      tmem_ld_wait(dpv);
+      // ALiBi bias slope*(key - query) in log2 units; column i has query qb + i.
+      const float slope2 = kAlibi ? p.slopes[hq] * 1.4426950408889634f : 0.f;
+      const float bias0 = slope2 * static_cast<float>(key - qb);
+      // Visible: key <= query (causal) and query - key < window.
+      auto vis = [&](int i) {
+        const int qq = qb + i;
+        return (!p.causal || key <= qq) && (p.window <= 0 || qq - key < p.window);
+      };
+      const bool full_vis = (!p.causal || key <= qb) && (p.window <= 0 || qb + 31 - key < p.window);
+      const bool masked = !__all_sync(0xffffffffu, full_vis);
+      uint32_t pk[16], dk[16];
+      if (masked)
+        grad_cols<kAlibi, true, true>(sv, dpv, l2c, ddc, 0.f, 0.f, true, c, bias0, -slope2, vis, pk, dk);
+      else
+        grad_cols<kAlibi, false, true>(sv, dpv, l2c, ddc, 0.f, 0.f, true, c, bias0, -slope2, vis, pk, dk);
+      tmem_st16(tmem + lane_off + col_s(buf) + 32 * wg, pk);
+      tmem_st16(tmem + lane_off + col_dp(buf) + 32 * wg, dk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[buf]);
+    }
+    if (ok && n_items > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort_flag, p.status));
+      if (ok) {
+        tc_fence_after();
+        // Warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
+        const uint32_t acc = tmem + lane_off + (wg == 0 ? kColAcc0 : kColAcc1);
+        const float mul = wg == 0 ? 1.f : p.scale;
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(wg == 0 ? p.dv : p.dk) +
+                             (static_cast<size_t>(bhk) * p.N + (key < p.N ? key : 0)) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(acc + cc * 32, v);
+          tmem_ld_wait(v);
+          uint32_t pkd[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            pkd[i >> 1] = pack_bf16x2(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
+          if (key < p.N) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              d4[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+          }
+        }
+      }
+    } else if (ok && n_items == 0) {
+      // No query sees this tile (cannot happen for keys < N): zero gradients.
+      __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(wg == 0 ? p.dv : p.dk) +
+                           (static_cast<size_t>(bhk) * p.N + (key < p.N ? key : 0)) * D;
+      if (key < p.N)
+        for (int cc = 0; cc < D; cc += 8) *reinterpret_cast<uint4 *>(dst + cc) = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------------- dQ
+template <int D, bool kAlibi>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p) {
+  using C = BCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem;
+  uint8_t *sdO = smem + C::BIG;
+  uint8_t *sRing = smem + C::Q_RING_OFF;
+  BBars *bars = reinterpret_cast<BBars *>(smem + C::Q_BAR_OFF);
+  volatile int *abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: 128-row Q tile of (batch, query head); causal: heaviest first.
+  const int nqt = (p.N + BT - 1) / BT;
+  const int BH = p.B * p.Hq;
+  int qt, bh;
+  {
+    const int lin = static_cast<int>(blockIdx.x);
+    if (!p.causal) {
+      bh = lin / nqt;
+      qt = lin % nqt;
+    } else {
+      const int grp = lin / (kHeadGroup * nqt);
+      const int first = grp * kHeadGroup;
+      const int hg = min(kHeadGroup, BH - first);
+      const int rr = lin - grp * kHeadGroup * nqt;
+      qt = nqt - 1 - rr / hg;
+      bh = first + rr % hg;
+    }
+  }
+  const int b = bh / p.Hq, hq = bh % p.Hq;
+  const int bhk = b * p.Hkv + hq / (p.Hq / p.Hkv);
+  const int row0 = qt * BT;
+  const int nkt = (p.N + BS - 1) / BS;
+  const int je = p.causal ? min((row0 + BT - 1) / BS + 1, nkt) : nkt;
+  const int js = p.window > 0 ? max(0, row0 - p.window + 1) / BS : 0;
+  const int n_items = max(0, je - js);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::Q_NST; ++i) {
+      mbar_init(&bars->full[i], 1);
+      mbar_init(&bars->empty[i], 1);
+    }
+    mbar_init(&bars->res_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 256);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    regs_dec<kRegsLow>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bars->res_full, 2 * C::BIG);
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_3d(sQ + c * CHUNK_BIG, &tm_q, &bars->res_full, 64 * c, row0, bh);
+        tma_load_3d(sdO + c * CHUNK_BIG, &tm_do, &bars->res_full, 64 * c, row0, bh);
+      }
+      int issued = 0;
+      for (int i = 0; i < 2 * n_items; ++i) {
+        const int slot = i % C::Q_NST, round = i / C::Q_NST;
+        if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&bars->full[slot], C::SMALL);
+        const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sRing + slot * C::SMALL + c * CHUNK_SMALL, map, &bars->full[slot], 64 * c,
+                      (js + (i >> 1)) * BS, bhk);
+        issued = i + 1;
+      }
+      mbar_wait_drain(&bars->res_full, 0, p.status);
+      for (int i = max(0, issued - C::Q_NST); i < issued; ++i)
+        mbar_wait_drain(&bars->full[i % C::Q_NST], (i / C::Q_NST) & 1, p.status);
+    }
+  } else if (warp == 1) {
+    // ================================================================== MMA
+    regs_dec<kRegsLow>();
+    if (lane == 0) {
+      const uint32_t ring = smem_u32(sRing);
+      const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dodesc = sdesc_sw128(smem_u32(sdO), 16, 1024);
+      const uint64_t rk0 = sdesc_sw128(ring, 16, 1024);             // K or V, K-major
+      const uint64_t rmn0 = sdesc_sw128(ring, CHUNK_SMALL, 1024);   // K, MN-major
+      auto slot_off = [](int i) { return static_cast<uint64_t>((i % C::Q_NST) * C::SMALL) >> 4; };
+      auto wait_full = [&](int i) {
+        return mbar_wait(&bars->full[i % C::Q_NST], (i / C::Q_NST) & 1, abort_flag, p.status);
+      };
+      auto issue_s = [&](int buf, int jj) {  // S = Q K^T, dP = dO V^T
+        const uint64_t sk = slot_off(2 * jj), sv = slot_off(2 * jj + 1);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t oa = ((ks >> 2) * CHUNK_BIG + (ks & 3) * 32) >> 4;
+          const uint64_t ob = ((ks >> 2) * CHUNK_SMALL + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + col_s(buf), qdesc + oa, rk0 + sk + ob, C::IDESC_S, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t oa = ((ks >> 2) * CHUNK_BIG + (ks & 3) * 32) >> 4;
+          const uint64_t ob = ((ks >> 2) * CHUNK_SMALL + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + col_dp(buf), dodesc + oa, rk0 + sv + ob, C::IDESC_S, ks > 0);
+        }
+      };
+      auto issue_dq = [&](int buf, int jj) {  // dQ += dS K
+        const uint64_t sk = slot_off(2 * jj);
+#pragma unroll
+        for (int ks = 0; ks < BS / 16; ++ks)
+          mma_ts(tmem + kColAcc0, tmem + col_s(buf) + packed_col(ks), rmn0 + sk + ((ks * 2048) >> 4),
+                 C::IDESC_G, (jj > 0 || ks > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&bars->res_full, 0, abort_flag, p.status);
+      for (int jj = 0; ok && jj < 2 && jj < n_items; ++jj) {
+        if (!(ok = wait_full(2 * jj) && wait_full(2 * jj + 1))) break;
+        tc_fence_after();
+        issue_s(jj, jj);
+        tc_commit(&bars->s_full[jj]);
+        tc_commit(&bars->empty[(2 * jj + 1) % C::Q_NST]);  // V(jj) consumed by dP
+      }
+      for (int jj = 0; ok && jj < n_items; ++jj) {
+        const int buf = jj & 1;
+        if (!(ok = mbar_wait(&bars->p_full[buf], (jj >> 1) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_dq(buf, jj);
+        tc_commit(&bars->empty[(2 * jj) % C::Q_NST]);  // K(jj) consumed
+        if (jj + 2 < n_items) {
+          if (!(ok = wait_full(2 * jj + 4) && wait_full(2 * jj + 5))) break;
+          tc_fence_after();
+          issue_s(buf, jj + 2);  // in order after dQ(jj), which reads dS from these columns
+          tc_commit(&bars->s_full[buf]);
+          tc_commit(&bars->empty[(2 * jj + 5) % C::Q_NST]);
+        }
+      }
+      tc_commit(&bars->mma_done);
+      mbar_wait_drain(&bars->mma_done, 0, p.status);
+    }
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();
+  } else {
+    // ============================================================ elementwise
+    regs_inc<kRegsHigh>();
+    const int wg = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int row = row0 + r;  // query row; rows >= N have l2 = +inf, so P = 0
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c = p.scale_log2;
+    const float l2s = p.l2[static_cast<size_t>(bh) * p.Npad + row];
+    const float dds = p.dvec[static_cast<size_t>(bh) * p.Npad + row];
+    const float slope2 = kAlibi ? p.slopes[hq] * 1.4426950408889634f : 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < n_items; ++jj) {
+      const int buf = jj & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[buf], (jj >> 1) & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      const int kb = (js + jj) * BS + 32 * wg;  // first key of this thread's 32 columns
+      uint32_t sv[32], dpv[32];
+      tmem_ld32(tmem + lane_off + col_s(buf) + 32 * wg, sv);
+      tmem_ld32(tmem + lane_off + col_dp(buf) + 32 * wg, dpv);
+      tmem_ld_wait(sv);
+      tmem_ld_wait(dpv);
+      const float bias0 = slope2 * static_cast<float>(kb - row);
+      auto vis = [&](int i) {
+        const int kk = kb + i;
+        return kk < p.N && (!p.causal || kk <= row) && (p.window <= 0 || row - kk < p.window);
+      };
+      const bool full_vis = kb + 31 < p.N && (!p.causal || kb + 31 <= row) &&
+                            (p.window <= 0 || row - kb < p.window);
+      const bool masked = !__all_sync(0xffffffffu, full_vis);
+      uint32_t pk[16], dk[16];
+      if (masked)
+        grad_cols<kAlibi, true, false>(sv, dpv, nullptr, nullptr, l2s, dds, false, c, bias0, slope2, vis, pk, dk);
+      else
+        grad_cols<kAlibi, false, false>(sv, dpv, nullptr, nullptr, l2s, dds, false, c, bias0, slope2, vis, pk, dk);
+      tmem_st16(tmem + lane_off + col_s(buf) + 32 * wg, dk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[buf]);
+    }
+    if (ok && n_items > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort_flag, p.status));
+      if (ok) {
+        tc_fence_after();
+        // Each warpgroup writes half of the row's D columns.
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.dq) +
+                             (static_cast<size_t>(bh) * p.N + (row < p.N ? row : 0)) * D;
+#pragma unroll
+        for (int cc = wg * (D / 64); cc < (wg + 1) * (D / 64); ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + kColAcc0 + cc * 32, v);
+          tmem_ld_wait(v);
+          uint32_t pkd[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            pkd[i >> 1] = pack_bf16x2(__uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale);
+          if (row < p.N) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              d4[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// [BH][N][D] bf16 as a 3-D tensor (D, N, BH); boxes of 64 columns x rows x 1, 128B swizzle.
+bool make_map_rows(CUtensorMap *map, const void *base, int D, int N, int BH, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool kAlibi>
+attn_status_t launch_bwd(const void *q, const void *k, const void *v, const void *dout,
+                         const BwdParams &prm, cudaStream_t stream) {
+  using C = BCfg<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(bwd_dkdv_kernel<D, kAlibi>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(bwd_dq_kernel<D, kAlibi>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::Q_SMEM);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  const int BHq = prm.B * prm.Hq, BHk = prm.B * prm.Hkv;
+  CUtensorMap k_big, v_big, q_small, do_small, q_big, do_big, k_small, v_small;
+  if (!make_map_rows(&k_big, k, D, prm.N, BHk, BT) || !make_map_rows(&v_big, v, D, prm.N, BHk, BT) ||
+      !make_map_rows(&q_small, q, D, prm.N, BHq, BS) ||
+      !make_map_rows(&do_small, dout, D, prm.N, BHq, BS) ||
+      !make_map_rows(&q_big, q, D, prm.N, BHq, BT) || !make_map_rows(&do_big, dout, D, prm.N, BHq, BT) ||
+      !make_map_rows(&k_small, k, D, prm.N, BHk, BS) || !make_map_rows(&v_small, v, D, prm.N, BHk, BS))
+    return ATTN_ERR_CUDA;
+  const long long kv_ctas = static_cast<long long>((prm.N + BT - 1) / BT) * BHk;
+  const long long q_ctas = static_cast<long long>((prm.N + BT - 1) / BT) * BHq;
+  if (kv_ctas > 0x7fffffffLL || q_ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  bwd_dkdv_kernel<D, kAlibi><<<static_cast<unsigned>(kv_ctas), NUM_THREADS, C::KV_SMEM, stream>>>(
+      k_big, v_big, q_small, do_small, prm);
+  bwd_dq_kernel<D, kAlibi><<<static_cast<unsigned>(q_ctas), NUM_THREADS, C::Q_SMEM, stream>>>(
+      q_big, do_big, k_small, v_small, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+int bwd_padded_rows(int N) { return (N + BT - 1) / BT * BT; }
+
+size_t bwd_workspace_bytes(int B, int Hq, int N) {
+  const size_t n = static_cast<size_t>(B) * Hq * bwd_padded_rows(N) * sizeof(float);
+  return 2 * ((n + 255) & ~static_cast<size_t>(255));
+}
+
+attn_status_t launch_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                              int window, const float *slopes, void *workspace,
+                              cudaStream_t stream, unsigned *status) {
+  BwdParams prm;
+  prm.dq = dq;
+  prm.dk = dk;
+  prm.dv = dv;
+  prm.Npad = bwd_padded_rows(N);
+  const size_t n = static_cast<size_t>(B) * Hq * prm.Npad;
+  float *l2 = static_cast<float *>(workspace);
+  float *dvec = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                          ((n * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+  prm.l2 = l2;
+  prm.dvec = dvec;
+  prm.status = status;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.N = N;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.causal = causal ? 1 : 0;
+  prm.window = window;
+  prm.slopes = slopes;
+  const long long rows = static_cast<long long>(n);
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (d == 128)
+    bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, l2,
+        dvec, B * Hq, N, prm.Npad);
+  else if (d == 64)
+    bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, l2,
+        dvec, B * Hq, N, prm.Npad);
+  else
+    return ATTN_ERR_UNSUPPORTED;
+  const bool alibi = slopes != nullptr;
+  if (d == 128)
+    return alibi ? launch_bwd<128, true>(q, k, v, dout, prm, stream)
+                 : launch_bwd<128, false>(q, k, v, dout, prm, stream);
+  return alibi ? launch_bwd<64, true>(q, k, v, dout, prm, stream)
+               : launch_bwd<64, false>(q, k, v, dout, prm, stream);
+}
+
+}  // namespace exattn

@@ -47,6 +47,15 @@ attn_status_t launch_decode_paged_q8(const void *q, const void *k_pages, const v
                                      int num_pages, float scale, void *workspace,
                                      cudaStream_t stream, unsigned *status);
 
+// Backward: workspace (L*log2e and rowsum(dO*O) per query row, padded to whole
+// 128-row tiles) and the three-kernel launch.
+size_t bwd_workspace_bytes(int B, int Hq, int N);
+attn_status_t launch_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                              int window, const float *slopes, void *workspace,
+                              cudaStream_t stream, unsigned *status);
+
 // cuTensorMapEncodeTiled, or nullptr if the driver does not provide it.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 

@@ -118,6 +118,36 @@ EXATTN_API attn_status_t attn_fwd_f32_ext(const float *q, const float *k, const 
                                           const float *alibi_slopes, attn_stream_t stream);
 
 /*
+ * attn_bwd -- gradients of the bf16 attention above (Phase 08 page, Concepts:
+ * the FlashAttention backward needs only the output O and the logsumexp L;
+ * Lab 01 step 6 and Extensions: the backward pass).  For the scalar
+ * sum(dO * O), with P = softmax(scale * Q K^T [mask] [+ALiBi]) recomputed tile by
+ * tile from L (never stored):
+ *   D = rowsum(dO * O), dP = dO V^T, dS = P * (dP - D),
+ *   dV = P^T dO,  dK = scale * dS^T Q,  dQ = scale * dS K.
+ * With grouped heads, dK and dV of a K/V head sum over its query heads.
+ *
+ *   q, o, dout   [B, Hq, N, d] bf16 (o and lse as attn_fwd / attn_fwd_ext
+ *                wrote them for the same q, k, v and options)
+ *   k, v         [B, Hkv, N, d] bf16
+ *   lse          [B, Hq, N] float32
+ *   dq           [B, Hq, N, d] bf16 (out)     dk, dv  [B, Hkv, N, d] bf16 (out)
+ *   causal, window, alibi_slopes   as for attn_fwd_ext
+ *   workspace    device scratch of at least attn_bwd_workspace_bytes(B, Hq, N)
+ *                bytes, owned by the caller; no initialisation needed.
+ * The result is deterministic: no atomics, every output element is written by
+ * one thread.  Errors as for attn_fwd_ext, plus ATTN_ERR_INVALID_ARG for a
+ * workspace that is too small.
+ */
+EXATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N);
+EXATTN_API attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                                  const float *lse, const void *dout, void *dq, void *dk,
+                                  void *dv, int B, int Hq, int Hkv, int N, int d, float scale,
+                                  int causal, int window, const float *alibi_slopes,
+                                  void *workspace, size_t workspace_bytes,
+                                  attn_stream_t stream);
+
+/*
  * attn_decode_workspace_bytes -- bytes of device workspace attn_decode_paged
  * needs for S sequences, Hq query heads, head dim d and at most max_blocks
  * pages per sequence.  Returns 0 for invalid sizes.
