@@ -66,6 +66,9 @@ def _load():
         lib.oracle_decode_paged_q8.restype = ci
         lib.oracle_e4m3_to_double.argtypes = [ci]
         lib.oracle_e4m3_to_double.restype = cd
+        lib.oracle_prefill_paged.argtypes = [f32p, u16p, u16p, i32p, i32p, i32p, f64p, f64p,
+                                             ci, ci, ci, ci, ci, ci, ci, cd, ci]
+        lib.oracle_prefill_paged.restype = ci
         lib.oracle_attn_bwd.argtypes = [f32p, f32p, f32p, f32p, f64p, f64p, f64p,
                                         ci, ci, ci, ci, ci, cd, ci, ci, f64p, ci]
         lib.oracle_attn_bwd.restype = ci
@@ -148,6 +151,39 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | No
                                   int(nthreads or max_threads()))
     if rc != 0:
         raise ValueError("oracle_attn_rows failed with code %d" % rc)
+    return o, lse
+
+
+def prefill_paged(q, k_pages_bf16_bits, v_pages_bf16_bits, block_table, seq_lens, cu_q,
+                  scale: float, nthreads: int | None = None):
+    """Chunked prefill over a paged cache in fp64.
+
+    q [T,Hq,d] (float32 values, token-major; sequence s owns rows
+    cu_q[s]..cu_q[s+1]-1, the last cu_q[s+1]-cu_q[s] of its seq_lens[s]
+    positions); pages [num_pages,Hkv,page_size,d] as bf16 bit patterns.
+    Returns (O [T,Hq,d], L [T,Hq]) in float64.
+    """
+    q = _f32(q)
+    kp = np.ascontiguousarray(np.asarray(k_pages_bf16_bits, dtype=np.uint16))
+    vp = np.ascontiguousarray(np.asarray(v_pages_bf16_bits, dtype=np.uint16))
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    T, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = kp.shape
+    S = sl.size
+    if d2 != d or vp.shape != kp.shape or cq.size != S + 1 or int(cq[-1]) != T:
+        raise ValueError("shape mismatch")
+    o = np.zeros((T, Hq, d), dtype=np.float64)
+    lse = np.zeros((T, Hq), dtype=np.float64)
+    rc = _load().oracle_prefill_paged(_ptr(q, ctypes.c_float), _ptr(kp, ctypes.c_uint16),
+                                      _ptr(vp, ctypes.c_uint16), _ptr(bt, ctypes.c_int32),
+                                      _ptr(sl, ctypes.c_int32), _ptr(cq, ctypes.c_int32),
+                                      _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                                      S, Hq, Hkv, d, page_size, bt.shape[1], num_pages,
+                                      float(scale), int(nthreads or max_threads()))
+    if rc != 0:
+        raise ValueError("oracle_prefill_paged failed with code %d" % rc)
     return o, lse
 
 

@@ -39,6 +39,8 @@
  * indirection table), then evaluates the same definition for its one query.
  * oracle_decode_paged_q8 is the same over 8-bit pages (E4M3 or INT8) with one
  * scale per (page, kv head): each element is dequantised to fp64 first.
+ * oracle_prefill_paged evaluates a chunk of queries at the end of each
+ * sequence against its paged keys (chunked prefill, causal from the end).
  * oracle_attn_bwd (and its sampled forms _dq_rows, _dkv_rows) evaluates the
  * gradients of the same definition with respect to Q, K and V.
  *
@@ -280,6 +282,74 @@ static double e4m3_to_double(uint8_t b)
     if (e == 0) v = ldexp((double)m / 8.0, -6);
     else v = ldexp(1.0 + (double)m / 8.0, e - 7);
     return sign ? -v : v;
+}
+
+/* Chunked prefill over the paged cache ("Phase 08" page, Concepts: chunked
+ * prefill splits a long prompt over several steps; Lab 03 Extensions: add
+ * chunked prefill; paged attention as above).  Read plainly: sequence s holds
+ * seq_lens[s] tokens in its pages, of which the last qlen_s = cu_q[s+1] - cu_q[s]
+ * are the current chunk's queries (their K/V already written to the cache).
+ * Query t of the chunk sits at position ctx_s + t, ctx_s = seq_lens[s] - qlen_s,
+ * and sees keys 0 .. ctx_s + t (causal, aligned to the end of the keys).
+ * q [T,Hq,d] float (T = cu_q[S], token-major), o [T,Hq,d], lse [T,Hq] double. */
+int oracle_prefill_paged(const float *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                         const int32_t *block_table, const int32_t *seq_lens,
+                         const int32_t *cu_q, double *o, double *lse,
+                         int S, int Hq, int Hkv, int d, int page_size, int max_blocks,
+                         int num_pages, double scale, int nthreads)
+{
+    int G, s, bad = 0, T;
+    if (S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || page_size <= 0 || max_blocks <= 0 ||
+        num_pages <= 0 || Hq % Hkv != 0) return -1;
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !cu_q || !o || !lse) return -1;
+    if (cu_q[0] != 0) return -1;
+    for (s = 0; s < S; ++s) {
+        int len = seq_lens[s], ql = cu_q[s + 1] - cu_q[s], t;
+        if (ql < 0 || len < ql || len > max_blocks * page_size) return -1;
+        for (t = 0; t < len; t += page_size) {
+            int32_t p = block_table[(size_t)s * max_blocks + t / page_size];
+            if (p < 0 || p >= num_pages) return -1;
+        }
+    }
+    G = Hq / Hkv;
+    T = cu_q[S];
+    if (nthreads <= 0) nthreads = 1;
+    (void)T;
+
+    #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) reduction(|:bad)
+    for (s = 0; s < S * Hkv; ++s) {
+        int seq = s / Hkv, g = s % Hkv;
+        int len = seq_lens[seq], q0 = cu_q[seq], ql = cu_q[seq + 1] - cu_q[seq];
+        int ctx = len - ql, t, c, hh;
+        double *kd = (double *)malloc(sizeof(double) * ((size_t)len * d + 1));
+        double *vd = (double *)malloc(sizeof(double) * ((size_t)len * d + 1));
+        double *sc = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+        if (!kd || !vd || !sc) { free(kd); free(vd); free(sc); bad = 1; continue; }
+        for (t = 0; t < len; ++t) {
+            int32_t p = block_table[(size_t)seq * max_blocks + t / page_size];
+            size_t base = (((size_t)p * Hkv + g) * page_size + (t % page_size)) * (size_t)d;
+            for (c = 0; c < d; ++c) {
+                kd[(size_t)t * d + c] = bf16_bits_to_double(k_pages[base + c]);
+                vd[(size_t)t * d + c] = bf16_bits_to_double(v_pages[base + c]);
+            }
+        }
+        for (hh = 0; hh < G; ++hh) {
+            int h = g * G + hh;
+            for (t = 0; t < ql; ++t) {
+                const float *qt = q + ((size_t)(q0 + t) * Hq + h) * (size_t)d;
+                int nvis = ctx + t + 1, j;
+                for (j = 0; j < nvis; ++j) {
+                    double acc = 0.0;
+                    for (c = 0; c < d; ++c) acc += (double)qt[c] * kd[(size_t)j * d + c];
+                    sc[j] = scale * acc;
+                }
+                softmax_row_times_v(sc, nvis, vd, d, o + ((size_t)(q0 + t) * Hq + h) * (size_t)d,
+                                    lse + (size_t)(q0 + t) * Hq + h);
+            }
+        }
+        free(kd); free(vd); free(sc);
+    }
+    return bad ? -2 : 0;
 }
 
 /* ------------------------------------------------------------------ backward

@@ -18,6 +18,9 @@ the mathematics fix, independently of the oracle's own code:
   power-of-two scales equals the bf16 paged decode of the dequantised cache
   exactly; scale linearity (V's scale multiplies O, K's acts as the softmax
   scale);
+* chunked prefill over the paged cache: rows ctx.. of a full causal prefill
+  over the contiguous sequence; one query per chunk is the paged decode;
+  splitting a chunk in two changes nothing;
 * backward: gradients equal a 4-point central-difference derivative of the
   forward oracle (inputs on a 2^-10 grid so every perturbed value is exact in
   float32); the two-key closed form; invariants (dK of a head sums to zero,
@@ -564,6 +567,84 @@ def test_q8_decode_rejects_bad_page_ids():
                                np.array([[0, 5]], np.int32), np.array([3], np.int32), scale=1.0)
 
 
+# --------------------------------------------------------- chunked prefill
+
+
+def _paged_case(lens, qlens, Hq, Hkv, d, ps=4, seed=0):
+    """A page pool holding each sequence's tokens in shuffled pages, and the
+    contiguous copies (bf16 values) for the checks."""
+    rng = np.random.default_rng(seed)
+    S = len(lens)
+    maxb = max(1, max(-(-n // ps) for n in lens))
+    P = sum(-(-n // ps) for n in lens) + 3
+    kp = _bf16_bits(rand(P, Hkv, ps, d, rng=rng))
+    vp = _bf16_bits(rand(P, Hkv, ps, d, rng=rng))
+    perm = rng.permutation(P).astype(np.int32)
+    bt = np.full((S, maxb), -1, dtype=np.int32)
+    nxt = 0
+    kc, vc = [], []
+    for s_, n in enumerate(lens):
+        k = -(-n // ps)
+        bt[s_, :k] = perm[nxt:nxt + k]
+        nxt += k
+        kc.append(np.stack([_bits_to_f32(kp[bt[s_, t // ps], :, t % ps]) for t in range(n)], axis=1)
+                  if n else np.zeros((Hkv, 0, d), np.float32))
+        vc.append(np.stack([_bits_to_f32(vp[bt[s_, t // ps], :, t % ps]) for t in range(n)], axis=1)
+                  if n else np.zeros((Hkv, 0, d), np.float32))
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = _bits_to_f32(_bf16_bits(rand(int(cu[-1]), Hq, d, rng=rng)))
+    return q, kp, vp, bt, np.array(lens, np.int32), cu, kc, vc
+
+
+def test_prefill_paged_equals_causal_rows_of_full_prefill():
+    # The chunk's queries placed at rows ctx..len-1 of a full causal prefill
+    # over the contiguous sequence give those rows (rows before ctx arbitrary).
+    lens, qlens = [9, 13, 5, 4], [3, 13, 1, 0]
+    Hq, Hkv, d = 4, 2, 8
+    q, kp, vp, bt, sl, cu, kc, vc = _paged_case(lens, qlens, Hq, Hkv, d, seed=51)
+    o, lse = oracle.prefill_paged(q, kp, vp, bt, sl, cu, scale=0.3)
+    rng = np.random.default_rng(52)
+    for s_, (n, ql) in enumerate(zip(lens, qlens)):
+        if ql == 0:
+            continue
+        ctx = n - ql
+        qf = rand(1, Hq, n, d, rng=rng)
+        qf[0, :, ctx:] = q[cu[s_]:cu[s_ + 1]].transpose(1, 0, 2)
+        of, lf = oracle.attention(qf, kc[s_][None], vc[s_][None], scale=0.3, causal=True)
+        np.testing.assert_allclose(o[cu[s_]:cu[s_ + 1]], of[0, :, ctx:].transpose(1, 0, 2),
+                                   rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[cu[s_]:cu[s_ + 1]], lf[0, :, ctx:].T, rtol=0, atol=1e-13)
+
+
+def test_prefill_paged_single_query_is_decode():
+    lens, qlens = [7, 1, 12], [1, 1, 1]
+    q, kp, vp, bt, sl, cu, _, _ = _paged_case(lens, qlens, 4, 1, 8, seed=53)
+    o, lse = oracle.prefill_paged(q, kp, vp, bt, sl, cu, scale=0.5)
+    od, ld = oracle.decode_paged(q, kp, vp, bt, sl, scale=0.5)
+    np.testing.assert_allclose(o, od, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, ld, rtol=0, atol=1e-14)
+
+
+def test_prefill_paged_chunking_invariance():
+    # Processing a prompt chunk in two pieces (the first piece with the
+    # shorter length) gives the same rows as processing it at once.
+    n, ql, split = 14, 9, 4
+    q, kp, vp, bt, sl, cu, _, _ = _paged_case([n], [ql], 2, 2, 8, seed=54)
+    o, lse = oracle.prefill_paged(q, kp, vp, bt, sl, cu, scale=0.4)
+    o1, l1 = oracle.prefill_paged(q[:split], kp, vp, bt, np.array([n - ql + split], np.int32),
+                                  np.array([0, split], np.int32), scale=0.4)
+    o2, l2 = oracle.prefill_paged(q[split:], kp, vp, bt, np.array([n], np.int32),
+                                  np.array([0, ql - split], np.int32), scale=0.4)
+    np.testing.assert_array_equal(np.concatenate([o1, o2]), o)
+    np.testing.assert_array_equal(np.concatenate([l1, l2]), lse)
+
+
+def test_prefill_paged_rejects_chunk_longer_than_sequence():
+    q, kp, vp, bt, sl, cu, _, _ = _paged_case([5], [5], 1, 1, 4, seed=55)
+    with pytest.raises(ValueError):
+        oracle.prefill_paged(q, kp, vp, bt, np.array([4], np.int32), cu, scale=1.0)
+
+
 # ------------------------------------------------------------------ backward
 
 
@@ -752,6 +833,22 @@ def _run_mutant(src_old, src_new, tmp_path, checks):
     finally:
         oracle.build = real_build
         oracle._lib = saved
+
+
+PAGED_PREFILL_MUTANTS = {
+    "chunk_visible_off_by_one": ("int nvis = ctx + t + 1, j;", "int nvis = ctx + t, j;"),
+    "chunk_ctx_ignored": ("int ctx = len - ql, t, c, hh;", "int ctx = 0, t, c, hh;"),
+    "chunk_wrong_query_row": ("const float *qt = q + ((size_t)(q0 + t) * Hq + h) * (size_t)d;",
+                              "const float *qt = q + ((size_t)(t) * Hq + h) * (size_t)d;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PAGED_PREFILL_MUTANTS))
+def test_prefill_paged_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = PAGED_PREFILL_MUTANTS[name]
+    checks = [test_prefill_paged_equals_causal_rows_of_full_prefill,
+              test_prefill_paged_single_query_is_decode, test_prefill_paged_chunking_invariance]
+    assert _run_mutant(old, new, tmp_path, checks) > 0, "mutant %s survived every pin" % name
 
 
 BWD_MUTANTS = {
