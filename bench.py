@@ -11,7 +11,8 @@ The JSON line also carries, measured in the same run:
     Hkv=8) prefill TFLOP/s, and the paged GQA decode (64 sequences, context
     U[512, 8192], 16-token pages) in HBM GB/s over a bf16 cache and over 8-bit
     (E4M3, INT8) caches of the same shape, each as a fraction of the measured
-    peak;
+    peak; and the backward (dQ, dK, dV) of the N=8192 MHA and causal
+    workloads in TFLOP/s of the algorithm's five products;
   * ``roofline`` for the prefill kernel (tensor-bound);
   * ``e2e``: the same sweep through the public API with pinned host buffers,
     host->device and device->host copies inside the timed region;
@@ -239,6 +240,40 @@ class Decode:
         return 2  # split + combine
 
 
+class Backward:
+    """Backward of a prefill workload: the forward's O and L are computed once
+    (outside the timing), dO is N(0,1); one launch = prep + dK/dV + dQ kernels.
+    FLOPs: the algorithm's five N x N x d products, 10 * B * Hq * N^2 * d
+    (half for causal), not the seven this implementation spends."""
+
+    def __init__(self, cfg, lib):
+        import exact_io_aware_101_b200 as ea
+        self.cfg = cfg
+        self.lib = lib
+        self.q, self.k, self.v = syn.prefill_inputs(cfg, device="cuda")
+        g = torch.Generator(device="cuda")
+        g.manual_seed(cfg.seed + 7)
+        self.do = torch.randn(self.q.shape, generator=g, device="cuda").to(torch.bfloat16)
+        self.o, self.lse = ea.attn_fwd(self.q, self.k, self.v, causal=cfg.causal)
+        self.dq = torch.empty_like(self.q)
+        self.dk = torch.empty_like(self.k)
+        self.dv = torch.empty_like(self.v)
+        self.ws_bytes = ea.bwd_workspace_bytes(cfg.B, cfg.Hq, cfg.N)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.flops = 2.5 * cfg.flops
+
+    def launch(self):
+        c = self.cfg
+        rc = self.lib.attn_bwd(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                               self.o.data_ptr(), self.lse.data_ptr(), self.do.data_ptr(),
+                               self.dq.data_ptr(), self.dk.data_ptr(), self.dv.data_ptr(), c.B, c.Hq,
+                               c.Hkv, c.N, c.d, c.scale, int(c.causal), 0, None, self.ws.data_ptr(),
+                               self.ws_bytes, torch.cuda.current_stream().cuda_stream)
+        if rc != 0:
+            raise RuntimeError("attn_bwd failed: %d" % rc)
+        return 3  # prep + dK/dV + dQ
+
+
 class DecodeQ8:
     """The decode workload over an 8-bit cache (same q, lengths and placement)."""
 
@@ -453,6 +488,16 @@ def run_ours(args):
             tf = cfg.flops / sec / 1e12
             comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3}
             del it
+        for cfg in (syn.MHA_SWEEP[-1], syn.CAUSAL):
+            it = Backward(cfg, lib)
+            timed_launches([it], flush, 3)
+            t, _ = timed_launches([it], flush, args.component_reps)
+            sec = sum(t[0]) / len(t[0]) / 1e3
+            tf = it.flops / sec / 1e12
+            comps["bwd_" + cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf,
+                                        "ms": sec * 1e3, "flops": it.flops,
+                                        "flops_counted": "5 products of the algorithm (2.5x fwd)"}
+            del it
         dec = Decode(syn.DECODE, lib)
         timed_launches([dec], flush, 3)
         t, _ = timed_launches([dec], flush, args.component_reps)
@@ -504,7 +549,10 @@ def run_only(args):
     lib = ea.library()
     table = {c.name: c for c in syn.MHA_SWEEP + (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI)}
     q8 = {syn.DECODE.name + "_" + f: f for f in ("e4m3", "int8")}
-    if args.only == syn.DECODE.name:
+    bwd = {"bwd_" + c.name: c for c in (syn.MHA_SWEEP[-1], syn.CAUSAL, syn.MHA_SWEEP[0])}
+    if args.only in bwd:
+        it = Backward(bwd[args.only], lib)
+    elif args.only == syn.DECODE.name:
         it = Decode(syn.DECODE, lib)
     elif args.only in q8:
         it = DecodeQ8(syn.DECODE, lib, q8[args.only])
@@ -512,7 +560,7 @@ def run_only(args):
         it = Prefill(table[args.only], lib)
     else:
         raise SystemExit("unknown workload %r; one of %s"
-                         % (args.only, sorted(table) + [syn.DECODE.name] + sorted(q8)))
+                         % (args.only, sorted(table) + [syn.DECODE.name] + sorted(q8) + sorted(bwd)))
     for _ in range(args.reps):
         it.launch()
     torch.cuda.synchronize()

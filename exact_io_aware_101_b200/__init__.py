@@ -21,6 +21,7 @@ import torch
 __all__ = [
     "attn_fwd", "attn_fwd_f32", "attn_decode_paged", "attn_decode_paged_noalloc",
     "attn_decode_paged_q8", "KV_FORMATS", "decode_workspace_bytes", "attn_bwd",
+    "attn_prefill_paged",
     "bwd_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
     "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
     "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "AttnError",
@@ -28,7 +29,7 @@ __all__ = [
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ext", "attn_fwd_f32_ext",
-                    "attn_bwd_workspace_bytes", "attn_bwd",
+                    "attn_bwd_workspace_bytes", "attn_bwd", "attn_prefill_paged",
                     "attn_decode_workspace_bytes",
                     "attn_decode_paged", "attn_decode_paged_noalloc", "attn_decode_paged_q8",
                     "attn_device_status",
@@ -68,6 +69,9 @@ def library() -> ctypes.CDLL:
         lib.attn_fwd_ext.restype = ci
         lib.attn_fwd_f32_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
         lib.attn_fwd_f32_ext.restype = ci
+        lib.attn_prefill_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci,
+                                           ci, ci, ci, cf, ci, vp, vp]
+        lib.attn_prefill_paged.restype = ci
         lib.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci]
         lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
@@ -175,6 +179,50 @@ def attn_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, out=
     """fp32 prefill with fp32 arithmetic throughout (same options as attn_fwd)."""
     return _prefill(library().attn_fwd_f32, "attn_fwd_f32", q, k, v, causal, scale, out, lse,
                     torch.float32, window, alibi_slopes)
+
+
+def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, cu_q, max_q: int,
+                       scale: float | None = None, window: int = 0, alibi_slopes=None,
+                       out=None, lse=None):
+    """Chunked prefill over the paged cache.
+
+    q [T,Hq,d] bf16 token-major (sequence s: rows cu_q[s]..cu_q[s+1]-1, the
+    last tokens of its seq_lens[s]); pages [num_pages,Hkv,16,d] bf16;
+    block_table [S,max_blocks], seq_lens [S], cu_q [S+1] int32 (GPU).  max_q
+    bounds every chunk length.  Returns (O bf16 [T,Hq,d], L fp32 [T,Hq]).
+    """
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _check(cu_q, "cu_q", torch.int32, 1)
+    T, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = k_pages.shape
+    S = seq_lens.shape[0]
+    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("page pools must be [num_pages, Hkv, page_size, d]")
+    if block_table.shape[0] != S or cu_q.shape[0] != S + 1:
+        raise ValueError("block_table needs S rows and cu_q S+1 entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", torch.bfloat16, 3)
+    _check(lse, "lse", torch.float32, 2)
+    slopes_ptr = None
+    if alibi_slopes is not None:
+        _check(alibi_slopes, "alibi_slopes", torch.float32, 1)
+        if alibi_slopes.numel() != Hq:
+            raise ValueError("alibi_slopes needs one value per query head")
+        slopes_ptr = alibi_slopes.data_ptr()
+    rc = library().attn_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                      block_table.data_ptr(), seq_lens.data_ptr(), cu_q.data_ptr(),
+                                      out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, T, int(max_q), d,
+                                      page_size, block_table.shape[1], num_pages, float(scale),
+                                      int(window), slopes_ptr, _stream(q))
+    _raise(rc, "attn_prefill_paged")
+    return out, lse
 
 
 def bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:

@@ -108,6 +108,34 @@ attn_status_t attn_fwd_f32(const float *q, const float *k, const float *v, float
   return attn_fwd_f32_ext(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, nullptr, stream);
 }
 
+attn_status_t attn_prefill_paged(const void *q, const void *k_pages, const void *v_pages,
+                                 const int32_t *block_table, const int32_t *seq_lens,
+                                 const int32_t *cu_q, void *o, float *lse, int S, int Hq, int Hkv,
+                                 int T, int max_q, int d, int page_size, int max_blocks,
+                                 int num_pages, float scale, int window,
+                                 const float *alibi_slopes, attn_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned4(block_table) ||
+      !aligned4(seq_lens) || !aligned4(cu_q) || !aligned16(o) || !aligned4(lse) ||
+      (alibi_slopes && !aligned4(alibi_slopes)))
+    return ATTN_ERR_INVALID_ARG;
+  if (S <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || T < 0 || max_q < 0 || d <= 0 ||
+      page_size <= 0 || max_blocks <= 0 || num_pages <= 0 || window < 0 || !good_scale(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || page_size != 16) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks) * page_size > (1LL << 30) ||
+      static_cast<long long>(num_pages) * Hkv >= (1LL << 31) ||
+      static_cast<long long>(T) * Hq * d >= (1LL << 40))
+    return ATTN_ERR_INVALID_ARG;
+  if (T == 0 || max_q == 0) return ATTN_OK;
+  unsigned *status = nullptr;
+  bool sm100 = false;
+  if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
+  if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  return launch_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, cu_q, o, lse, S, Hq, Hkv,
+                              T, max_q, d, max_blocks, num_pages, scale, window, alibi_slopes,
+                              reinterpret_cast<cudaStream_t>(stream), status);
+}
+
 size_t attn_bwd_workspace_bytes(int B, int Hq, int N) {
   if (B <= 0 || Hq <= 0 || N <= 0) return 0;
   return bwd_workspace_bytes(B, Hq, N);

@@ -163,22 +163,26 @@ __device__ __forceinline__ void grad_cols(const uint32_t (&sv)[32], const uint32
                                           const float *l2c, const float *ddc, float l2s, float dds,
                                           bool per_col, float c, float bias0, float bias_step,
                                           Vis vis, uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+  const float2 c2 = make_float2(c, c);
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
-    float p[2], ds[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float lv = per_col ? l2c[i + e] : l2s;
-      const float dv = per_col ? ddc[i + e] : dds;
-      float x = fmaf(__uint_as_float(sv[i + e]), c, -lv);
-      if (kAlibi) x = fmaf(bias_step, static_cast<float>(i + e), x + bias0);
-      float pe = ex2(x);
-      if (kMasked && !vis(i + e)) pe = 0.f;
-      p[e] = pe;
-      ds[e] = pe * (__uint_as_float(dpv[i + e]) - dv);
+    const float2 lv = per_col ? make_float2(l2c[i], l2c[i + 1]) : make_float2(l2s, l2s);
+    const float2 dv = per_col ? make_float2(ddc[i], ddc[i + 1]) : make_float2(dds, dds);
+    float2 x = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2,
+                    make_float2(-lv.x, -lv.y));
+    if (kAlibi)
+      x = fma2(make_float2(bias_step, bias_step),
+               make_float2(static_cast<float>(i), static_cast<float>(i + 1)),
+               make_float2(x.x + bias0, x.y + bias0));
+    float2 pe = make_float2(ex2(x.x), ex2(x.y));
+    if (kMasked) {
+      if (!vis(i)) pe.x = 0.f;
+      if (!vis(i + 1)) pe.y = 0.f;
     }
-    if (kWantP) pk[i >> 1] = pack_bf16x2(p[0], p[1]);
-    dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
+    const float2 t = add2(make_float2(__uint_as_float(dpv[i]), __uint_as_float(dpv[i + 1])),
+                          make_float2(-dv.x, -dv.y));
+    if (kWantP) pk[i >> 1] = pack_bf16x2(pe.x, pe.y);
+    dk[i >> 1] = pack_bf16x2(pe.x * t.x, pe.y * t.y);
   }
 }
 

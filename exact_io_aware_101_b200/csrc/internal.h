@@ -16,6 +16,13 @@ attn_status_t launch_prefill_bf16(const void *q, const void *k, const void *v, v
                                   int window, const float *slopes, cudaStream_t stream,
                                   unsigned *status);
 
+// Chunked prefill over a paged cache (causal from the end of each sequence).
+attn_status_t launch_prefill_paged(const void *q, const void *k_pages, const void *v_pages,
+                                   const int *block_table, const int *seq_lens, const int *cu_q,
+                                   void *o, float *lse, int S, int Hq, int Hkv, int T, int max_q,
+                                   int d, int max_blocks, int num_pages, float scale, int window,
+                                   const float *slopes, cudaStream_t stream, unsigned *status);
+
 attn_status_t launch_prefill_f32(const float *q, const float *k, const float *v, float *o,
                                  float *lse, int B, int Hq, int Hkv, int N, int d, float scale,
                                  int causal, int window, const float *slopes,

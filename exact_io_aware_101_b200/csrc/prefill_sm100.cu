@@ -93,6 +93,11 @@ struct Params {
   int causal;
   int window;            // > 0: key j visible to query i only if i - j < window
   const float *slopes;   // ALiBi slope per query head (kernel variant with the bias)
+  // Chunked prefill over a paged cache (kernel variant kPaged): B = sequences;
+  // queries token-major [T][Hq][D], sequence s owning rows cu_q[s]..cu_q[s+1]-1
+  // at positions seq_lens[s] - qlen_s ...; keys through the block table.
+  const int *block_table, *seq_lens, *cu_q;
+  int max_blocks, num_pages, T;
 };
 
 // One thread's 128-column score row -> P (bf16 pairs in TMEM at s_addr) and
@@ -124,11 +129,13 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float c, flo
   return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
 }
 
-template <int D, bool kAlibi>
+template <int D, bool kAlibi, bool kPaged>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_k1,
+                        const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -165,17 +172,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int hq = bh % p.Hq;
   const int hkv = hq / (p.Hq / p.Hkv);
   const int row0 = pair * 2 * BM;
-  const int nkv = (p.N + BN - 1) / BN;
+  // Rows of this (batch, head) or sequence chunk (nq), keys (nk), and the
+  // position of row 0 among the keys (ctx: 0 for self-attention; for a chunk,
+  // its queries are the last nq of the sequence's nk positions).
+  int nq = p.N, nk = p.N, ctx = 0, qrow0 = 0;
+  if constexpr (kPaged) {
+    const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1];
+    nk = p.seq_lens[b];
+    nq = q1 - q0;
+    qrow0 = q0;
+    // (For a chunk, p.N is the caller's bound max_q on every chunk length; the
+    // grid covers it.)
+    const bool bad_len = q0 < 0 || nq < 0 || q1 > p.T || nk < nq || nk > p.max_blocks * 16 ||
+                         nq > p.N;
+    if (bad_len) {
+      if (threadIdx.x == 0 && pair == 0 && hq == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
+      return;
+    }
+    if (row0 >= nq) return;  // pair past the chunk: nothing to do
+    ctx = nk - nq;
+  }
+  const int nkv = (nk + BN - 1) / BN;
   // KV tiles [js_t, je_t) of each Q tile: the causal diagonal caps the end,
-  // a sliding window moves the start; a Q tile past N has none.
+  // a sliding window moves the start; a Q tile past the rows has none.
   // (Scalars, not arrays: the issuing thread reads them every iteration.)
-  const bool rows1 = row0 + BM < p.N;
-  const int je0 = p.causal ? min(row0 / BN + 1, nkv) : nkv;
-  const int je1 = !rows1 ? 0 : (p.causal ? min((row0 + BM) / BN + 1, nkv) : nkv);
-  const int js0 = p.window > 0 ? max(0, row0 - p.window + 1) / BN : 0;
-  const int js1 = (!rows1 || p.window <= 0) ? 0 : max(0, row0 + BM - p.window + 1) / BN;
+  const bool rows1 = row0 + BM < nq;
+  int je0, je1, js0, js1;
+  if constexpr (kPaged) {  // the diagonal sits ctx keys to the right
+    const int last0 = min(row0 + BM, nq) - 1, last1 = min(row0 + 2 * BM, nq) - 1;
+    je0 = p.causal ? min((ctx + last0) / BN + 1, nkv) : nkv;
+    je1 = !rows1 ? 0 : (p.causal ? min((ctx + last1) / BN + 1, nkv) : nkv);
+    js0 = p.window > 0 ? max(0, ctx + row0 - p.window + 1) / BN : 0;
+    js1 = (!rows1 || p.window <= 0) ? 0 : max(0, ctx + row0 + BM - p.window + 1) / BN;
+  } else {
+    je0 = p.causal ? min(row0 / BN + 1, nkv) : nkv;
+    je1 = !rows1 ? 0 : (p.causal ? min((row0 + BM) / BN + 1, nkv) : nkv);
+    js0 = p.window > 0 ? max(0, row0 - p.window + 1) / BN : 0;
+    js1 = (!rows1 || p.window <= 0) ? 0 : max(0, row0 + BM - p.window + 1) / BN;
+  }
   const int jlo = js0;
   const int jhi = max(je0, je1);
+  if constexpr (kPaged) {
+    // Every page the tiles [jlo, jhi) read must be in the pool; a sequence
+    // with a bad entry gets NaN rows and the status bit, and no copy is issued.
+    const int pg_end = min(jhi * (BN / 16), (nk + 15) / 16);
+    bool bad = false;
+    for (int i = jlo * (BN / 16) + static_cast<int>(threadIdx.x); i < pg_end; i += NUM_THREADS) {
+      const int pid = p.block_table[static_cast<size_t>(b) * p.max_blocks + i];
+      bad |= pid < 0 || pid >= p.num_pages;
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
+      for (int idx = threadIdx.x; idx < 2 * BM * (D + 1); idx += NUM_THREADS) {
+        const int r = idx / (D + 1), c = idx % (D + 1);
+        const int row = row0 + r;
+        if (row >= nq) continue;
+        const size_t tok = static_cast<size_t>(qrow0 + row) * p.Hq + hq;
+        if (c < D)
+          reinterpret_cast<__nv_bfloat16 *>(p.o)[tok * D + c] = __float2bfloat16_rn(NAN);
+        else
+          p.lse[tok] = NAN;
+      }
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -215,9 +275,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int zkv = b * p.Hkv + hkv;
       mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
       for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
-                      row0 + t * BM, zq);
+        for (int c = 0; c < C::CH; ++c) {
+          if constexpr (kPaged)  // token-major queries: (D, Hq, T) boxes of 64 x 1 x 128
+            tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
+                        hq, qrow0 + row0 + t * BM);
+          else
+            tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
+                        row0 + t * BM, zq);
+        }
       int issued = 0;
       for (int i = 0; i < 2 * (jhi - jlo); ++i) {
         const int slot = i % C::NST;
@@ -226,9 +291,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
         const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
-        for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
-                      64 * c, (jlo + (i >> 1)) * BN, zkv);
+        if constexpr (kPaged) {
+          // Gather the tile's 8 pages: whole pages as 16-row boxes; the last,
+          // partly filled page row by row; rows past the keys from an
+          // out-of-range coordinate, i.e. zeros (never stale shared memory,
+          // which a zero P could not cancel if it held a NaN).
+          const CUtensorMap *map1 = (i & 1) ? &tm_v1 : &tm_k1;
+          const int key_base = (jlo + (i >> 1)) * BN;
+          for (int pp = 0; pp < BN / 16; ++pp) {
+            const int key0 = key_base + pp * 16;
+            const int ntok = min(16, nk - key0);
+            const int z = ntok > 0
+                ? p.block_table[static_cast<size_t>(b) * p.max_blocks + key0 / 16] * p.Hkv + hkv
+                : -1;
+            uint8_t *dst = sRing + slot * C::TILE_BYTES + pp * 16 * 128;
+            for (int c = 0; c < C::CH; ++c) {
+              if (ntok >= 16 || ntok <= 0) {
+                tma_load_3d(dst + c * CHUNK_BYTES, map, &bars->full[slot], 64 * c, 0, z);
+              } else {
+                for (int r = 0; r < 16; ++r)
+                  tma_load_3d(dst + c * CHUNK_BYTES + r * 128, map1, &bars->full[slot], 64 * c, r,
+                              r < ntok ? z : -1);
+              }
+            }
+          }
+        } else {
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
+                        64 * c, (jlo + (i >> 1)) * BN, zkv);
+        }
         issued = i + 1;
       }
       // Drain: no copy may still be writing shared memory when the CTA exits.
@@ -357,18 +448,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       // Visible columns [lo, hi) of this row in KV tile j: the end of the keys,
       // the causal diagonal and the sliding window.
-      int hi = min(BN, p.N - j * BN);
-      if (p.causal) hi = min(hi, row - j * BN + 1);
-      // (Rows past N take the last real row's window so that they never force
-      // the masked path on a warp whose real rows need none.)
-      const int lo = p.window > 0 ? min(row, p.N - 1) - p.window + 1 - j * BN : 0;
+      int hi = min(BN, nk - j * BN);
+      if (p.causal) hi = min(hi, ctx + row - j * BN + 1);
+      // (Rows past the last take the last real row's window so that they never
+      // force the masked path on a warp whose real rows need none.)
+      const int lo = p.window > 0 ? ctx + min(row, nq - 1) - p.window + 1 - j * BN : 0;
       // The whole 128-column score row of this thread, in one TMEM load.
       uint32_t sv[128];
       tmem_ld128(s_addr, sv);
       tmem_ld_wait128(sv);
       float cx = c;  // factor still to apply to sv in the exponent
       if (kAlibi) {
-        const float rb = slope2 * static_cast<float>(j * BN - row);
+        const float rb = slope2 * static_cast<float>(j * BN - (ctx + row));
         const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2), rb2 = make_float2(rb, rb);
 #pragma unroll
         for (int i = 0; i < 128; i += 2) {
@@ -437,9 +528,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (ok) {
         tc_fence_after();
         const float inv_l = 1.0f / l;
-        const bool valid = row < p.N;
-        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) +
-                              ((static_cast<size_t>(b) * p.Hq + hq) * p.N + (valid ? row : 0)) * D;
+        const bool valid = row < nq;
+        // Row of O and L: [B][Hq][N] for self-attention, [T][Hq] for a chunk.
+        const size_t orow_idx =
+            kPaged ? static_cast<size_t>(qrow0 + (valid ? row : 0)) * p.Hq + hq
+                   : (static_cast<size_t>(b) * p.Hq + hq) * p.N + (valid ? row : 0);
+        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + orow_idx * D;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t ov[32];
@@ -456,9 +550,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
         }
-        if (valid)
-          p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.N + row] =
-              (m + log2f(l)) * 0.6931471805599453f;
+        if (valid) p.lse[orow_idx] = (m + log2f(l)) * 0.6931471805599453f;
       }
     }
   }
@@ -507,23 +599,59 @@ bool make_map(CUtensorMap *map, const void *base, int D, int N, int BH) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool kAlibi>
-attn_status_t launch(const void *q, const void *k, const void *v, void *o, float *lse, int B,
-                     int Hq, int Hkv, int N, float scale, int causal, int window,
-                     const float *slopes, cudaStream_t stream, unsigned *status) {
+// Page pool [P][Hkv][16][D] bf16 as a 3-D tensor (D, 16, P*Hkv); boxes of 64
+// columns x `rows` rows of one (page, K/V head) slice, 128B swizzle.
+bool make_page_map(CUtensorMap *map, const void *base, int D, long long slices, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), 16, static_cast<cuuint64_t>(slices)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(16) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Token-major queries [T][Hq][D] bf16 as (D, Hq, T); boxes of 64 x 1 x 128.
+bool make_tok_map(CUtensorMap *map, const void *base, int D, int Hq, int T) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool kAlibi, bool kPaged>
+attn_status_t launch_kernel(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                            const CUtensorMap &mk1, const CUtensorMap &mv1, const Params &prm,
+                            long long ctas, cudaStream_t stream) {
   using C = Cfg<D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D, kAlibi>,
+    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D, kAlibi, kPaged>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, N, B * Hq) || !make_map(&mk, k, D, N, B * Hkv) ||
-      !make_map(&mv, v, D, N, B * Hkv))
-    return ATTN_ERR_CUDA;
-  Params prm;
+  if (ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (ctas == 0) return ATTN_OK;
+  prefill_bf16_kernel<D, kAlibi, kPaged>
+      <<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mk1, mv1,
+                                                                             prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+Params base_params(void *o, float *lse, unsigned *status, int B, int Hq, int Hkv, int N,
+                   float scale, int causal, int window, const float *slopes) {
+  Params prm{};
   prm.o = o;
   prm.lse = lse;
   prm.status = status;
@@ -536,11 +664,43 @@ attn_status_t launch(const void *q, const void *k, const void *v, void *o, float
   prm.causal = causal ? 1 : 0;
   prm.window = window;
   prm.slopes = slopes;
+  return prm;
+}
+
+template <int D, bool kAlibi>
+attn_status_t launch(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                     int Hq, int Hkv, int N, float scale, int causal, int window,
+                     const float *slopes, cudaStream_t stream, unsigned *status) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, N, B * Hq) || !make_map(&mk, k, D, N, B * Hkv) ||
+      !make_map(&mv, v, D, N, B * Hkv))
+    return ATTN_ERR_CUDA;
+  const Params prm = base_params(o, lse, status, B, Hq, Hkv, N, scale, causal, window, slopes);
   const long long ctas = static_cast<long long>(prm.pairs) * B * Hq;
-  if (ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  prefill_bf16_kernel<D, kAlibi><<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(
-      mq, mk, mv, prm);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return launch_kernel<D, kAlibi, false>(mq, mk, mv, mk, mv, prm, ctas, stream);
+}
+
+template <int D, bool kAlibi>
+attn_status_t launch_paged(const void *q, const void *k_pages, const void *v_pages,
+                           const int *block_table, const int *seq_lens, const int *cu_q, void *o,
+                           float *lse, int S, int Hq, int Hkv, int T, int max_q, int max_blocks,
+                           int num_pages, float scale, int window, const float *slopes,
+                           cudaStream_t stream, unsigned *status) {
+  CUtensorMap mq, mk, mv, mk1, mv1;
+  const long long slices = static_cast<long long>(num_pages) * Hkv;
+  if (!make_tok_map(&mq, q, D, Hq, T) || !make_page_map(&mk, k_pages, D, slices, 16) ||
+      !make_page_map(&mv, v_pages, D, slices, 16) || !make_page_map(&mk1, k_pages, D, slices, 1) ||
+      !make_page_map(&mv1, v_pages, D, slices, 1))
+    return ATTN_ERR_CUDA;
+  Params prm = base_params(o, lse, status, S, Hq, Hkv, max_q, scale, 1, window, slopes);
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.cu_q = cu_q;
+  prm.max_blocks = max_blocks;
+  prm.num_pages = num_pages;
+  prm.T = T;
+  const long long ctas = static_cast<long long>(prm.pairs) * S * Hq;
+  return launch_kernel<D, kAlibi, true>(mq, mk, mv, mk1, mv1, prm, ctas, stream);
 }
 
 }  // namespace
@@ -560,6 +720,29 @@ attn_status_t launch_prefill_bf16(const void *q, const void *k, const void *v, v
                                     stream, status)
                  : launch<64, false>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, window,
                                      nullptr, stream, status);
+  return ATTN_ERR_UNSUPPORTED;
+}
+
+attn_status_t launch_prefill_paged(const void *q, const void *k_pages, const void *v_pages,
+                                   const int *block_table, const int *seq_lens, const int *cu_q,
+                                   void *o, float *lse, int S, int Hq, int Hkv, int T, int max_q,
+                                   int d, int max_blocks, int num_pages, float scale, int window,
+                                   const float *slopes, cudaStream_t stream, unsigned *status) {
+  const bool alibi = slopes != nullptr;
+  if (d == 128)
+    return alibi ? launch_paged<128, true>(q, k_pages, v_pages, block_table, seq_lens, cu_q, o, lse,
+                                           S, Hq, Hkv, T, max_q, max_blocks, num_pages, scale,
+                                           window, slopes, stream, status)
+                 : launch_paged<128, false>(q, k_pages, v_pages, block_table, seq_lens, cu_q, o,
+                                            lse, S, Hq, Hkv, T, max_q, max_blocks, num_pages, scale,
+                                            window, nullptr, stream, status);
+  if (d == 64)
+    return alibi ? launch_paged<64, true>(q, k_pages, v_pages, block_table, seq_lens, cu_q, o, lse,
+                                          S, Hq, Hkv, T, max_q, max_blocks, num_pages, scale,
+                                          window, slopes, stream, status)
+                 : launch_paged<64, false>(q, k_pages, v_pages, block_table, seq_lens, cu_q, o,
+                                           lse, S, Hq, Hkv, T, max_q, max_blocks, num_pages, scale,
+                                           window, nullptr, stream, status);
   return ATTN_ERR_UNSUPPORTED;
 }
 

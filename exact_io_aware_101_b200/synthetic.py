@@ -18,6 +18,9 @@ causal, grouped-query and paged-decode extensions):
   by a random permutation                                        seed 4
   The 8-bit cache variants (E4M3, INT8) quantise the same pools per
   (page, K/V head) slice with scale = amax / qmax (quantize_pages).
+* ``CHUNKED`` chunked prefill over a paged cache: 16 sequences, a 512-token
+  chunk each after ctx ~ U[0, 7680] cached tokens, Hq=32, Hkv=8, d=128,
+  16-token pages placed by a random permutation                  seed 7
 
 Generation order for a prefill workload: q, k, v from one generator.  For the
 decode workload: seq_lens (randint, CPU), the page permutation (randperm, CPU),
@@ -166,6 +169,73 @@ def decode_inputs(cfg: Decode = DECODE, device="cpu", seq_lens=None):
     v_pages = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
     return dict(q=q, k_pages=k_pages, v_pages=v_pages,
                 block_table=table.to(device), seq_lens=seq_lens.to(device))
+
+
+@dataclass(frozen=True)
+class Chunked:
+    """Chunked prefill over a paged cache: S sequences, each with a chunk of
+    qlen new tokens after ctx cached ones, ctx uniform in [ctx_lo, ctx_hi]."""
+    name: str = "chunked_prefill_gqa"
+    S: int = 16
+    qlen: int = 512
+    Hq: int = 32
+    Hkv: int = 8
+    d: int = 128
+    page_size: int = 16
+    ctx_lo: int = 0
+    ctx_hi: int = 7680
+    max_blocks: int = 512
+    seed: int = 7
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+CHUNKED = Chunked()
+
+
+def chunked_inputs(cfg: Chunked = CHUNKED, device="cpu", qlens=None, ctxs=None, num_pages=None):
+    """dict(q [T,Hq,d] bf16 token-major, k_pages/v_pages [P,Hkv,16,d] bf16,
+    block_table [S,max_blocks], seq_lens [S] (= ctx + qlen), cu_q [S+1]).
+
+    Generation order: ctx (randint, CPU), the page permutation, then q,
+    k_pages, v_pages from a generator on ``device``.  The pool holds exactly the
+    pages the sequences use plus 16 spare ones."""
+    gc = _gen("cpu", cfg.seed)
+    S = cfg.S if qlens is None else len(qlens)
+    if ctxs is None:
+        ctxs = torch.randint(cfg.ctx_lo, cfg.ctx_hi + 1, (S,), generator=gc, dtype=torch.int64)
+    ctxs = torch.as_tensor(ctxs, dtype=torch.int64)
+    qlens = torch.full((S,), cfg.qlen, dtype=torch.int64) if qlens is None else \
+        torch.as_tensor(qlens, dtype=torch.int64)
+    seq_lens = (ctxs + qlens).to(torch.int32)
+    if num_pages is None:
+        num_pages = int(sum((int(n) + cfg.page_size - 1) // cfg.page_size for n in seq_lens)) + 16
+    table = page_placement(seq_lens, num_pages, cfg.max_blocks, cfg.page_size, cfg.seed)
+    cu_q = torch.zeros(S + 1, dtype=torch.int32)
+    cu_q[1:] = torch.cumsum(qlens, 0).to(torch.int32)
+    T = int(cu_q[-1])
+    g = _gen(device, cfg.seed)
+    q = torch.randn(T, cfg.Hq, cfg.d, generator=g, device=device).to(torch.bfloat16)
+    shape = (num_pages, cfg.Hkv, cfg.page_size, cfg.d)
+    k_pages = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+    v_pages = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+    return dict(q=q, k_pages=k_pages, v_pages=v_pages, block_table=table.to(device),
+                seq_lens=seq_lens.to(device), cu_q=cu_q.to(device))
+
+
+def chunked_flops(seq_lens, cu_q, Hq: int, d: int) -> float:
+    """4*d per visible (query, key) pair: chunk query t of sequence s sees
+    ctx_s + t + 1 keys."""
+    total = 0
+    lens = [int(x) for x in seq_lens]
+    cq = [int(x) for x in cu_q]
+    for s, n in enumerate(lens):
+        ql = cq[s + 1] - cq[s]
+        ctx = n - ql
+        total += ql * ctx + ql * (ql + 1) // 2
+    return 4.0 * d * Hq * total
 
 
 def decode_bytes(seq_lens, Hkv: int, d: int, Hq: int, page_size: int = 16,

@@ -118,6 +118,38 @@ EXATTN_API attn_status_t attn_fwd_f32_ext(const float *q, const float *k, const 
                                           const float *alibi_slopes, attn_stream_t stream);
 
 /*
+ * attn_prefill_paged -- chunked prefill over the paged KV cache (Phase 08
+ * page, Concepts: chunked prefill splits a long prompt over several steps so
+ * it does not block decoding; Lab 03 Extensions: add chunked prefill; paged
+ * attention as for attn_decode_paged).  Sequence s holds seq_lens[s] tokens in
+ * its pages; the current chunk is its last qlen_s = cu_q[s+1] - cu_q[s] tokens,
+ * whose K/V the caller has already written to the cache.  Chunk query t sits
+ * at position ctx_s + t (ctx_s = seq_lens[s] - qlen_s) and attends causally to
+ * keys 0 .. ctx_s + t (the causal diagonal aligned to the end of the keys);
+ * window > 0 additionally keeps only keys with ctx_s + t - j < window, and
+ * alibi_slopes add a_h * (j - (ctx_s + t)) to the scores, as for attn_fwd_ext.
+ *
+ *   q            [T, Hq, d] bf16, token-major: rows cu_q[s] .. cu_q[s+1]-1 are
+ *                sequence s's chunk (T = cu_q[S])
+ *   k_pages, v_pages, block_table, seq_lens   as for attn_decode_paged
+ *   cu_q         [S+1] int32, non-decreasing, cu_q[0] = 0, cu_q[S] = T
+ *   max_q        an upper bound of every qlen_s (sizes the grid)
+ *   o            [T, Hq, d] bf16 (out)      lse [T, Hq] float32 (out)
+ * d in {64, 128}; page_size == 16.  A sequence whose lengths are inconsistent
+ * (qlen_s < 0, qlen_s > seq_lens[s], qlen_s > max_q, cu_q[s+1] > T, or
+ * seq_lens[s] > max_blocks * 16) is skipped and sets ATTN_DEV_BAD_PAGE; one
+ * whose block table names a page outside [0, num_pages) gets NaN rows and sets
+ * it; no out-of-range address is dereferenced.  T == 0 is a no-op.
+ */
+EXATTN_API attn_status_t attn_prefill_paged(const void *q, const void *k_pages,
+                                            const void *v_pages, const int32_t *block_table,
+                                            const int32_t *seq_lens, const int32_t *cu_q,
+                                            void *o, float *lse, int S, int Hq, int Hkv, int T,
+                                            int max_q, int d, int page_size, int max_blocks,
+                                            int num_pages, float scale, int window,
+                                            const float *alibi_slopes, attn_stream_t stream);
+
+/*
  * attn_bwd -- gradients of the bf16 attention above (Phase 08 page, Concepts:
  * the FlashAttention backward needs only the output O and the logsumexp L;
  * Lab 01 step 6 and Extensions: the backward pass).  For the scalar
