@@ -11,8 +11,10 @@ The JSON line also carries, measured in the same run:
     Hkv=8) prefill TFLOP/s, and the paged GQA decode (64 sequences, context
     U[512, 8192], 16-token pages) in HBM GB/s over a bf16 cache and over 8-bit
     (E4M3, INT8) caches of the same shape, each as a fraction of the measured
-    peak; and the backward (dQ, dK, dV) of the N=8192 MHA and causal
-    workloads in TFLOP/s of the algorithm's five products;
+    peak; the chunked prefill over the paged cache (16 sequences, a 512-token
+    chunk after U[0, 7680] cached tokens) in TFLOP/s; and the backward (dQ,
+    dK, dV) of the N=8192 MHA and causal workloads in TFLOP/s of the
+    algorithm's five products;
   * ``roofline`` for the prefill kernel (tensor-bound);
   * ``e2e``: the same sweep through the public API with pinned host buffers,
     host->device and device->host copies inside the timed region;
@@ -274,6 +276,33 @@ class Backward:
         return 3  # prep + dK/dV + dQ
 
 
+class ChunkedPrefill:
+    """Chunked prefill over the paged cache (the CHUNKED workload)."""
+
+    def __init__(self, cfg, lib):
+        self.cfg, self.lib = cfg, lib
+        self.inp = syn.chunked_inputs(cfg, device="cuda")
+        i = self.inp
+        self.T = int(i["q"].shape[0])
+        self.o = torch.empty_like(i["q"])
+        self.lse = torch.empty(self.T, cfg.Hq, dtype=torch.float32, device="cuda")
+        self.num_pages = int(i["k_pages"].shape[0])
+        self.flops = syn.chunked_flops(i["seq_lens"].cpu().tolist(), i["cu_q"].cpu().tolist(),
+                                       cfg.Hq, cfg.d)
+
+    def launch(self):
+        c, i = self.cfg, self.inp
+        rc = self.lib.attn_prefill_paged(
+            i["q"].data_ptr(), i["k_pages"].data_ptr(), i["v_pages"].data_ptr(),
+            i["block_table"].data_ptr(), i["seq_lens"].data_ptr(), i["cu_q"].data_ptr(),
+            self.o.data_ptr(), self.lse.data_ptr(), c.S, c.Hq, c.Hkv, self.T, c.qlen, c.d,
+            c.page_size, c.max_blocks, self.num_pages, c.scale, 0, None,
+            torch.cuda.current_stream().cuda_stream)
+        if rc != 0:
+            raise RuntimeError("attn_prefill_paged failed: %d" % rc)
+        return 1
+
+
 class DecodeQ8:
     """The decode workload over an 8-bit cache (same q, lengths and placement)."""
 
@@ -488,6 +517,14 @@ def run_ours(args):
             tf = cfg.flops / sec / 1e12
             comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3}
             del it
+        it = ChunkedPrefill(syn.CHUNKED, lib)
+        timed_launches([it], flush, 3)
+        t, _ = timed_launches([it], flush, args.component_reps)
+        sec = sum(t[0]) / len(t[0]) / 1e3
+        tf = it.flops / sec / 1e12
+        comps[syn.CHUNKED.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3,
+                                   "flops": it.flops, "flops_counted": "4*d per visible pair"}
+        del it
         for cfg in (syn.MHA_SWEEP[-1], syn.CAUSAL):
             it = Backward(cfg, lib)
             timed_launches([it], flush, 3)
@@ -552,6 +589,8 @@ def run_only(args):
     bwd = {"bwd_" + c.name: c for c in (syn.MHA_SWEEP[-1], syn.CAUSAL, syn.MHA_SWEEP[0])}
     if args.only in bwd:
         it = Backward(bwd[args.only], lib)
+    elif args.only == syn.CHUNKED.name:
+        it = ChunkedPrefill(syn.CHUNKED, lib)
     elif args.only == syn.DECODE.name:
         it = Decode(syn.DECODE, lib)
     elif args.only in q8:
@@ -560,7 +599,7 @@ def run_only(args):
         it = Prefill(table[args.only], lib)
     else:
         raise SystemExit("unknown workload %r; one of %s"
-                         % (args.only, sorted(table) + [syn.DECODE.name] + sorted(q8) + sorted(bwd)))
+                         % (args.only, sorted(table) + [syn.DECODE.name] + sorted(q8) + sorted(bwd) + [syn.CHUNKED.name]))
     for _ in range(args.reps):
         it.launch()
     torch.cuda.synchronize()
