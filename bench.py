@@ -586,7 +586,7 @@ def run_only(args):
     lib = ea.library()
     table = {c.name: c for c in syn.MHA_SWEEP + (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI)}
     q8 = {syn.DECODE.name + "_" + f: f for f in ("e4m3", "int8")}
-    bwd = {"bwd_" + c.name: c for c in (syn.MHA_SWEEP[-1], syn.CAUSAL, syn.MHA_SWEEP[0])}
+    bwd = {"bwd_" + c.name: c for c in (syn.MHA_SWEEP[-1], syn.CAUSAL, syn.MHA_SWEEP[2])}
     if args.only in bwd:
         it = Backward(bwd[args.only], lib)
     elif args.only == syn.CHUNKED.name:
