@@ -21,19 +21,24 @@
 // E4M3 and INT8 codes convert to f16 exactly (cvt.rn.f16x2.e4m3x2; for INT8
 // the byte goes into the mantissa of 1024 and 1152 is subtracted), so the only
 // roundings are Q's (bf16 -> f16 after a per-head power-of-two normalisation,
-// exact for every element within 2^28 of the head's largest), P's (f16) and
-// the f32 accumulations.  The page scales are applied in f32: the K scale to
-// the scores, the V scale when the page's P.V is added to the accumulator.
+// exact for every element within 2^28 of the head's largest), the p.v
+// operand's (f16) and the f32 accumulations.  The page scales are applied in
+// f32: the K scale to the scores; the V scale multiplies P before it is
+// rounded to f16, relative to the running largest contribution, so the f16
+// operand is each token's actual contribution.
 //
-// Data movement.  One CTA per (chunk of kPagesPerSplit pages, K/V head, head
-// chunk, sequence); warp 4 is the producer: it TMA-loads each page's K and V
-// slices (16 rows x d bytes, 128-byte swizzle for d = 128, 64-byte for d = 64)
-// into a kStages-deep ring.  The swizzle makes both fragment patterns
-// conflict-free: K rows read along d, and V read across token rows at one
-// column.  Warps 0..3 take pages round-robin, keep a running max / sum per
-// head (online softmax, lazily rescaled), and the CTA merges them into one
-// normalised partial per head; the combine kernel of decode_paged.cu merges
-// the chunks exactly as for the 16-bit cache.
+// Data movement.  At one byte per element a (page, K/V head) slice is only
+// 2 KiB, and a stream of such copies was measured to stop near 4 TB/s however
+// it was placed or staged.  So the kernel is page-major: one CTA serves up to
+// 8 K/V heads of a chunk of a sequence's pages, and each page arrives as one
+// TMA box holding all those heads' slices (16 KiB of K, 16 KiB of V at d =
+// 128, contiguous in the pool).  The box is 128-byte swizzled (64-byte for d =
+// 64), which makes both fragment patterns conflict-free: K rows read along d,
+// and V read across token rows at one column.  Each consumer warp owns one
+// K/V head, walks every page of the chunk with a running max / sum (online
+// softmax, lazily rescaled), and writes its heads' normalised partials; the
+// combine kernel of decode_paged.cu merges the chunks exactly as for the
+// 16-bit cache.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -48,15 +53,9 @@ namespace exattn {
 namespace {
 
 constexpr int kPage = 16;
-// 64 pages (1024 tokens) per chunk: at one byte per element a chunk holds as
-// many bytes as the 16-bit kernel's 32-page chunk, so start-up (block table,
-// first copies) is amortised as well; the workspace of the 32-page chunking
-// is larger than this one needs.
-constexpr int kPagesPerSplitQ8 = 64;
-constexpr int kWarpsQ8 = 4;
-// 16 stages of 4 KiB (d = 128): the same bytes in flight per CTA as the 16-bit
-// kernel's 8 stages of 8 KiB.
-constexpr int kStagesQ8 = 16;
+// 32 pages (512 tokens) per chunk, as the 16-bit kernel (same workspace); a
+// chunk of 8 K/V heads is 1 MiB of codes.
+constexpr int kPagesPerSplitQ8 = 32;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale: move the max only when it grows by > 2^8
 
 template <int D>
@@ -167,8 +166,26 @@ __device__ __forceinline__ VRow<D> load_vrow(const uint8_t *tile, int row, int g
 // Workspace and partial layout as in decode_paged.cu: o_part [S][Hq][nsplit][D]
 // f32 (normalised), l2_part [S][Hq][nsplit] f32 (log2-sum-exp; NaN marks a bad
 // sequence).
-template <int D, int GB, int FMT>
-__global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
+//
+// One CTA per (chunk of kPagesPerSplitQ8 pages, sequence, group of HC K/V
+// heads, chunk of GB query heads per K/V head).  Warp HC is the producer: its
+// lane 0 TMA-loads, per page, the page's K slices of all HC heads as one box
+// (HC x 16 rows x d bytes, contiguous in the pool) and likewise V, into a
+// ring of NST stages.  Warp w < HC owns K/V head g0 + w: it walks every page
+// of the chunk, keeps its own running max / sum / accumulator, and writes its
+// heads' normalised partials; no cross-warp merge.
+template <int HC, int D>
+struct Q8Cfg {
+  static constexpr int SLICE = kPage * D;       // one (page, head) slice of K (or V)
+  static constexpr int STAGE = 2 * HC * SLICE;  // K and V of all HC heads of one page
+  // Bytes in flight: 6 x 32 KiB for 8 heads (one CTA per SM); more stages
+  // for fewer heads, whose CTAs share an SM.
+  static constexpr int NST = (HC >= 4) ? 6 : 12;
+  static constexpr int SMEM = NST * STAGE + 1024;
+};
+
+template <int D, int GB, int FMT, int HC>
+__global__ void __launch_bounds__((HC + 1) * 32)
     decode_q8_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const __nv_bfloat16 *__restrict__ q, const float *__restrict__ k_scales,
@@ -177,21 +194,19 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
                            float *__restrict__ o_part, float *__restrict__ l2_part, int Hq,
                            int Hkv, int max_blocks, int num_pages, float scale_log2, int nsplit,
                            int head_chunks, unsigned *status) {
+  using C = Q8Cfg<HC, D>;
   constexpr int KS = D / 16;   // k-steps of the q.k MMA = M-tiles of the p.v MMA
   constexpr int KCH = D / 64;  // 16-byte chunks of a K row held by one thread
-  constexpr int TILE = tile_bytes<D>();
-  constexpr int STAGE = 2 * TILE;
-  static_assert(GB >= 1 && GB <= 8, "one n8 tile of heads per CTA");
-  static_assert(kPagesPerSplitQ8 <= 64 && kPagesPerSplitQ8 / kWarpsQ8 <= 32,
-                "two block-table entries per producer lane, one page per consumer lane");
-  static_assert(kWarpsQ8 * GB * D * 4 + 2 * kWarpsQ8 * GB * 4 <= kStagesQ8 * STAGE,
-                "the merge scratch fits in the ring");
+  static_assert(GB >= 1 && GB <= 8, "one n8 tile of heads per warp");
+  static_assert(kPagesPerSplitQ8 <= 32, "one block-table entry and one page's scales per lane");
   const int split = blockIdx.x;
-  const int kvh = blockIdx.y / head_chunks;
-  const int h0 = kvh * (Hq / Hkv) + (blockIdx.y % head_chunks) * GB;
-  const int s = blockIdx.z;
+  const int s = blockIdx.y;
+  const int kvgrp = blockIdx.z / head_chunks;
+  const int hchunk = blockIdx.z % head_chunks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;  // MMA fragment coordinates
+  const int kvh = kvgrp * HC + min(warp, HC - 1);  // this consumer warp's K/V head
+  const int h0 = kvh * (Hq / Hkv) + hchunk * GB;   // its first query head
 
   const int len = seq_lens[s];
   const bool bad_len = len < 0 || len > max_blocks * kPage;
@@ -203,37 +218,30 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t full[kStagesQ8], empty[kStagesQ8];
-  __shared__ int stage_ntok[kStagesQ8];
+  __shared__ uint64_t full[C::NST], empty[C::NST];
+  __shared__ int stage_ntok[C::NST];
   __shared__ int sm_pid[kPagesPerSplitQ8];
   __shared__ int sm_bad, sm_abort;
-  // Merge scratch, over the ring once every page has been consumed.
-  float(*sm_acc)[GB][D] = reinterpret_cast<float(*)[GB][D]>(ring);
-  float(*sm_m)[GB] = reinterpret_cast<float(*)[GB]>(ring + kWarpsQ8 * GB * D * 4);
-  float(*sm_l)[GB] = reinterpret_cast<float(*)[GB]>(ring + kWarpsQ8 * GB * D * 4 + kWarpsQ8 * GB * 4);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStagesQ8; ++i) {
+    for (int i = 0; i < C::NST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], HC);
     }
     sm_bad = bad_len ? 1 : 0;
     sm_abort = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpsQ8) {
-    for (int i = lane; i < npg; i += 32)
-      sm_pid[i] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + i];
-  }
+  if (warp == HC && lane < npg)
+    sm_pid[lane] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + lane];
   __syncthreads();
 
-  if (warp == kWarpsQ8) {
+  if (warp == HC) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < npg; ++i) {
-        const int st = i % kStagesQ8;
-        if (i >= kStagesQ8 &&
-            !mbar_wait(&empty[st], ((i / kStagesQ8) - 1) & 1, &sm_abort, status))
+        const int st = i % C::NST;
+        if (i >= C::NST && !mbar_wait(&empty[st], ((i / C::NST) - 1) & 1, &sm_abort, status))
           break;
         const int pid = sm_pid[i];
         if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
@@ -242,17 +250,17 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
           mbar_arrive(&full[st]);
         } else {
           stage_ntok[st] = min(kPage, len - (page_begin + i) * kPage);
-          uint8_t *dst = ring + st * STAGE;
-          const int z = pid * Hkv + kvh;
-          mbar_arrive_expect_tx(&full[st], STAGE);
+          uint8_t *dst = ring + st * C::STAGE;
+          const int z = pid * Hkv + kvgrp * HC;
+          mbar_arrive_expect_tx(&full[st], C::STAGE);
           tma_load_3d(dst, &tm_k, &full[st], 0, 0, z);
-          tma_load_3d(dst + TILE, &tm_v, &full[st], 0, 0, z);
+          tma_load_3d(dst + HC * C::SLICE, &tm_v, &full[st], 0, 0, z);
         }
         issued = i + 1;
       }
       // Let every copy land before the CTA (and its shared memory) goes away.
-      for (int i = max(0, issued - kStagesQ8); i < issued; ++i)
-        mbar_wait_drain(&full[i % kStagesQ8], (i / kStagesQ8) & 1, status);
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
+        mbar_wait_drain(&full[i % C::NST], (i / C::NST) & 1, status);
     }
   } else {
     // ------------------------------------------------------------ compute
@@ -303,22 +311,29 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
     const float sq0 = __shfl_sync(0xffffffffu, sq_own, 8 * c);
     const float sq1 = __shfl_sync(0xffffffffu, sq_own, 8 * c + 4);
 
-    // Page scales of this warp's pages: lane j holds those of its j-th page.
+    // Page scales: lane i holds those of page i of the chunk.
     float ks_r = 0.f, vs_r = 0.f;
-    {
-      const int i = warp + kWarpsQ8 * lane;
-      if (lane < kPagesPerSplitQ8 / kWarpsQ8 && i < npg) {
-        const int pid = sm_pid[i];
-        if (pid >= 0 && pid < num_pages) {
-          ks_r = k_scales[static_cast<size_t>(pid) * Hkv + kvh];
-          vs_r = v_scales[static_cast<size_t>(pid) * Hkv + kvh];
-        }
+    if (lane < npg) {
+      const int pid = sm_pid[lane];
+      if (pid >= 0 && pid < num_pages) {
+        ks_r = k_scales[static_cast<size_t>(pid) * Hkv + kvh];
+        vs_r = v_scales[static_cast<size_t>(pid) * Hkv + kvh];
       }
     }
 
-    float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2c, 2c+1 (log2 units)
+    // Two running references per head (columns 2c, 2c+1), both lazily moved
+    // (only when exceeded by more than 2^8): m for the scores, which normalise
+    // the sum l (fp32), and mv for the log2 contribution scale score + log2(V
+    // scale), which normalises the f16 operand of the p.v MMA.  The operand is
+    // then each token's contribution relative to the largest one, so it stays
+    // below 2^9 and underflows only for contributions below 2^-24 of the
+    // largest -- not when a page with a large V scale is barely attended.
+    // The accumulator holds sum_t 2^(s_t - mv) * vscale_t * code_t, so
+    // O = acc * 2^(mv - m) / l.
+    float m0 = -INFINITY, m1 = -INFINITY;
+    float mv0 = -INFINITY, mv1 = -INFINITY;
     float l0 = 0.f, l1 = 0.f;              // this thread's share of the running sums
-    float acc[KS][4];                      // O^T: rows d = (D/8)g + 2i (+1), cols 2c, 2c+1
+    float acc[KS][4];                      // rows d = (D/8)g + 2i (+1), cols 2c, 2c+1
 #pragma unroll
     for (int i = 0; i < KS; ++i)
 #pragma unroll
@@ -327,16 +342,16 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
     const int src0 = 8 * c + (g >> 1), src1 = src0 + 4;
     const uint32_t psel = (g & 1) ? 0x7632u : 0x5410u;
 
-    for (int j = 0, i = warp; i < npg; ++j, i += kWarpsQ8) {
-      const int st = i % kStagesQ8;
-      const bool ok = mbar_wait(&full[st], (i / kStagesQ8) & 1, &sm_abort, status);
+    for (int i = 0; i < npg; ++i) {
+      const int st = i % C::NST;
+      const bool ok = mbar_wait(&full[st], (i / C::NST) & 1, &sm_abort, status);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int ntok = stage_ntok[st];
-      const float ks = __shfl_sync(0xffffffffu, ks_r, j);
-      const float vs = __shfl_sync(0xffffffffu, vs_r, j);
+      const float ks = __shfl_sync(0xffffffffu, ks_r, i);
+      const float vs = __shfl_sync(0xffffffffu, vs_r, i);
       if (ntok > 0) {
-        const uint8_t *kt = ring + st * (2 * TILE);
-        const uint8_t *vt = kt + TILE;
+        const uint8_t *kt = ring + st * C::STAGE + warp * C::SLICE;
+        const uint8_t *vt = ring + st * C::STAGE + (HC + warp) * C::SLICE;
         // ---- S^T = K . Q^T for tokens g and g+8.
         uint4 ka[KCH], kb[KCH];
 #pragma unroll
@@ -370,14 +385,22 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
         }
-        const bool grow = (mx0 > m0 + kRescaleLog2) || (mx1 > m1 + kRescaleLog2);
-        if (__any_sync(0xffffffffu, grow)) {
+        if (__any_sync(0xffffffffu, (mx0 > m0 + kRescaleLog2) || (mx1 > m1 + kRescaleLog2))) {
           const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-          const float a0 = ex2(m0 - n0), a1 = ex2(m1 - n1);
+          l0 *= ex2(m0 - n0);
+          l1 *= ex2(m1 - n1);
           m0 = n0;
           m1 = n1;
-          l0 *= a0;
-          l1 *= a1;
+        }
+        const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        // ---- contribution scale of the page: its score max plus log2(V scale).
+        const float lvs = vs > 0.f ? __log2f(vs) : -INFINITY;
+        const float cv0 = mx0 + lvs, cv1 = mx1 + lvs;
+        if (__any_sync(0xffffffffu, (cv0 > mv0 + kRescaleLog2) || (cv1 > mv1 + kRescaleLog2))) {
+          const float n0 = fmaxf(mv0, cv0), n1 = fmaxf(mv1, cv1);
+          const float a0 = ex2(mv0 - n0), a1 = ex2(mv1 - n1);  // 0 while mv was -inf
 #pragma unroll
           for (int i2 = 0; i2 < KS; ++i2) {
             acc[i2][0] *= a0;
@@ -385,12 +408,14 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
             acc[i2][2] *= a0;
             acc[i2][3] *= a1;
           }
+          mv0 = n0;
+          mv1 = n1;
         }
-        const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
-        l0 += p0 + p2;
-        l1 += p1 + p3;
+        // f16 operand: p * vscale * 2^(m - mv) = 2^(s + log2 vscale - mv).
+        const float f0 = mv0 == -INFINITY ? 0.f : vs * ex2(m0 - mv0);
+        const float f1 = mv1 == -INFINITY ? 0.f : vs * ex2(m1 - mv1);
         // ---- P^T fragment: (P[head g][tok 2c], [2c+1]) and tokens 2c+8, 2c+9.
-        const uint32_t P01 = pack_f16x2(p0, p1), P23 = pack_f16x2(p2, p3);
+        const uint32_t P01 = pack_f16x2(p0 * f0, p1 * f1), P23 = pack_f16x2(p2 * f0, p3 * f1);
         const uint32_t x0 = __shfl_sync(0xffffffffu, P01, src0);
         const uint32_t x1 = __shfl_sync(0xffffffffu, P01, src1);
         const uint32_t y0 = __shfl_sync(0xffffffffu, P23, src0);
@@ -411,10 +436,10 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
             float t4[4] = {0.f, 0.f, 0.f, 0.f};
             mma_f16(t4, lo[2 * e2], lo[2 * e2 + 1], hi[2 * e2], hi[2 * e2 + 1], pb0, pb1);
             float(&a)[4] = acc[2 * w + e2];
-            a[0] = fmaf(t4[0], vs, a[0]);
-            a[1] = fmaf(t4[1], vs, a[1]);
-            a[2] = fmaf(t4[2], vs, a[2]);
-            a[3] = fmaf(t4[3], vs, a[3]);
+            a[0] += t4[0];
+            a[1] += t4[1];
+            a[2] += t4[2];
+            a[3] += t4[3];
           }
         }
       }
@@ -422,70 +447,51 @@ __global__ void __launch_bounds__((kWarpsQ8 + 1) * 32, 3)
       if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
     }
 
-    // Sums over the warp's tokens (lanes sharing c hold the same heads).
+    // Sums over the page tokens (lanes sharing c hold the same heads).
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
-    // The merge scratch lives in the ring: wait until every warp is done with it.
-    asm volatile("bar.sync 1, %0;" ::"n"(kWarpsQ8 * 32) : "memory");
+    // sm_bad / sm_abort are final once every page has been consumed.
+    __syncwarp();
+    const bool bad = *reinterpret_cast<volatile int *>(&sm_bad) != 0 ||
+                     *reinterpret_cast<volatile int *>(&sm_abort) != 0;
+    // O = acc * 2^(mv - m) / l.
+    const float inv0 = (mv0 == -INFINITY ? 0.f : ex2(mv0 - m0)) / l0;
+    const float inv1 = (mv1 == -INFINITY ? 0.f : ex2(mv1 - m1)) / l1;
     const int hA = 2 * c, hB = 2 * c + 1;
+    const size_t slotA = (static_cast<size_t>(s) * Hq + h0 + hA) * nsplit + split;
+    const size_t slotB = (static_cast<size_t>(s) * Hq + h0 + hB) * nsplit + split;
 #pragma unroll
     for (int i = 0; i < KS; ++i) {
       const int d0 = (D / 8) * g + 2 * i;
-      if (hA < GB) {
-        sm_acc[warp][hA][d0] = acc[i][0];
-        sm_acc[warp][hA][d0 + 1] = acc[i][2];
-      }
-      if (hB < GB) {
-        sm_acc[warp][hB][d0] = acc[i][1];
-        sm_acc[warp][hB][d0 + 1] = acc[i][3];
-      }
+      if (hA < GB)
+        *reinterpret_cast<float2 *>(o_part + slotA * D + d0) =
+            bad ? make_float2(NAN, NAN) : make_float2(acc[i][0] * inv0, acc[i][2] * inv0);
+      if (hB < GB)
+        *reinterpret_cast<float2 *>(o_part + slotB * D + d0) =
+            bad ? make_float2(NAN, NAN) : make_float2(acc[i][1] * inv1, acc[i][3] * inv1);
     }
     if (g == 0) {
-      if (hA < GB) {
-        sm_m[warp][hA] = m0;
-        sm_l[warp][hA] = l0;
-      }
-      if (hB < GB) {
-        sm_m[warp][hB] = m1;
-        sm_l[warp][hB] = l1;
-      }
+      if (hA < GB) l2_part[slotA] = bad ? NAN : m0 + log2f(l0);
+      if (hB < GB) l2_part[slotB] = bad ? NAN : m1 + log2f(l1);
     }
   }
   __syncthreads();
-
-  // Merge the warps and write this chunk's normalised partial per head.
-  const bool bad = sm_bad != 0 || sm_abort != 0;
-  if (bad && threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
-  for (int idx = threadIdx.x; idx < GB * D; idx += blockDim.x) {
-    const int hh = idx / D, col = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarpsQ8; ++w) M = fmaxf(M, sm_m[w][hh]);
-    float wsum = 0.f, num = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarpsQ8; ++w) {
-      const float wt = (sm_m[w][hh] == -INFINITY) ? 0.f : ex2(sm_m[w][hh] - M);
-      wsum += wt * sm_l[w][hh];
-      num += wt * sm_acc[w][hh][col];
-    }
-    const size_t slot = (static_cast<size_t>(s) * Hq + h0 + hh) * nsplit + split;
-    o_part[slot * D + col] = bad ? NAN : num / wsum;
-    if (col == 0) l2_part[slot] = bad ? NAN : M + log2f(wsum);
-  }
+  if (threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
 }
 
 // Page pool [num_pages][Hkv][16][D] bytes as a 3-D tensor (D, 16, num_pages*Hkv);
-// one box is one page slice of one K/V head.
-bool make_page_map(CUtensorMap *map, const void *base, int D, long long slices) {
+// one box is the page slices of `hc` consecutive K/V heads.
+bool make_page_map(CUtensorMap *map, const void *base, int D, long long slices, int hc) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(kPage),
                         static_cast<cuuint64_t>(slices)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(kPage) * D};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(kPage), 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(kPage),
+                       static_cast<cuuint32_t>(hc)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -494,36 +500,50 @@ bool make_page_map(CUtensorMap *map, const void *base, int D, long long slices) 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int GB, int FMT>
+template <int D, int GB, int FMT, int HC>
 attn_status_t launch_split_q8(dim3 grid, cudaStream_t st, const CUtensorMap &mk,
                               const CUtensorMap &mv, const void *q, const float *ks,
                               const float *vs, const int *bt, const int *sl, float *op, float *lp,
                               int Hq, int Hkv, int maxb, int npages, float sl2, int nsplit, int hc,
                               unsigned *status) {
-  constexpr int kSmem = kStagesQ8 * 2 * tile_bytes<D>() + 1024;
+  using C = Q8Cfg<HC, D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(decode_q8_split_kernel<D, GB, FMT>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    attr_err = cudaFuncSetAttribute(decode_q8_split_kernel<D, GB, FMT, HC>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-  decode_q8_split_kernel<D, GB, FMT><<<grid, (kWarpsQ8 + 1) * 32, kSmem, st>>>(
+  decode_q8_split_kernel<D, GB, FMT, HC><<<grid, (HC + 1) * 32, C::SMEM, st>>>(
       mk, mv, static_cast<const __nv_bfloat16 *>(q), ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages,
       sl2, nsplit, hc, status);
   return ATTN_OK;
 }
 
-template <int D, int FMT>
-attn_status_t dispatch_q8(int GB, dim3 grid, cudaStream_t st, const CUtensorMap &mk,
+template <int D, int FMT, int HC>
+attn_status_t dispatch_gb(int GB, dim3 grid, cudaStream_t st, const CUtensorMap &mk,
                           const CUtensorMap &mv, const void *q, const float *ks, const float *vs,
                           const int *bt, const int *sl, float *op, float *lp, int Hq, int Hkv,
                           int maxb, int npages, float sl2, int nsplit, int hc, unsigned *status) {
   switch (GB) {
-    case 8: return launch_split_q8<D, 8, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
-    case 4: return launch_split_q8<D, 4, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
-    case 2: return launch_split_q8<D, 2, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
-    case 1: return launch_split_q8<D, 1, FMT>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 8: return launch_split_q8<D, 8, FMT, HC>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 4: return launch_split_q8<D, 4, FMT, HC>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 2: return launch_split_q8<D, 2, FMT, HC>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 1: return launch_split_q8<D, 1, FMT, HC>(grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+  }
+  return ATTN_ERR_UNSUPPORTED;
+}
+
+template <int D, int FMT>
+attn_status_t dispatch_q8(int HC, int GB, dim3 grid, cudaStream_t st, const CUtensorMap &mk,
+                          const CUtensorMap &mv, const void *q, const float *ks, const float *vs,
+                          const int *bt, const int *sl, float *op, float *lp, int Hq, int Hkv,
+                          int maxb, int npages, float sl2, int nsplit, int hc, unsigned *status) {
+  switch (HC) {
+    case 8: return dispatch_gb<D, FMT, 8>(GB, grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 4: return dispatch_gb<D, FMT, 4>(GB, grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 2: return dispatch_gb<D, FMT, 2>(GB, grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 1: return dispatch_gb<D, FMT, 1>(GB, grid, st, mk, mv, q, ks, vs, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
   }
   return ATTN_ERR_UNSUPPORTED;
 }
@@ -539,28 +559,30 @@ attn_status_t launch_decode_paged_q8(const void *q, const void *k_pages, const v
   const int G = Hq / Hkv;
   const int GB = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
   const int head_chunks = G / GB;
+  const int HC = (Hkv % 8 == 0) ? 8 : (Hkv % 4 == 0) ? 4 : (Hkv % 2 == 0) ? 2 : 1;
   const int nsplit = (max_blocks + kPagesPerSplitQ8 - 1) / kPagesPerSplitQ8;
   const size_t parts = static_cast<size_t>(S) * Hq * nsplit;
   float *o_part = static_cast<float *>(workspace);
   float *l2_part = reinterpret_cast<float *>(
       static_cast<uint8_t *>(workspace) +
       ((parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255)));
-  if (static_cast<long long>(Hkv) * head_chunks > 65535 || S > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(Hkv / HC) * head_chunks > 65535 || S > 65535)
+    return ATTN_ERR_UNSUPPORTED;
   CUtensorMap mk, mv;
   const long long slices = static_cast<long long>(num_pages) * Hkv;
-  if (!make_page_map(&mk, k_pages, d, slices) || !make_page_map(&mv, v_pages, d, slices))
+  if (!make_page_map(&mk, k_pages, d, slices, HC) || !make_page_map(&mv, v_pages, d, slices, HC))
     return ATTN_ERR_CUDA;
-  dim3 grid(nsplit, Hkv * head_chunks, S);
+  dim3 grid(nsplit, S, (Hkv / HC) * head_chunks);
   const float sl2 = scale * 1.4426950408889634f;
   attn_status_t st;
   if (d == 128 && kv_format == ATTN_KV_E4M3)
-    st = dispatch_q8<128, ATTN_KV_E4M3>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+    st = dispatch_q8<128, ATTN_KV_E4M3>(HC, GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
   else if (d == 128 && kv_format == ATTN_KV_INT8)
-    st = dispatch_q8<128, ATTN_KV_INT8>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+    st = dispatch_q8<128, ATTN_KV_INT8>(HC, GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
   else if (d == 64 && kv_format == ATTN_KV_E4M3)
-    st = dispatch_q8<64, ATTN_KV_E4M3>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+    st = dispatch_q8<64, ATTN_KV_E4M3>(HC, GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
   else if (d == 64 && kv_format == ATTN_KV_INT8)
-    st = dispatch_q8<64, ATTN_KV_INT8>(GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+    st = dispatch_q8<64, ATTN_KV_INT8>(HC, GB, grid, stream, mk, mv, q, k_scales, v_scales, block_table, seq_lens, o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
   else
     return ATTN_ERR_UNSUPPORTED;
   if (st != ATTN_OK) return st;

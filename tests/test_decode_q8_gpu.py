@@ -104,11 +104,22 @@ def test_q8_bad_page_sets_status_and_nan(fmt):
     assert ea.device_status() == 0
 
 
+def _abs_codes(codes: torch.Tensor, fmt: str) -> torch.Tensor:
+    """Codes of |value|: E4M3 with the sign bit cleared, INT8 by abs (no -128)."""
+    if fmt == "e4m3":
+        return (codes.view(torch.uint8) & 0x7F).view(torch.float8_e4m3fn)
+    return codes.abs()
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_q8_scales_over_many_binades(fmt):
     # Scales are applied in f32 per page: multiply V's by 2^-12 .. 2^12 and K's
     # by 2^-3 .. 2^3 (independently per page and head; K's range is kept small
     # so that the scores stay of the order of ten) and the result still matches.
+    # With V spread over 24 binades and mixed signs, O is a sum of terms that
+    # cancel, so the error is measured against the terms' magnitude
+    # sum_t p_t |v_t| (the oracle run on |V|), the scale the f16 / bf16
+    # roundings act on: |dO| <= 2e-2 * sum_t p_t |v_t| element-wise.
     cfg, inp = make_case([700, 260, 31], 16, 4, 128, num_pages=80, max_blocks=50, seed=8,
                          fmt=fmt)
     g = torch.Generator().manual_seed(11)
@@ -117,13 +128,12 @@ def test_q8_scales_over_many_binades(fmt):
     vmul = 2.0 ** torch.randint(-12, 13, (P, Hkv), generator=g).float()
     inp = dict(inp, k_scales=inp["k_scales"] * kmul, v_scales=inp["v_scales"] * vmul)
     o_ref, l_ref = oracle_q8(inp, cfg.scale, fmt)
+    mag, _ = oracle_q8(dict(inp, v_pages=_abs_codes(inp["v_pages"], fmt)), cfg.scale, fmt)
     o, l = gpu_q8(inp, cfg.scale, fmt)
-    # O scales with the V multipliers (up to 2^12): compare relative to the
-    # largest output of each head.
     of = f32(o).astype(np.float64)
-    scale_o = np.maximum(np.abs(o_ref).max(axis=-1, keepdims=True), 1e-30)
     assert np.all(np.isfinite(of))
-    assert np.max(np.abs(of - o_ref) / scale_o) <= 2e-2
+    ratio = np.abs(of - o_ref) / (2e-2 * mag + 1e-30)
+    assert ratio.max() <= 1.0, (fmt, float(ratio.max()))
     assert np.max(np.abs(f32(l) - l_ref)) <= 5e-3
 
 
