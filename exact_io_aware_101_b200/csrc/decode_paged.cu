@@ -9,13 +9,14 @@
 //
 // Decode is bound by HBM bandwidth (quiz page, question 1: few FLOPs per byte),
 // so the design is about moving each K/V byte exactly once at full rate:
-//  * split kernel: one CTA per (key chunk of kPagesPerSplit pages, K/V head,
-//    sequence).  Each warp takes every 4th page of the chunk and reads it with
-//    16-byte vector loads (a 16 x d page slice is one contiguous 4 KiB run for
-//    d = 128), scores it for the group's query heads (warp-shuffle reductions),
-//    and folds it into a running max / sum / accumulator (online softmax, Lab 01
-//    talking points).  The CTA merges its warps and writes one normalised
-//    partial output and its log2-sum-exp per head to the workspace.
+//  * split kernel: one CTA per (key chunk of kPagesPerSplit pages, sequence,
+//    group of up to 8 K/V heads).  A producer warp brings each page of the
+//    chunk into shared memory with one bulk copy per tensor covering all the
+//    group's heads (they are contiguous in the pool); each compute warp owns
+//    one K/V head, scores every page for the head's query heads (warp-shuffle
+//    reductions), folds it into a running max / sum / accumulator (online
+//    softmax, Lab 01 talking points), and writes one normalised partial
+//    output and its log2-sum-exp per head to the workspace.
 //  * combine kernel: per (sequence, head), merges the chunks' partials with
 //    weights 2^(L_r - L) -- the same rescaling rule applied across chunks --
 //    and writes O (bf16) and L (natural log, float32).
@@ -33,7 +34,6 @@ namespace {
 
 constexpr int kPageSize = 16;
 constexpr int kPagesPerSplit = 32;  // 512 tokens per chunk
-constexpr int kWarps = 4;
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -50,21 +50,25 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-constexpr int kStages = 8;  // shared-memory ring of (K page, V page) slices
-
-template <int D>
-constexpr int stage_bytes() { return 2 * kPageSize * D * 2; }
+// Page-major: one CTA per (chunk of kPagesPerSplit pages, sequence, group of
+// HC K/V heads, chunk of GB query heads per K/V head).  The K slices of the HC
+// heads of one page are contiguous in the pool ([page][head][16][d]), so warp
+// HC (the producer) brings each page in with one bulk copy per tensor -- 32 KiB
+// of K and 32 KiB of V for 8 heads at d = 128 -- instead of one small copy per
+// (page, head): a stream of small copies stops well short of the HBM rate.
+// Warp w < HC owns K/V head g0 + w and walks every page of the chunk.
+template <int HC, int D>
+struct DecCfg {
+  static constexpr int SLICE = kPageSize * D * 2;  // bytes of one (page, head) K or V slice
+  static constexpr int STAGE = 2 * HC * SLICE;
+  static constexpr int NST = (196608 / STAGE) < 2 ? 2 : ((196608 / STAGE) > 8 ? 8 : 196608 / STAGE);
+  static constexpr int SMEM = NST * STAGE;
+};
 
 // Workspace: o_part [S][Hq][nsplit][D] f32 (normalised), l2_part [S][Hq][nsplit]
 // f32 (log2-sum-exp of scale*log2(e)*scores over the chunk; NaN marks a bad sequence).
-//
-// Warps 0..kWarps-1 compute; warp kWarps is the producer: its lane 0 copies the
-// visible rows of each page's K and V slices into a kStages-deep shared-memory
-// ring with bulk async copies, so the bytes in flight do not depend on how many
-// registers the compute warps hold.  Page i of the chunk goes to stage
-// i % kStages and is consumed by warp i % kWarps.
-template <int D, int GB>
-__global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
+template <int D, int GB, int HC>
+__global__ void __launch_bounds__((HC + 1) * 32)
     decode_split_kernel(const __nv_bfloat16 *__restrict__ q,
                         const __nv_bfloat16 *__restrict__ k_pages,
                         const __nv_bfloat16 *__restrict__ v_pages,
@@ -72,16 +76,18 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
                         float *__restrict__ o_part, float *__restrict__ l2_part, int Hq, int Hkv,
                         int max_blocks, int num_pages, float scale_log2, int nsplit,
                         int head_chunks, unsigned *status) {
+  using C = DecCfg<HC, D>;
   constexpr int LPT = D / 8;           // lanes per token row (8 bf16 = 16 B each)
   constexpr int TPI = 32 / LPT;        // token rows per warp-wide access
   constexpr int IT = kPageSize / TPI;  // accesses per page per lane
-  constexpr int SLICE = kPageSize * D; // elements of one page's K (or V) slice
   static_assert(kPagesPerSplit <= 32, "one block-table entry per producer lane");
   const int split = blockIdx.x;
-  const int g = blockIdx.y / head_chunks;
-  const int h0 = g * (Hq / Hkv) + (blockIdx.y % head_chunks) * GB;
-  const int s = blockIdx.z;
+  const int s = blockIdx.y;
+  const int kvgrp = blockIdx.z / head_chunks;
+  const int hchunk = blockIdx.z % head_chunks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = kvgrp * HC + min(warp, HC - 1);      // this consumer warp's K/V head
+  const int h0 = g * (Hq / Hkv) + hchunk * GB;       // its first query head
   const int sub = lane / LPT;          // token row of an access held by this lane
   const int dc = lane % LPT;           // 8-column slice held by this lane
 
@@ -93,52 +99,51 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
   const int npg = bad_len ? 0 : min(n_pages, page_begin + kPagesPerSplit) - page_begin;
 
   extern __shared__ __align__(128) uint8_t ring[];
-  __shared__ uint64_t full[kStages], empty[kStages];
-  __shared__ int stage_ntok[kStages];
+  __shared__ uint64_t full[C::NST], empty[C::NST];
+  __shared__ int stage_ntok[C::NST];
   __shared__ int sm_pid[kPagesPerSplit];
-  __shared__ float sm_m[kWarps][GB], sm_l[kWarps][GB];
-  __shared__ float sm_acc[kWarps][GB][D];
   __shared__ int sm_bad, sm_abort;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < C::NST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], HC);
     }
     sm_bad = bad_len ? 1 : 0;
     sm_abort = 0;
     fence_mbar_init();
   }
+  if (warp == HC && lane < npg)
+    sm_pid[lane] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + lane];
   __syncthreads();
 
-  if (warp == kWarps) {
+  if (warp == HC) {
     // ------------------------------------------------------------ producer
-    if (lane < npg) sm_pid[lane] = block_table[static_cast<size_t>(s) * max_blocks + page_begin + lane];
-    __syncwarp();
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < npg; ++i) {
-        const int st = i % kStages;
-        if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1, &sm_abort, status)) break;
+        const int st = i % C::NST;
+        if (i >= C::NST && !mbar_wait(&empty[st], ((i / C::NST) - 1) & 1, &sm_abort, status))
+          break;
         const int pid = sm_pid[i];
-        const int ntok = min(kPageSize, len - (page_begin + i) * kPageSize);
         if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
           sm_bad = 1;
           stage_ntok[st] = 0;
           mbar_arrive(&full[st]);
         } else {
-          stage_ntok[st] = ntok;
-          const uint32_t bytes = static_cast<uint32_t>(ntok * D * 2);
-          const size_t base = (static_cast<size_t>(pid) * Hkv + g) * SLICE;
-          uint8_t *dst = ring + st * stage_bytes<D>();
-          mbar_arrive_expect_tx(&full[st], 2 * bytes);
-          bulk_load(dst, k_pages + base, bytes, &full[st]);
-          bulk_load(dst + SLICE * 2, v_pages + base, bytes, &full[st]);
+          // The whole page (16 rows of every head); rows past the sequence end
+          // are never read by the compute warps.
+          stage_ntok[st] = min(kPageSize, len - (page_begin + i) * kPageSize);
+          const size_t base = (static_cast<size_t>(pid) * Hkv + kvgrp * HC) * (C::SLICE / 2);
+          uint8_t *dst = ring + st * C::STAGE;
+          mbar_arrive_expect_tx(&full[st], C::STAGE);
+          bulk_load(dst, k_pages + base, HC * C::SLICE, &full[st]);
+          bulk_load(dst + HC * C::SLICE, v_pages + base, HC * C::SLICE, &full[st]);
         }
         issued = i + 1;
       }
       // Let every copy land before the CTA (and its shared memory) goes away.
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        mbar_wait_drain(&full[i % kStages], (i / kStages) & 1, status);
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
+        mbar_wait_drain(&full[i % C::NST], (i / C::NST) & 1, status);
     }
   } else {
     // ------------------------------------------------------------ compute
@@ -175,14 +180,14 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[hh][e] = make_float2(0.f, 0.f);
 
-    for (int i = warp; i < npg; i += kWarps) {
-      const int st = i % kStages;
-      bool ok = mbar_wait(&full[st], (i / kStages) & 1, &sm_abort, status);
+    for (int i = 0; i < npg; ++i) {
+      const int st = i % C::NST;
+      bool ok = mbar_wait(&full[st], (i / C::NST) & 1, &sm_abort, status);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int ntok = stage_ntok[st];
       if (ntok > 0) {
-        const uint8_t *ks = ring + st * stage_bytes<D>();
-        const uint8_t *vs = ks + SLICE * 2;
+        const uint8_t *ks = ring + st * C::STAGE + warp * C::SLICE;
+        const uint8_t *vs = ring + st * C::STAGE + (HC + warp) * C::SLICE;
         // q . k for this lane's rows: partial dot over 8 columns per head, then a
         // butterfly over the LPT lanes of the row that also transposes, so each
         // lane ends with one head's full score (log2 units).
@@ -242,7 +247,8 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
           const float pw = ex2f(sc[it] - m);  // 0 for rows past the sequence end
           l += pw;
           float vf[8];
-          // Rows past ntok were not copied this time: read zeros, never stale data.
+          // Rows past the sequence end hold whatever the cache slots hold:
+          // read zeros instead (a NaN there would survive a zero weight).
           const uint4 vraw = row < ntok ? *reinterpret_cast<const uint4 *>(vs + (row * D + dc * 8) * 2)
                                         : make_uint4(0, 0, 0, 0);
           bf16x8_to_f32(vraw, vf);
@@ -272,41 +278,30 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, GB >= 8 ? 2 : 3)
           acc[hh][e].y += __shfl_xor_sync(0xffffffffu, acc[hh][e].y, o);
         }
     }
-    if (lane < LPT) {
+    // The warp's partial is the chunk's for its heads: normalise and write.
+    // sm_bad / sm_abort are final once every page has been consumed.
+    const bool bad = *reinterpret_cast<volatile int *>(&sm_bad) != 0 ||
+                     *reinterpret_cast<volatile int *>(&sm_abort) != 0;
 #pragma unroll
-      for (int hh = 0; hh < GB; ++hh)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          sm_acc[warp][hh][dc * 8 + 2 * e] = acc[hh][e].x;
-          sm_acc[warp][hh][dc * 8 + 2 * e + 1] = acc[hh][e].y;
-        }
-      if (lane % (LPT / GB) == 0) {
-        sm_m[warp][my_head] = m;
-        sm_l[warp][my_head] = l;
+    for (int hh = 0; hh < GB; ++hh) {
+      const float mh = __shfl_sync(0xffffffffu, m, hh * (LPT / GB));
+      const float lh = __shfl_sync(0xffffffffu, l, hh * (LPT / GB));
+      const size_t slot = (static_cast<size_t>(s) * Hq + h0 + hh) * nsplit + split;
+      if (lane < LPT) {
+        const float inv = 1.f / lh;
+        float4 *dst = reinterpret_cast<float4 *>(o_part + slot * D + dc * 8);
+        dst[0] = bad ? make_float4(NAN, NAN, NAN, NAN)
+                     : make_float4(acc[hh][0].x * inv, acc[hh][0].y * inv, acc[hh][1].x * inv,
+                                   acc[hh][1].y * inv);
+        dst[1] = bad ? make_float4(NAN, NAN, NAN, NAN)
+                     : make_float4(acc[hh][2].x * inv, acc[hh][2].y * inv, acc[hh][3].x * inv,
+                                   acc[hh][3].y * inv);
       }
+      if (lane == 0) l2_part[slot] = bad ? NAN : mh + log2f(lh);
     }
   }
   __syncthreads();
-
-  // Merge the warps and write this chunk's normalised partial per head.
-  const bool bad = sm_bad != 0 || sm_abort != 0;
-  if (bad && threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
-  for (int idx = threadIdx.x; idx < GB * D; idx += blockDim.x) {
-    const int hh = idx / D, c = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][hh]);
-    float wsum = 0.f, num = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float wt = (sm_m[w][hh] == -INFINITY) ? 0.f : ex2f(sm_m[w][hh] - M);
-      wsum += wt * sm_l[w][hh];
-      num += wt * sm_acc[w][hh][c];
-    }
-    const size_t slot = (static_cast<size_t>(s) * Hq + h0 + hh) * nsplit + split;
-    o_part[slot * D + c] = bad ? NAN : num / wsum;
-    if (c == 0) l2_part[slot] = bad ? NAN : M + log2f(wsum);
-  }
+  if (threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
 }
 
 // One warp per (sequence, head): merge the chunk partials.
@@ -364,32 +359,45 @@ __global__ void __launch_bounds__(128)
   if (lane == 0) lse[head] = (M + log2f(wsum)) * 0.6931471805599453f;
 }
 
-template <int D, int GB>
+template <int D, int GB, int HC>
 void launch_split(dim3 grid, cudaStream_t st, const void *q, const void *kp, const void *vp,
                   const int *bt, const int *sl, float *op, float *lp, int Hq, int Hkv, int maxb,
                   int npages, float sl2, int nsplit, int hc, unsigned *status) {
-  constexpr int kSmem = kStages * stage_bytes<D>();
+  constexpr int kSmem = DecCfg<HC, D>::SMEM;
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(decode_split_kernel<D, GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(decode_split_kernel<D, GB, HC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kSmem);
   });
-  decode_split_kernel<D, GB><<<grid, (kWarps + 1) * 32, kSmem, st>>>(
+  decode_split_kernel<D, GB, HC><<<grid, (HC + 1) * 32, kSmem, st>>>(
       static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kp),
       static_cast<const __nv_bfloat16 *>(vp), bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit,
       hc, status);
 }
 
+template <int D, int HC>
+bool dispatch_gb(int GB, dim3 grid, cudaStream_t st, const void *q, const void *kp,
+                 const void *vp, const int *bt, const int *sl, float *op, float *lp, int Hq,
+                 int Hkv, int maxb, int npages, float sl2, int nsplit, int hc, unsigned *status) {
+  switch (GB) {
+    case 8: launch_split<D, 8, HC>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
+    case 4: launch_split<D, 4, HC>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
+    case 2: launch_split<D, 2, HC>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
+    case 1: launch_split<D, 1, HC>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
+  }
+  return false;
+}
+
 template <int D>
-bool dispatch_split(int GB, dim3 grid, cudaStream_t st, const void *q, const void *kp,
+bool dispatch_split(int HC, int GB, dim3 grid, cudaStream_t st, const void *q, const void *kp,
                     const void *vp, const int *bt, const int *sl, float *op, float *lp, int Hq,
                     int Hkv, int maxb, int npages, float sl2, int nsplit, int hc,
                     unsigned *status) {
-  switch (GB) {
-    case 8: launch_split<D, 8>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
-    case 4: launch_split<D, 4>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
-    case 2: launch_split<D, 2>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
-    case 1: launch_split<D, 1>(grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status); return true;
+  switch (HC) {
+    case 8: return dispatch_gb<D, 8>(GB, grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 4: return dispatch_gb<D, 4>(GB, grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 2: return dispatch_gb<D, 2>(GB, grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
+    case 1: return dispatch_gb<D, 1>(GB, grid, st, q, kp, vp, bt, sl, op, lp, Hq, Hkv, maxb, npages, sl2, nsplit, hc, status);
   }
   return false;
 }
@@ -439,22 +447,26 @@ attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void
   const int G = Hq / Hkv;
   const int GB = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
   const int head_chunks = G / GB;
+  const int HC = (Hkv % 8 == 0) ? 8 : (Hkv % 4 == 0) ? 4 : (Hkv % 2 == 0) ? 2 : 1;
   const int nsplit = decode_max_splits(max_blocks);
   const size_t parts = static_cast<size_t>(S) * Hq * nsplit;
   float *o_part = static_cast<float *>(workspace);
   float *l2_part = reinterpret_cast<float *>(
       static_cast<uint8_t *>(workspace) +
       ((parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255)));
-  if (static_cast<long long>(Hkv) * head_chunks > 65535 || S > 65535) return ATTN_ERR_UNSUPPORTED;
-  dim3 grid(nsplit, Hkv * head_chunks, S);
+  if (static_cast<long long>(Hkv / HC) * head_chunks > 65535 || S > 65535)
+    return ATTN_ERR_UNSUPPORTED;
+  dim3 grid(nsplit, S, (Hkv / HC) * head_chunks);
   const float sl2 = scale * 1.4426950408889634f;
   bool ok;
   if (d == 128)
-    ok = dispatch_split<128>(GB, grid, stream, q, k_pages, v_pages, block_table, seq_lens, o_part,
-                             l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+    ok = dispatch_split<128>(HC, GB, grid, stream, q, k_pages, v_pages, block_table, seq_lens,
+                             o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit,
+                             head_chunks, status);
   else if (d == 64)
-    ok = dispatch_split<64>(GB, grid, stream, q, k_pages, v_pages, block_table, seq_lens, o_part,
-                            l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit, head_chunks, status);
+    ok = dispatch_split<64>(HC, GB, grid, stream, q, k_pages, v_pages, block_table, seq_lens,
+                            o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit,
+                            head_chunks, status);
   else
     return ATTN_ERR_UNSUPPORTED;
   if (!ok) return ATTN_ERR_UNSUPPORTED;
