@@ -267,7 +267,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ================================================================ producer
     regs_dec<kRegsLow>();
-    if (lane == 0) {
+    if constexpr (kPaged) {
+      // The whole warp gathers: lane 0 runs the barrier protocol and the Q
+      // copies, lanes 0-7 each bring one page of every K/V tile, so the eight
+      // block-table reads and sixteen or more box copies per tile proceed in
+      // parallel.
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_k1);
+        tma_prefetch_desc(&tm_v1);
+        mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
+                        hq, qrow0 + row0 + t * BM);
+      }
+      int issued = 0;
+      for (int i = 0; i < 2 * (jhi - jlo); ++i) {
+        const int slot = i % C::NST;
+        const int round = i / C::NST;
+        bool go = true;
+        if (lane == 0 && round > 0)
+          go = mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status);
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
+        __syncwarp();
+        if (lane < BN / 16) {
+          // Page `lane` of the tile: a whole page as one 16-row box per 64
+          // columns; the last, partly filled page row by row; rows past the
+          // keys from an out-of-range coordinate, i.e. zeros (never stale
+          // shared memory, which a zero P could not cancel if it held a NaN).
+          const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
+          const CUtensorMap *map1 = (i & 1) ? &tm_v1 : &tm_k1;
+          const int key0 = (jlo + (i >> 1)) * BN + lane * 16;
+          const int ntok = min(16, nk - key0);
+          const int z = ntok > 0
+              ? p.block_table[static_cast<size_t>(b) * p.max_blocks + key0 / 16] * p.Hkv + hkv
+              : -1;
+          uint8_t *dst = sRing + slot * C::TILE_BYTES + lane * 16 * 128;
+          for (int c = 0; c < C::CH; ++c) {
+            if (ntok >= 16 || ntok <= 0) {
+              tma_load_3d(dst + c * CHUNK_BYTES, map, &bars->full[slot], 64 * c, 0, z);
+            } else {
+              for (int r = 0; r < 16; ++r)
+                tma_load_3d(dst + c * CHUNK_BYTES + r * 128, map1, &bars->full[slot], 64 * c, r,
+                            r < ntok ? z : -1);
+            }
+          }
+        }
+        issued = i + 1;
+      }
+      // Drain: no copy may still be writing shared memory when the CTA exits.
+      if (lane == 0) {
+        mbar_wait_drain(&bars->q_full, 0, p.status);
+        for (int i = max(0, issued - C::NST); i < issued; ++i)
+          mbar_wait_drain(&bars->full[i % C::NST], (i / C::NST) & 1, p.status);
+      }
+    } else if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -275,14 +333,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int zkv = b * p.Hkv + hkv;
       mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
       for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < C::CH; ++c) {
-          if constexpr (kPaged)  // token-major queries: (D, Hq, T) boxes of 64 x 1 x 128
-            tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
-                        hq, qrow0 + row0 + t * BM);
-          else
-            tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
-                        row0 + t * BM, zq);
-        }
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
+                      row0 + t * BM, zq);
       int issued = 0;
       for (int i = 0; i < 2 * (jhi - jlo); ++i) {
         const int slot = i % C::NST;
@@ -291,35 +344,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
         const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
-        if constexpr (kPaged) {
-          // Gather the tile's 8 pages: whole pages as 16-row boxes; the last,
-          // partly filled page row by row; rows past the keys from an
-          // out-of-range coordinate, i.e. zeros (never stale shared memory,
-          // which a zero P could not cancel if it held a NaN).
-          const CUtensorMap *map1 = (i & 1) ? &tm_v1 : &tm_k1;
-          const int key_base = (jlo + (i >> 1)) * BN;
-          for (int pp = 0; pp < BN / 16; ++pp) {
-            const int key0 = key_base + pp * 16;
-            const int ntok = min(16, nk - key0);
-            const int z = ntok > 0
-                ? p.block_table[static_cast<size_t>(b) * p.max_blocks + key0 / 16] * p.Hkv + hkv
-                : -1;
-            uint8_t *dst = sRing + slot * C::TILE_BYTES + pp * 16 * 128;
-            for (int c = 0; c < C::CH; ++c) {
-              if (ntok >= 16 || ntok <= 0) {
-                tma_load_3d(dst + c * CHUNK_BYTES, map, &bars->full[slot], 64 * c, 0, z);
-              } else {
-                for (int r = 0; r < 16; ++r)
-                  tma_load_3d(dst + c * CHUNK_BYTES + r * 128, map1, &bars->full[slot], 64 * c, r,
-                              r < ntok ? z : -1);
-              }
-            }
-          }
-        } else {
-          for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
-                        64 * c, (jlo + (i >> 1)) * BN, zkv);
-        }
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
+                      64 * c, (jlo + (i >> 1)) * BN, zkv);
         issued = i + 1;
       }
       // Drain: no copy may still be writing shared memory when the CTA exits.
