@@ -24,7 +24,7 @@ __all__ = [
     "attn_prefill_paged",
     "bwd_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
     "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
-    "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "AttnError",
+    "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "ATTN_DEV_LAYOUT", "AttnError",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libexattn.so")
@@ -38,6 +38,7 @@ EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ext", "attn_fwd_f32_ex
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 ATTN_DEV_BAD_PAGE = 0x1
 ATTN_DEV_TIMEOUT = 0x2
+ATTN_DEV_LAYOUT = 0x4
 # kv_format codes of attn_decode_paged_q8 and the torch dtypes accepted for each.
 KV_FORMATS = {"e4m3": 0, "int8": 1}
 _KV_DTYPES = {"e4m3": (torch.float8_e4m3fn, torch.uint8), "int8": (torch.int8,)}

@@ -14,31 +14,33 @@
 //    workspace padded to whole 128-row tiles (+inf / 0 past N, so padded rows
 //    get P = 0 without a mask).
 //  * bwd_dkdv: one CTA per 128-key tile of one (batch, K/V head).  K and V stay
-//    in shared memory; 128-row tiles of Q and dO (and their L, D) stream
-//    through a ring, for every query head of the group.  Per tile:
+//    in shared memory; 128-row tiles of Q and of dO (with their L, D) stream
+//    through two rings, for every query head of the group.  Per tile:
 //      S^T = K Q^T, dP^T = V dO^T        (128x128x16 MMAs, both K-major)
 //      P^T = 2^(S^T c - L2), dS^T = P^T (dP^T - D)   (CUDA cores, TMEM ld/st)
 //      dV += P^T dO, dK += dS^T Q          (A = P^T / dS^T from TMEM, B MN-major)
 //  * bwd_dq: one CTA per 128-row Q tile of one (batch, query head); 128-key
-//    tiles of K and V stream through a ring.  S = Q K^T, dP = dO V^T,
+//    tiles of K and of V stream through two rings.  S = Q K^T, dP = dO V^T,
 //    dS as above, dQ += dS K (A = dS from TMEM, B = K MN-major).
 // The recomputation costs two more tile products than a single kernel that
 // scatters dQ with atomic adds (7 instead of 5); the FLOP rate reported counts
 // the 5 of the algorithm.
 //
-// Scheduling.  All MMAs are 128 wide.  TMEM holds S (or S^T) and dP (or dP^T),
-// 128 columns each, and the 128-column accumulators (dV and dK, or dQ): 512
-// columns, so the score tiles are single-buffered.  The overlap comes from
-// splitting every tile's columns between the two elementwise warpgroups: a
-// warpgroup computes P from S while the tensor pipe still computes dP, and
-// hands over its half of P / dS as soon as it is written, so the gradient MMAs
-// of one half run while the other half is still being computed.  The next
-// tile's S is issued right after the gradient MMAs that read the current one
-// (tcgen05 ops from one thread execute in order).
+// Scheduling.  All MMAs are 128 wide.  Each tile uses one 128-column TMEM
+// buffer twice: the score tile S (S^T) is written there, the elementwise warps
+// load it into registers and say so, and the tensor pipe then writes dP (dP^T)
+// over it; the warps finally store their bf16 results (P^T and dS^T, or dS)
+// into the same columns.  Two such buffers next to the 128-column
+// accumulators (dV and dK, or dQ) keep two tiles in flight, and the two
+// elementwise warpgroups take alternate tiles.  Per tile the MMA issuer runs
+// dP(i), then the gradient products of tile i-1 and the scores of tile i+1,
+// so the exponentials of one tile overlap the other tile's products.  The
+// streamed tile whose product comes last (Q for dK, K for dQ) is live for
+// three iterations and gets a three-slot ring; the other (dO, V) two slots.
 //
 // Warp roles (both GEMM kernels, 384 threads, as in the forward): warp 0 TMA
-// producer, warp 1 TMEM owner and MMA issuer, warps 4-7 and 8-11 two
-// elementwise warpgroups, each owning 64 of a tile's 128 columns.
+// producer (lane 0 for one ring, lane 1 for the other), warp 1 TMEM owner and
+// MMA issuer, warps 4-7 and 8-11 the two elementwise warpgroups.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -61,47 +63,53 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= NUM_THREADS * 168 && kRegsLow 
               "setmaxnreg split must fit the block's launch registers");
 constexpr int kHeadGroup = 8;
 constexpr int CHUNK = BT * 128;  // 128 rows x 128 bytes: one 64-column block of a tile
+constexpr int NA = 3;            // slots of the three-iteration ring (Q or K)
+constexpr int NB = 2;            // slots of the two-iteration ring (dO + vectors, or V)
 
-// TMEM columns: S / S^T, dP / dP^T, and the accumulators.  Warpgroup w writes
-// its 64 bf16 results (P^T and dS^T, or dS) over columns [64w, 64w+32) of the
-// tile it read them from.
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColDP = 128;
+// TMEM: two 128-column tile buffers, then the accumulators.  In a buffer the
+// bf16 results sit at columns [0, 64) (P^T, or dS) and [64, 128) (dS^T): the
+// 128 values of a row, two per column.
+__device__ __forceinline__ uint32_t col_x(int buf) { return static_cast<uint32_t>(buf) * 128; }
 constexpr uint32_t kColAcc0 = 256;  // dV (dK/dV kernel) or dQ (dQ kernel)
 constexpr uint32_t kColAcc1 = 384;  // dK (dK/dV kernel)
-__device__ __forceinline__ uint32_t packed_col(int ks) {  // k-step of 16 -> its 8 bf16 columns
-  return 64 * (ks >> 2) + (ks & 3) * 8;
-}
 
 template <int D>
 struct BCfg {
   static constexpr int CH = D / 64;
   static constexpr int TILE = BT * D * 2;
-  // dK/dV kernel: K, V resident; stages of {Q, dO, L2[128], D[128]}.
-  static constexpr int KV_NST = (D == 64) ? 4 : 2;
-  static constexpr int KV_STAGE = ((2 * TILE + 2 * BT * 4) + 1023) / 1024 * 1024;
-  static constexpr int KV_RING_OFF = 2 * TILE;
-  static constexpr int KV_BAR_OFF = KV_RING_OFF + KV_NST * KV_STAGE;
-  // dQ kernel: Q, dO resident; slots of one K or V tile.
-  static constexpr int Q_NST = (D == 64) ? 8 : 4;
-  static constexpr int Q_RING_OFF = 2 * TILE;
-  static constexpr int Q_BAR_OFF = Q_RING_OFF + Q_NST * TILE;
-  // At least 116 KiB so that one CTA fills an SM: each CTA allocates all 512
-  // TMEM columns.
+  static constexpr int VEC = 2 * BT * 4;  // L2 and D of a 128-row Q tile
+  static constexpr int BSLOT_KV = TILE + VEC;  // dO tile + vectors (a multiple of 1024)
+  // dK/dV kernel: K, V resident; Q ring (NA); dO + vector ring (NB).  At d =
+  // 128 this is 226 KiB, so the kernel relies on the dynamic shared memory
+  // starting 1024-aligned (it checks) instead of reserving slack.
+  static constexpr int KV_A_OFF = 2 * TILE;
+  static constexpr int KV_B_OFF = KV_A_OFF + NA * TILE;
+  static constexpr int KV_BAR_OFF = KV_B_OFF + NB * BSLOT_KV;
+  static constexpr int KV_SMEM = KV_BAR_OFF + 512;
+  // dQ kernel: Q, dO resident; K ring (NA); V ring (NB).
+  static constexpr int Q_A_OFF = 2 * TILE;
+  static constexpr int Q_B_OFF = Q_A_OFF + NA * TILE;
+  static constexpr int Q_BAR_OFF = Q_B_OFF + NB * TILE;
+  static constexpr int Q_SMEM = Q_BAR_OFF + 512;
+  // Each CTA allocates all 512 TMEM columns, so one CTA per SM: at d = 64
+  // the launch asks for at least this much shared memory to make sure of it.
   static constexpr int MIN_SMEM = 116 * 1024;
-  static constexpr int KV_SMEM = (KV_BAR_OFF + 2048 > MIN_SMEM) ? KV_BAR_OFF + 2048 : MIN_SMEM;
-  static constexpr int Q_SMEM = (Q_BAR_OFF + 2048 > MIN_SMEM) ? Q_BAR_OFF + 2048 : MIN_SMEM;
+  static constexpr int KV_LAUNCH = KV_SMEM > MIN_SMEM ? KV_SMEM : MIN_SMEM;
+  static constexpr int Q_LAUNCH = Q_SMEM > MIN_SMEM ? Q_SMEM : MIN_SMEM;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BT, false, false);
   static constexpr uint32_t IDESC_G = idesc_bf16_f32(BT, D, false, true);
 };
+static_assert(BCfg<128>::KV_SMEM <= 232448 && BCfg<128>::Q_SMEM <= 232448,
+              "shared memory of one CTA");
 
 struct BBars {
-  uint64_t full[8];
-  uint64_t empty[8];
-  uint64_t res_full;  // the resident tiles (K,V or Q,dO)
-  uint64_t s_full;    // S (or S^T) of the current tile is in TMEM
-  uint64_t dp_full;   // dP (or dP^T) likewise
-  uint64_t p_full[2]; // warpgroup w's half of P / dS is in TMEM
+  uint64_t a_full[NA], a_empty[NA];  // Q (dK/dV kernel) or K (dQ kernel) ring
+  uint64_t b_full[NB], b_empty[NB];  // dO + vectors, or V ring
+  uint64_t res_full;                 // the resident tiles
+  uint64_t s_full[2];    // buffer w holds S (S^T) of its tile
+  uint64_t s_read[2];    // warpgroup w has loaded it into registers (count 128)
+  uint64_t dp_full[2];   // buffer w holds dP (dP^T)
+  uint64_t p_full[2];    // warpgroup w's bf16 results are in buffer w (count 128)
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -162,15 +170,14 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// P = 2^(s*c + bias - l2) for 32 columns (0 where vis(i) is false); bias =
-// bias0 + bias_step * i (ALiBi); l2 per column (per_col) or one value.  On
-// unmasked columns one pair in four takes 2^x from the FMA-pipe cubic
-// (relative error < 2^-13, below the bf16 rounding that follows), which
-// shortens the special-function unit's share of the tile.
+// P = 2^(s*c + bias - l2) for 32 columns (0 where vis(i) is false), packed to
+// bf16 pairs; bias = bias0 + bias_step * i (ALiBi); l2 per column (per_col) or
+// one value.  On unmasked columns one pair in four takes 2^x from the FMA-pipe
+// cubic (relative error < 2^-13, below the bf16 rounding that follows).
 template <bool kAlibi, bool kMasked, typename Vis>
-__device__ __forceinline__ void p_cols(const uint32_t (&sv)[32], const float *l2c, float l2s,
+__device__ __forceinline__ void p_cols(const uint32_t *sv, const float *l2c, float l2s,
                                        bool per_col, float c, float bias0, float bias_step,
-                                       Vis vis, float (&pv)[32]) {
+                                       Vis vis, uint32_t *pk) {
   const float2 c2 = make_float2(c, c);
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
@@ -181,36 +188,31 @@ __device__ __forceinline__ void p_cols(const uint32_t (&sv)[32], const float *l2
       x = fma2(make_float2(bias_step, bias_step),
                make_float2(static_cast<float>(i), static_cast<float>(i + 1)),
                make_float2(x.x + bias0, x.y + bias0));
-    if (!kMasked && (i & 6) == 6) {  // one pair in four on the FMA pipe
-      const float2 e = exp2_poly2(x);
-      pv[i] = e.x;
-      pv[i + 1] = e.y;
+    float2 e;
+    if (!kMasked && (i & 6) == 6) {
+      e = exp2_poly2(x);
     } else {
-      pv[i] = ex2(x.x);
-      pv[i + 1] = ex2(x.y);
+      e = make_float2(ex2(x.x), ex2(x.y));
+      if (kMasked) {
+        if (!vis(i)) e.x = 0.f;
+        if (!vis(i + 1)) e.y = 0.f;
+      }
     }
-    if (kMasked) {
-      if (!vis(i)) pv[i] = 0.f;
-      if (!vis(i + 1)) pv[i + 1] = 0.f;
-    }
+    pk[i >> 1] = pack_bf16x2(e.x, e.y);
   }
 }
 
-__device__ __forceinline__ void pack_cols(const float (&pv)[32], uint32_t (&pk)[16]) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16x2(pv[i], pv[i + 1]);
-}
-
-// dS = P * (dp - D) for 32 columns, packed bf16; D per column or one value.
-__device__ __forceinline__ void ds_cols(const float (&pv)[32], const uint32_t (&dpv)[32],
-                                        const float *ddc, float dds, bool per_col,
-                                        uint32_t (&dk)[16]) {
+// dS = P * (dp - D) for 32 columns from bf16-packed P; packed bf16 out.
+__device__ __forceinline__ void ds_cols(const uint32_t *pk, const uint32_t *dpv, const float *ddc,
+                                        float dds, bool per_col, uint32_t *dk) {
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const float2 dv = per_col ? *reinterpret_cast<const float2 *>(ddc + i) : make_float2(dds, dds);
+    const uint32_t w = pk[i >> 1];
+    const float2 pv = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
     const float2 t = add2(make_float2(__uint_as_float(dpv[i]), __uint_as_float(dpv[i + 1])),
                           make_float2(-dv.x, -dv.y));
-    dk[i >> 1] = pack_bf16x2(pv[i] * t.x, pv[i + 1] * t.y);
+    dk[i >> 1] = pack_bf16x2(pv.x * t.x, pv.y * t.y);
   }
 }
 
@@ -221,12 +223,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using C = BCfg<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the layout needs a 1024-aligned base (see BCfg)
+    if (threadIdx.x == 0) atomicOr(p.status, ATTN_DEV_LAYOUT);
+    return;
+  }
   uint8_t *sK = smem;
   uint8_t *sV = smem + C::TILE;
-  uint8_t *sRing = smem + C::KV_RING_OFF;
+  uint8_t *sA = smem + C::KV_A_OFF;  // Q ring
+  uint8_t *sB = smem + C::KV_B_OFF;  // dO + vector ring
   BBars *bars = reinterpret_cast<BBars *>(smem + C::KV_BAR_OFF);
   volatile int *abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -261,15 +266,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_items = G * nq;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::KV_NST; ++i) {
-      mbar_init(&bars->full[i], 1);
-      mbar_init(&bars->empty[i], 1);
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&bars->a_full[i], 1);
+      mbar_init(&bars->a_empty[i], 1);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&bars->b_full[i], 1);
+      mbar_init(&bars->b_empty[i], 1);
     }
     mbar_init(&bars->res_full, 1);
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_full[0], 128);
-    mbar_init(&bars->p_full[1], 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->s_read[t], 128);
+      mbar_init(&bars->dp_full[t], 1);
+      mbar_init(&bars->p_full[t], 128);
+    }
     mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -287,10 +298,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ================================================================ producer
     regs_dec<kRegsLow>();
     if (lane == 0) {
+      // K, V once; then the Q ring.
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(&bars->res_full, 2 * C::TILE);
       for (int c = 0; c < C::CH; ++c) {
         tma_load_3d(sK + c * CHUNK, &tm_k, &bars->res_full, 64 * c, k0, bhk);
@@ -298,93 +309,119 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       int issued = 0;
       for (int it = 0; it < n_items; ++it) {
-        const int slot = it % C::KV_NST, round = it / C::KV_NST;
-        if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status)) break;
-        const int hq = g * G + it / nq;
+        const int slot = it % NA, round = it / NA;
+        if (round > 0 && !mbar_wait(&bars->a_empty[slot], (round - 1) & 1, abort_flag, p.status))
+          break;
+        const int zq = b * p.Hq + g * G + it / nq;
         const int q0 = (qs + it % nq) * BT;
-        const int zq = b * p.Hq + hq;
-        uint8_t *st = sRing + slot * C::KV_STAGE;
-        mbar_arrive_expect_tx(&bars->full[slot], 2 * C::TILE + 2 * BT * 4);
-        for (int c = 0; c < C::CH; ++c) {
-          tma_load_3d(st + c * CHUNK, &tm_q, &bars->full[slot], 64 * c, q0, zq);
-          tma_load_3d(st + C::TILE + c * CHUNK, &tm_do, &bars->full[slot], 64 * c, q0, zq);
-        }
-        const size_t vo = static_cast<size_t>(zq) * p.Npad + q0;
-        bulk_load(st + 2 * C::TILE, p.l2 + vo, BT * 4, &bars->full[slot]);
-        bulk_load(st + 2 * C::TILE + BT * 4, p.dvec + vo, BT * 4, &bars->full[slot]);
+        mbar_arrive_expect_tx(&bars->a_full[slot], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sA + slot * C::TILE + c * CHUNK, &tm_q, &bars->a_full[slot], 64 * c, q0, zq);
         issued = it + 1;
       }
       mbar_wait_drain(&bars->res_full, 0, p.status);
-      for (int i = max(0, issued - C::KV_NST); i < issued; ++i)
-        mbar_wait_drain(&bars->full[i % C::KV_NST], (i / C::KV_NST) & 1, p.status);
+      for (int i = max(0, issued - NA); i < issued; ++i)
+        mbar_wait_drain(&bars->a_full[i % NA], (i / NA) & 1, p.status);
+    } else if (lane == 1) {
+      // The dO ring, with each tile's L2 and D vectors.
+      tma_prefetch_desc(&tm_do);
+      int issued = 0;
+      for (int it = 0; it < n_items; ++it) {
+        const int slot = it % NB, round = it / NB;
+        if (round > 0 && !mbar_wait(&bars->b_empty[slot], (round - 1) & 1, abort_flag, p.status))
+          break;
+        const int zq = b * p.Hq + g * G + it / nq;
+        const int q0 = (qs + it % nq) * BT;
+        uint8_t *st = sB + slot * C::BSLOT_KV;
+        mbar_arrive_expect_tx(&bars->b_full[slot], C::BSLOT_KV);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(st + c * CHUNK, &tm_do, &bars->b_full[slot], 64 * c, q0, zq);
+        const size_t vo = static_cast<size_t>(zq) * p.Npad + q0;
+        bulk_load(st + C::TILE, p.l2 + vo, BT * 4, &bars->b_full[slot]);
+        bulk_load(st + C::TILE + BT * 4, p.dvec + vo, BT * 4, &bars->b_full[slot]);
+        issued = it + 1;
+      }
+      for (int i = max(0, issued - NB); i < issued; ++i)
+        mbar_wait_drain(&bars->b_full[i % NB], (i / NB) & 1, p.status);
     }
   } else if (warp == 1) {
     // ================================================================== MMA
     regs_dec<kRegsLow>();
     if (lane == 0) {
-      const uint32_t ring = smem_u32(sRing);
       const uint64_t kdesc = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t vdesc = kdesc + (C::TILE >> 4);
-      const uint64_t qk0 = sdesc_sw128(ring, 16, 1024);               // Q, K-major
-      const uint64_t dok0 = qk0 + (C::TILE >> 4);                     // dO, K-major
-      const uint64_t qmn0 = sdesc_sw128(ring, CHUNK, 1024);           // Q, MN-major
-      const uint64_t domn0 = qmn0 + (C::TILE >> 4);                   // dO, MN-major
-      auto wait_full = [&](int it) {
-        return mbar_wait(&bars->full[it % C::KV_NST], (it / C::KV_NST) & 1, abort_flag, p.status);
+      const uint64_t qk0 = sdesc_sw128(smem_u32(sA), 16, 1024);        // Q, K-major
+      const uint64_t qmn0 = sdesc_sw128(smem_u32(sA), CHUNK, 1024);    // Q, MN-major
+      const uint64_t dok0 = sdesc_sw128(smem_u32(sB), 16, 1024);       // dO, K-major
+      const uint64_t domn0 = sdesc_sw128(smem_u32(sB), CHUNK, 1024);   // dO, MN-major
+      auto a_off = [](int it) { return static_cast<uint64_t>((it % NA) * C::TILE) >> 4; };
+      auto b_off = [](int it) { return static_cast<uint64_t>((it % NB) * C::BSLOT_KV) >> 4; };
+      auto wait_a = [&](int it) {
+        return mbar_wait(&bars->a_full[it % NA], (it / NA) & 1, abort_flag, p.status);
       };
-      auto stage_off = [](int it) {
-        return static_cast<uint64_t>((it % C::KV_NST) * C::KV_STAGE) >> 4;
+      auto wait_b = [&](int it) {
+        return mbar_wait(&bars->b_full[it % NB], (it / NB) & 1, abort_flag, p.status);
       };
-      auto issue_scores = [&](int it) {  // S^T = K Q^T, commit; dP^T = V dO^T, commit
-        const uint64_t so = stage_off(it);
+      auto issue_s = [&](int it) {  // S^T = K Q^T into buffer it & 1
+        const uint32_t d = tmem + col_x(it & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t off = ((ks >> 2) * CHUNK + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + kColS, kdesc + off, qk0 + so + off, C::IDESC_S, ks > 0);
+          mma_ss(d, kdesc + off, qk0 + a_off(it) + off, C::IDESC_S, ks > 0);
         }
-        tc_commit(&bars->s_full);
+        tc_commit(&bars->s_full[it & 1]);
+      };
+      auto issue_dp = [&](int it) {  // dP^T = V dO^T over S^T (already read)
+        const uint32_t d = tmem + col_x(it & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t off = ((ks >> 2) * CHUNK + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + kColDP, vdesc + off, dok0 + so + off, C::IDESC_S, ks > 0);
+          mma_ss(d, vdesc + off, dok0 + b_off(it) + off, C::IDESC_S, ks > 0);
         }
-        tc_commit(&bars->dp_full);
+        tc_commit(&bars->dp_full[it & 1]);
       };
-      auto issue_grad_half = [&](int it, int h) {  // queries [64h, 64h+64)
-        const uint64_t so = stage_off(it);
+      auto issue_grads = [&](int it) {  // dV += P^T dO, dK += dS^T Q
+        const uint32_t x = tmem + col_x(it & 1);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int ks = 4 * h + kk;
-          mma_ts(tmem + kColAcc0, tmem + kColS + packed_col(ks), domn0 + so + ((ks * 2048) >> 4),
-                 C::IDESC_G, (it > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < BT / 16; ++ks)
+          mma_ts(tmem + kColAcc0, x + ks * 8, domn0 + b_off(it) + ((ks * 2048) >> 4), C::IDESC_G,
+                 (it > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(&bars->b_empty[it % NB]);  // dO(it) consumed: the next dO lands sooner
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int ks = 4 * h + kk;
-          mma_ts(tmem + kColAcc1, tmem + kColDP + packed_col(ks), qmn0 + so + ((ks * 2048) >> 4),
+        for (int ks = 0; ks < BT / 16; ++ks)
+          mma_ts(tmem + kColAcc1, x + 64 + ks * 8, qmn0 + a_off(it) + ((ks * 2048) >> 4),
                  C::IDESC_G, (it > 0 || ks > 0) ? 1u : 0u);
-        }
+        tc_commit(&bars->a_empty[it % NA]);
       };
       bool ok = mbar_wait(&bars->res_full, 0, abort_flag, p.status);
-      if (ok && n_items > 0 && (ok = wait_full(0))) {
+      for (int it = 0; ok && it < 2 && it < n_items; ++it) {
+        if (!(ok = wait_a(it))) break;
         tc_fence_after();
-        issue_scores(0);
+        issue_s(it);
       }
       for (int it = 0; ok && it < n_items; ++it) {
-        for (int h = 0; h < 2; ++h) {
-          if (!(ok = mbar_wait(&bars->p_full[h], it & 1, abort_flag, p.status))) break;
+        const int bb = it & 1;
+        if (!(ok = mbar_wait(&bars->s_read[bb], (it >> 1) & 1, abort_flag, p.status) && wait_b(it)))
+          break;
+        tc_fence_after();
+        issue_dp(it);
+        if (it >= 1) {
+          if (!(ok = mbar_wait(&bars->p_full[bb ^ 1], ((it - 1) >> 1) & 1, abort_flag, p.status)))
+            break;
           tc_fence_after();
-          issue_grad_half(it, h);
+          issue_grads(it - 1);
+          if (it + 1 < n_items) {
+            if (!(ok = wait_a(it + 1))) break;
+            tc_fence_after();
+            issue_s(it + 1);  // in order after grads(it-1), which read this buffer
+          }
         }
-        if (!ok) break;
-        tc_commit(&bars->empty[it % C::KV_NST]);  // Q/dO stage consumed
-        if (it + 1 < n_items) {
-          if (!(ok = wait_full(it + 1))) break;
-          tc_fence_after();
-          // In order after the gradient MMAs above, which read P^T / dS^T from
-          // these columns: no completion wait needed.
-          issue_scores(it + 1);
-        }
+      }
+      if (ok && n_items > 0 &&
+          (ok = mbar_wait(&bars->p_full[(n_items - 1) & 1], ((n_items - 1) >> 1) & 1, abort_flag,
+                          p.status))) {
+        tc_fence_after();
+        issue_grads(n_items - 1);
       }
       tc_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, p.status);
@@ -394,74 +431,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ============================================================ elementwise
     regs_inc<kRegsHigh>();
-    const int wg = (warp - 4) >> 2;      // this warpgroup's 64 columns: [64wg, 64wg+64)
+    const int wg = (warp - 4) >> 2;      // this warpgroup takes tiles wg, wg + 2, ...
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;   // key row in the tile
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + 64 * wg;
-    const uint32_t tDP = tmem + lane_off + kColDP + 64 * wg;
+    const uint32_t tX = tmem + lane_off + col_x(wg);
     const float c = p.scale_log2;
     bool ok = true;
-    for (int it = 0; it < n_items; ++it) {
-      ok = mbar_wait(&bars->s_full, it & 1, abort_flag, p.status) &&
-           mbar_wait(&bars->full[it % C::KV_NST], (it / C::KV_NST) & 1, abort_flag, p.status);
-      ok = __all_sync(0xffffffffu, ok);
+    for (int it = wg; it < n_items; it += 2) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[wg], (it >> 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t sv[128];
+      tmem_ld128(tX, sv);
+      tmem_ld_wait128(sv);
+      tc_fence_before();
+      mbar_arrive(&bars->s_read[wg]);  // the tensor pipe may now write dP^T here
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&bars->b_full[it % NB], (it / NB) & 1, abort_flag, p.status));
+      if (!ok) break;
       const int hq = g * G + it / nq;
-      const int qb = (qs + it % nq) * BT + 64 * wg;  // first query of this warpgroup's columns
-      const uint8_t *st = sRing + (it % C::KV_NST) * C::KV_STAGE;
-      const float *l2v = reinterpret_cast<const float *>(st + 2 * C::TILE) + 64 * wg;
+      const int qb0 = (qs + it % nq) * BT;  // first query of the tile
+      const uint8_t *st = sB + (it % NB) * C::BSLOT_KV;
+      const float *l2v = reinterpret_cast<const float *>(st + C::TILE);
       const float *ddv = l2v + BT;
       const float slope2 = kAlibi ? p.slopes[hq] * 1.4426950408889634f : 0.f;
-      // ---- P^T from S^T (while the tensor pipe computes dP^T)
-      float pv0[32], pv1[32];
-      {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(tS, s0);
-        tmem_ld32(tS + 32, s1);
-        tmem_ld_wait(s0);
-        tmem_ld_wait(s1);
-        auto vis0 = [&](int i) {
+      // ---- P^T (bf16 pairs) for the tile's 128 queries, while dP^T runs.
+      uint32_t pk[64];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int qb = qb0 + 32 * h;
+        auto vis = [&](int i) {
           const int qq = qb + i;
           return (!p.causal || key <= qq) && (p.window <= 0 || qq - key < p.window);
         };
-        auto vis1 = [&](int i) { return vis0(i + 32); };
-        const bool full0 = (!p.causal || key <= qb) && (p.window <= 0 || qb + 31 - key < p.window);
-        const bool full1 =
-            (!p.causal || key <= qb + 32) && (p.window <= 0 || qb + 63 - key < p.window);
+        const bool full = (!p.causal || key <= qb) && (p.window <= 0 || qb + 31 - key < p.window);
         // ALiBi bias slope*(key - query) in log2 units; column i has query qb + i.
         const float bias0 = slope2 * static_cast<float>(key - qb);
-        if (__all_sync(0xffffffffu, full0))
-          p_cols<kAlibi, false>(s0, l2v, 0.f, true, c, bias0, -slope2, vis0, pv0);
+        if (__all_sync(0xffffffffu, full))
+          p_cols<kAlibi, false>(sv + 32 * h, l2v + 32 * h, 0.f, true, c, bias0, -slope2, vis,
+                                pk + 16 * h);
         else
-          p_cols<kAlibi, true>(s0, l2v, 0.f, true, c, bias0, -slope2, vis0, pv0);
-        if (__all_sync(0xffffffffu, full1))
-          p_cols<kAlibi, false>(s1, l2v + 32, 0.f, true, c, bias0 - 32.f * slope2, -slope2, vis1, pv1);
-        else
-          p_cols<kAlibi, true>(s1, l2v + 32, 0.f, true, c, bias0 - 32.f * slope2, -slope2, vis1, pv1);
-        uint32_t pk[16];
-        pack_cols(pv0, pk);
-        tmem_st16(tS, pk);
-        pack_cols(pv1, pk);
-        tmem_st16(tS + 16, pk);
+          p_cols<kAlibi, true>(sv + 32 * h, l2v + 32 * h, 0.f, true, c, bias0, -slope2, vis,
+                               pk + 16 * h);
       }
-      // ---- dS^T from P^T and dP^T
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status));
+      // ---- dS^T from P^T and dP^T; results over the buffer.
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full[wg], (it >> 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t ds[64];
       {
-        uint32_t d0[32], d1[32];
-        tmem_ld32(tDP, d0);
-        tmem_ld32(tDP + 32, d1);
-        tmem_ld_wait(d0);
-        tmem_ld_wait(d1);
-        uint32_t dk[16];
-        ds_cols(pv0, d0, ddv, 0.f, true, dk);
-        tmem_st16(tDP, dk);
-        ds_cols(pv1, d1, ddv + 32, 0.f, true, dk);
-        tmem_st16(tDP + 16, dk);
+        uint32_t dp[64];
+        tmem_ld64(tX, dp);  // queries 0..63
+        tmem_ld_wait64(dp);
+        ds_cols(pk, dp, ddv, 0.f, true, ds);
+        ds_cols(pk + 16, dp + 32, ddv + 32, 0.f, true, ds + 16);
+      }
+      {
+        // Columns [0, 64) are read: P^T goes there.
+        uint32_t (&pk0)[32] = *reinterpret_cast<uint32_t (*)[32]>(pk);
+        uint32_t (&pk1)[32] = *reinterpret_cast<uint32_t (*)[32]>(pk + 32);
+        tmem_st32(tX, pk0);
+        tmem_st32(tX + 32, pk1);
+      }
+      {
+        uint32_t dp[64];
+        tmem_ld64(tX + 64, dp);  // queries 64..127
+        tmem_ld_wait64(dp);
+        ds_cols(pk + 32, dp, ddv + 64, 0.f, true, ds + 32);
+        ds_cols(pk + 48, dp + 32, ddv + 96, 0.f, true, ds + 48);
+      }
+      {
+        uint32_t (&ds0)[32] = *reinterpret_cast<uint32_t (*)[32]>(ds);
+        uint32_t (&ds1)[32] = *reinterpret_cast<uint32_t (*)[32]>(ds + 32);
+        tmem_st32(tX + 64, ds0);
+        tmem_st32(tX + 96, ds1);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -518,12 +563,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p) {
   using C = BCfg<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the layout needs a 1024-aligned base (see BCfg)
+    if (threadIdx.x == 0) atomicOr(p.status, ATTN_DEV_LAYOUT);
+    return;
+  }
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + C::TILE;
-  uint8_t *sRing = smem + C::Q_RING_OFF;
+  uint8_t *sA = smem + C::Q_A_OFF;  // K ring
+  uint8_t *sB = smem + C::Q_B_OFF;  // V ring
   BBars *bars = reinterpret_cast<BBars *>(smem + C::Q_BAR_OFF);
   volatile int *abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -555,15 +603,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_items = max(0, je - js);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::Q_NST; ++i) {
-      mbar_init(&bars->full[i], 1);
-      mbar_init(&bars->empty[i], 1);
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&bars->a_full[i], 1);
+      mbar_init(&bars->a_empty[i], 1);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&bars->b_full[i], 1);
+      mbar_init(&bars->b_empty[i], 1);
     }
     mbar_init(&bars->res_full, 1);
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_full[0], 128);
-    mbar_init(&bars->p_full[1], 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->s_read[t], 128);
+      mbar_init(&bars->dp_full[t], 1);
+      mbar_init(&bars->p_full[t], 128);
+    }
     mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -581,86 +635,119 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ================================================================ producer
     regs_dec<kRegsLow>();
     if (lane == 0) {
+      // Q, dO once; then the K ring.
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(&bars->res_full, 2 * C::TILE);
       for (int c = 0; c < C::CH; ++c) {
         tma_load_3d(sQ + c * CHUNK, &tm_q, &bars->res_full, 64 * c, row0, bh);
         tma_load_3d(sdO + c * CHUNK, &tm_do, &bars->res_full, 64 * c, row0, bh);
       }
       int issued = 0;
-      for (int i = 0; i < 2 * n_items; ++i) {
-        const int slot = i % C::Q_NST, round = i / C::Q_NST;
-        if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(&bars->full[slot], C::TILE);
-        const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
+      for (int j = 0; j < n_items; ++j) {
+        const int slot = j % NA, round = j / NA;
+        if (round > 0 && !mbar_wait(&bars->a_empty[slot], (round - 1) & 1, abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(&bars->a_full[slot], C::TILE);
         for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(sRing + slot * C::TILE + c * CHUNK, map, &bars->full[slot], 64 * c,
-                      (js + (i >> 1)) * BT, bhk);
-        issued = i + 1;
+          tma_load_3d(sA + slot * C::TILE + c * CHUNK, &tm_k, &bars->a_full[slot], 64 * c,
+                      (js + j) * BT, bhk);
+        issued = j + 1;
       }
       mbar_wait_drain(&bars->res_full, 0, p.status);
-      for (int i = max(0, issued - C::Q_NST); i < issued; ++i)
-        mbar_wait_drain(&bars->full[i % C::Q_NST], (i / C::Q_NST) & 1, p.status);
+      for (int i = max(0, issued - NA); i < issued; ++i)
+        mbar_wait_drain(&bars->a_full[i % NA], (i / NA) & 1, p.status);
+    } else if (lane == 1) {
+      // The V ring.
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int j = 0; j < n_items; ++j) {
+        const int slot = j % NB, round = j / NB;
+        if (round > 0 && !mbar_wait(&bars->b_empty[slot], (round - 1) & 1, abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(&bars->b_full[slot], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sB + slot * C::TILE + c * CHUNK, &tm_v, &bars->b_full[slot], 64 * c,
+                      (js + j) * BT, bhk);
+        issued = j + 1;
+      }
+      for (int i = max(0, issued - NB); i < issued; ++i)
+        mbar_wait_drain(&bars->b_full[i % NB], (i / NB) & 1, p.status);
     }
   } else if (warp == 1) {
     // ================================================================== MMA
     regs_dec<kRegsLow>();
     if (lane == 0) {
-      const uint32_t ring = smem_u32(sRing);
       const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dodesc = qdesc + (C::TILE >> 4);
-      const uint64_t rk0 = sdesc_sw128(ring, 16, 1024);        // K or V, K-major
-      const uint64_t rmn0 = sdesc_sw128(ring, CHUNK, 1024);    // K, MN-major
-      auto slot_off = [](int i) { return static_cast<uint64_t>((i % C::Q_NST) * C::TILE) >> 4; };
-      auto wait_full = [&](int i) {
-        return mbar_wait(&bars->full[i % C::Q_NST], (i / C::Q_NST) & 1, abort_flag, p.status);
+      const uint64_t kk0 = sdesc_sw128(smem_u32(sA), 16, 1024);       // K, K-major
+      const uint64_t kmn0 = sdesc_sw128(smem_u32(sA), CHUNK, 1024);   // K, MN-major
+      const uint64_t vk0 = sdesc_sw128(smem_u32(sB), 16, 1024);       // V, K-major
+      auto a_off = [](int j) { return static_cast<uint64_t>((j % NA) * C::TILE) >> 4; };
+      auto b_off = [](int j) { return static_cast<uint64_t>((j % NB) * C::TILE) >> 4; };
+      auto wait_a = [&](int j) {
+        return mbar_wait(&bars->a_full[j % NA], (j / NA) & 1, abort_flag, p.status);
       };
-      auto issue_scores = [&](int jj) {  // S = Q K^T, commit; dP = dO V^T, commit
-        const uint64_t sk = slot_off(2 * jj), sv = slot_off(2 * jj + 1);
+      auto wait_b = [&](int j) {
+        return mbar_wait(&bars->b_full[j % NB], (j / NB) & 1, abort_flag, p.status);
+      };
+      auto issue_s = [&](int j) {  // S = Q K^T into buffer j & 1
+        const uint32_t d = tmem + col_x(j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t off = ((ks >> 2) * CHUNK + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + kColS, qdesc + off, rk0 + sk + off, C::IDESC_S, ks > 0);
+          mma_ss(d, qdesc + off, kk0 + a_off(j) + off, C::IDESC_S, ks > 0);
         }
-        tc_commit(&bars->s_full);
+        tc_commit(&bars->s_full[j & 1]);
+      };
+      auto issue_dp = [&](int j) {  // dP = dO V^T over S (already read)
+        const uint32_t d = tmem + col_x(j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t off = ((ks >> 2) * CHUNK + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + kColDP, dodesc + off, rk0 + sv + off, C::IDESC_S, ks > 0);
+          mma_ss(d, dodesc + off, vk0 + b_off(j) + off, C::IDESC_S, ks > 0);
         }
-        tc_commit(&bars->dp_full);
-        tc_commit(&bars->empty[(2 * jj + 1) % C::Q_NST]);  // V(jj) consumed by dP
+        tc_commit(&bars->dp_full[j & 1]);
+        tc_commit(&bars->b_empty[j % NB]);  // V(j) consumed
       };
-      auto issue_dq_half = [&](int jj, int h) {  // dQ += dS K over keys [64h, 64h+64)
-        const uint64_t sk = slot_off(2 * jj);
+      auto issue_dq = [&](int j) {  // dQ += dS K
+        const uint32_t x = tmem + col_x(j & 1);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int ks = 4 * h + kk;
-          mma_ts(tmem + kColAcc0, tmem + kColS + packed_col(ks), rmn0 + sk + ((ks * 2048) >> 4),
-                 C::IDESC_G, (jj > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < BT / 16; ++ks)
+          mma_ts(tmem + kColAcc0, x + ks * 8, kmn0 + a_off(j) + ((ks * 2048) >> 4), C::IDESC_G,
+                 (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(&bars->a_empty[j % NA]);  // K(j) consumed
       };
       bool ok = mbar_wait(&bars->res_full, 0, abort_flag, p.status);
-      if (ok && n_items > 0 && (ok = wait_full(0) && wait_full(1))) {
+      for (int j = 0; ok && j < 2 && j < n_items; ++j) {
+        if (!(ok = wait_a(j))) break;
         tc_fence_after();
-        issue_scores(0);
+        issue_s(j);
       }
-      for (int jj = 0; ok && jj < n_items; ++jj) {
-        for (int h = 0; h < 2; ++h) {
-          if (!(ok = mbar_wait(&bars->p_full[h], jj & 1, abort_flag, p.status))) break;
+      for (int j = 0; ok && j < n_items; ++j) {
+        const int bb = j & 1;
+        if (!(ok = mbar_wait(&bars->s_read[bb], (j >> 1) & 1, abort_flag, p.status) && wait_b(j)))
+          break;
+        tc_fence_after();
+        issue_dp(j);
+        if (j >= 1) {
+          if (!(ok = mbar_wait(&bars->p_full[bb ^ 1], ((j - 1) >> 1) & 1, abort_flag, p.status)))
+            break;
           tc_fence_after();
-          issue_dq_half(jj, h);
+          issue_dq(j - 1);
+          if (j + 1 < n_items) {
+            if (!(ok = wait_a(j + 1))) break;
+            tc_fence_after();
+            issue_s(j + 1);  // in order after dQ(j-1), which read this buffer
+          }
         }
-        if (!ok) break;
-        tc_commit(&bars->empty[(2 * jj) % C::Q_NST]);  // K(jj) consumed
-        if (jj + 1 < n_items) {
-          if (!(ok = wait_full(2 * jj + 2) && wait_full(2 * jj + 3))) break;
-          tc_fence_after();
-          issue_scores(jj + 1);  // in order after dQ(jj), which reads dS from these columns
-        }
+      }
+      if (ok && n_items > 0 &&
+          (ok = mbar_wait(&bars->p_full[(n_items - 1) & 1], ((n_items - 1) >> 1) & 1, abort_flag,
+                          p.status))) {
+        tc_fence_after();
+        issue_dq(n_items - 1);
       }
       tc_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, p.status);
@@ -670,63 +757,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ============================================================ elementwise
     regs_inc<kRegsHigh>();
-    const int wg = (warp - 4) >> 2;  // this warpgroup's 64 key columns
+    const int wg = (warp - 4) >> 2;  // this warpgroup takes tiles wg, wg + 2, ...
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int row = row0 + r;  // query row; rows >= N have l2 = +inf, so P = 0
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + 64 * wg;
-    const uint32_t tDP = tmem + lane_off + kColDP + 64 * wg;
+    const uint32_t tX = tmem + lane_off + col_x(wg);
     const float c = p.scale_log2;
     const float l2s = p.l2[static_cast<size_t>(bh) * p.Npad + row];
     const float dds = p.dvec[static_cast<size_t>(bh) * p.Npad + row];
     const float slope2 = kAlibi ? p.slopes[hq] * 1.4426950408889634f : 0.f;
     bool ok = true;
-    for (int jj = 0; jj < n_items; ++jj) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, jj & 1, abort_flag, p.status));
+    for (int j = wg; j < n_items; j += 2) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[wg], (j >> 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      const int kb = (js + jj) * BT + 64 * wg;  // first key of this warpgroup's columns
-      float pv0[32], pv1[32];
-      {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(tS, s0);
-        tmem_ld32(tS + 32, s1);
-        tmem_ld_wait(s0);
-        tmem_ld_wait(s1);
-        auto vis0 = [&](int i) {
+      uint32_t sv[128];
+      tmem_ld128(tX, sv);
+      tmem_ld_wait128(sv);
+      tc_fence_before();
+      mbar_arrive(&bars->s_read[wg]);  // the tensor pipe may now write dP here
+      const int kb0 = (js + j) * BT;     // first key of the tile
+      uint32_t pk[64];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int kb = kb0 + 32 * h;
+        auto vis = [&](int i) {
           const int kk = kb + i;
           return kk < p.N && (!p.causal || kk <= row) && (p.window <= 0 || row - kk < p.window);
         };
-        auto vis1 = [&](int i) { return vis0(i + 32); };
-        const bool full0 = kb + 31 < p.N && (!p.causal || kb + 31 <= row) &&
-                           (p.window <= 0 || row - kb < p.window);
-        const bool full1 = kb + 63 < p.N && (!p.causal || kb + 63 <= row) &&
-                           (p.window <= 0 || row - kb - 32 < p.window);
+        const bool full = kb + 31 < p.N && (!p.causal || kb + 31 <= row) &&
+                          (p.window <= 0 || row - kb < p.window);
         const float bias0 = slope2 * static_cast<float>(kb - row);
-        if (__all_sync(0xffffffffu, full0))
-          p_cols<kAlibi, false>(s0, nullptr, l2s, false, c, bias0, slope2, vis0, pv0);
+        if (__all_sync(0xffffffffu, full))
+          p_cols<kAlibi, false>(sv + 32 * h, nullptr, l2s, false, c, bias0, slope2, vis, pk + 16 * h);
         else
-          p_cols<kAlibi, true>(s0, nullptr, l2s, false, c, bias0, slope2, vis0, pv0);
-        if (__all_sync(0xffffffffu, full1))
-          p_cols<kAlibi, false>(s1, nullptr, l2s, false, c, bias0 + 32.f * slope2, slope2, vis1, pv1);
-        else
-          p_cols<kAlibi, true>(s1, nullptr, l2s, false, c, bias0 + 32.f * slope2, slope2, vis1, pv1);
+          p_cols<kAlibi, true>(sv + 32 * h, nullptr, l2s, false, c, bias0, slope2, vis, pk + 16 * h);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, jj & 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full[wg], (j >> 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t ds[64];
       {
-        uint32_t d0[32], d1[32];
-        tmem_ld32(tDP, d0);
-        tmem_ld32(tDP + 32, d1);
-        tmem_ld_wait(d0);
-        tmem_ld_wait(d1);
-        uint32_t dk[16];
-        ds_cols(pv0, d0, nullptr, dds, false, dk);
-        tmem_st16(tS, dk);
-        ds_cols(pv1, d1, nullptr, dds, false, dk);
-        tmem_st16(tS + 16, dk);
+        uint32_t dp[64];
+        tmem_ld64(tX, dp);  // keys 0..63
+        tmem_ld_wait64(dp);
+        ds_cols(pk, dp, nullptr, dds, false, ds);
+        ds_cols(pk + 16, dp + 32, nullptr, dds, false, ds + 16);
+      }
+      {
+        uint32_t dp[64];
+        tmem_ld64(tX + 64, dp);  // keys 64..127
+        tmem_ld_wait64(dp);
+        ds_cols(pk + 32, dp, nullptr, dds, false, ds + 32);
+        ds_cols(pk + 48, dp + 32, nullptr, dds, false, ds + 48);
+      }
+      {
+        uint32_t (&ds0)[32] = *reinterpret_cast<uint32_t (*)[32]>(ds);
+        uint32_t (&ds1)[32] = *reinterpret_cast<uint32_t (*)[32]>(ds + 32);
+        tmem_st32(tX, ds0);
+        tmem_st32(tX + 32, ds1);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -791,10 +881,10 @@ attn_status_t launch_bwd(const void *q, const void *k, const void *v, const void
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(bwd_dkdv_kernel<D, kAlibi>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM);
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_LAUNCH);
     if (attr_err == cudaSuccess)
       attr_err = cudaFuncSetAttribute(bwd_dq_kernel<D, kAlibi>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::Q_SMEM);
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::Q_LAUNCH);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
   const int BHq = prm.B * prm.Hq, BHk = prm.B * prm.Hkv;
@@ -805,9 +895,9 @@ attn_status_t launch_bwd(const void *q, const void *k, const void *v, const void
   const long long kv_ctas = static_cast<long long>((prm.N + BT - 1) / BT) * BHk;
   const long long q_ctas = static_cast<long long>((prm.N + BT - 1) / BT) * BHq;
   if (kv_ctas > 0x7fffffffLL || q_ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  bwd_dkdv_kernel<D, kAlibi><<<static_cast<unsigned>(kv_ctas), NUM_THREADS, C::KV_SMEM, stream>>>(
+  bwd_dkdv_kernel<D, kAlibi><<<static_cast<unsigned>(kv_ctas), NUM_THREADS, C::KV_LAUNCH, stream>>>(
       mk, mv, mq, mdo, prm);
-  bwd_dq_kernel<D, kAlibi><<<static_cast<unsigned>(q_ctas), NUM_THREADS, C::Q_SMEM, stream>>>(
+  bwd_dq_kernel<D, kAlibi><<<static_cast<unsigned>(q_ctas), NUM_THREADS, C::Q_LAUNCH, stream>>>(
       mq, mdo, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -65,6 +65,9 @@ typedef enum {
                                    outputs are NaN */
 #define ATTN_DEV_TIMEOUT 0x2u   /* a bounded wait inside the prefill kernel expired; the
                                    kernel returned early and its outputs are undefined */
+#define ATTN_DEV_LAYOUT 0x4u    /* a backward kernel found its dynamic shared memory not
+                                   1024-byte aligned and returned at once; the gradients
+                                   are undefined */
 
 /*
  * attn_fwd -- bf16 prefill, forward only.  Lab 01 steps 2 and 4 of the Phase 08
