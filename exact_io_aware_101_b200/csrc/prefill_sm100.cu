@@ -56,6 +56,7 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= NUM_THREADS * 168 && kRegsLow 
                   kRegsHigh % 8 == 0,
               "setmaxnreg split must fit the block's launch registers");
 constexpr int kHeadGroup = 8;  // causal schedule: heads whose K/V share L2 at a time
+constexpr int kRankMax = NUM_THREADS;  // chunked prefill: sequences ranked by length
 constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 128-byte swizzle column block
 
 template <int D>
@@ -154,7 +155,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // while a group's K/V stays in L2.
   const int BH = p.B * p.Hq;
   int pair, bh;
-  {
+  if constexpr (kPaged) {
+    // Chunked prefill: a CTA's work grows with its sequence's key count, which
+    // varies by up to the longest context over the shortest.  The grid takes
+    // the sequences longest first (ranked here by key count, ties by index),
+    // each one's heaviest pair first, all heads of a pair together, so that
+    // the last wave holds the short ones.  Past kRankMax sequences the order
+    // stays as given (the grid is then large enough to balance by itself).
+    const int lin = static_cast<int>(blockIdx.x);
+    const int per_seq = p.pairs * p.Hq;
+    const int r = lin / per_seq;
+    const int rem = lin - r * per_seq;
+    pair = p.pairs - 1 - rem / p.Hq;
+    int seq = r;
+    if (p.B <= kRankMax) {
+      __shared__ int s_len[kRankMax];
+      __shared__ int s_seq;
+      const int t = static_cast<int>(threadIdx.x);
+      if (t < p.B) s_len[t] = p.seq_lens[t];
+      __syncthreads();
+      if (t < p.B) {
+        const int nt = s_len[t];
+        int rank = 0;
+        for (int u = 0; u < p.B; ++u) rank += (s_len[u] > nt) || (s_len[u] == nt && u < t);
+        if (rank == r) s_seq = t;
+      }
+      __syncthreads();
+      seq = s_seq;
+    }
+    bh = seq * p.Hq + rem % p.Hq;
+  } else {
     const int lin = static_cast<int>(blockIdx.x);
     if (!p.causal) {
       bh = lin / p.pairs;
