@@ -348,6 +348,20 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start before the grid ahead of it in the
+// stream has finished; grid_dependency_wait() blocks until that grid has
+// completed and its memory writes are visible (it returns at once when the
+// kernel was launched without the attribute).  grid_dependents_launch() lets
+// such a dependent grid be scheduled once every CTA of this grid has called
+// it or exited; it does not make this grid's writes visible early.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Round two floats to bf16 (nearest-even) and pack: lo in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

@@ -76,6 +76,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
                         float *__restrict__ o_part, float *__restrict__ l2_part, int Hq, int Hkv,
                         int max_blocks, int num_pages, float scale_log2, int nsplit,
                         int head_chunks, unsigned *status) {
+  grid_dependents_launch();  // the combine kernel may be scheduled behind this grid
   using C = DecCfg<HC, D>;
   constexpr int LPT = D / 8;           // lanes per token row (8 bf16 = 16 B each)
   constexpr int TPI = 32 / LPT;        // token rows per warp-wide access
@@ -304,7 +305,13 @@ __global__ void __launch_bounds__((HC + 1) * 32)
   if (threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
 }
 
-// One warp per (sequence, head): merge the chunk partials.
+// One warp per (sequence, head): merge the chunk partials.  The lanes read the
+// chunks' log-sum-exps side by side (lane r holds chunks r, r + 32, ...), so
+// the weights cost one load round and two shuffle reductions; the weighted
+// rows are then summed eight chunks at a time with their loads issued
+// together.  Launched as a programmatic dependent of the split kernel: it may
+// start while the split kernel's last CTAs run, and waits for that grid to
+// finish (and its writes to be visible) before it reads a partial.
 template <int D>
 __global__ void __launch_bounds__(128)
     decode_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ l2_part,
@@ -312,8 +319,10 @@ __global__ void __launch_bounds__(128)
                           float *__restrict__ lse, int S, int Hq, int max_blocks, int nsplit,
                           int pages_per_split) {
   constexpr int DPL = D / 32;
+  constexpr int kBatch = 8;
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  grid_dependency_wait();
   if (gw >= S * Hq) return;
   const int s = gw / Hq;
   const int len = seq_lens[s];
@@ -331,11 +340,14 @@ __global__ void __launch_bounds__(128)
   const float *lp = l2_part + head * nsplit;
   bool bad = bad_len;
   float M = -INFINITY;
-  for (int r = 0; r < nparts; ++r) {
+  for (int r = lane; r < nparts; r += 32) {
     const float x = lp[r];
     bad |= isnan(x);
     M = fmaxf(M, x);
   }
+  bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   if (bad) {
 #pragma unroll
     for (int e = 0; e < DPL; ++e) orow[lane + 32 * e] = __float2bfloat16_rn(NAN);
@@ -346,13 +358,31 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
   float wsum = 0.f;
-  for (int r = 0; r < nparts; ++r) {
-    const float wt = ex2f(lp[r] - M);
-    wsum += wt;
-    const float *op = o_part + (head * nsplit + r) * D;
+  for (int r0 = 0; r0 < nparts; r0 += 32) {
+    // This lane's chunk weight; lanes past the end hold 0.
+    const float wl = r0 + lane < nparts ? ex2f(lp[r0 + lane] - M) : 0.f;
+    wsum += wl;
+    const int n = min(32, nparts - r0);
+    for (int rb = 0; rb < n; rb += kBatch) {
+      float v[kBatch][DPL];
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wt, op[lane + 32 * e], acc[e]);
+      for (int u = 0; u < kBatch; ++u) {
+        const float *op = o_part + (head * nsplit + r0 + min(rb + u, n - 1)) * D;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) v[u][e] = op[lane + 32 * e];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        // Chunks past the end re-read the last one with weight 0.
+        const float wt = __shfl_sync(0xffffffffu, wl, min(rb + u, 31));
+        const float w = rb + u < n ? wt : 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
+      }
+    }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
   const float inv = 1.f / wsum;
 #pragma unroll
   for (int e = 0; e < DPL; ++e) orow[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
@@ -479,16 +509,29 @@ attn_status_t launch_decode_combine(const float *o_part, const float *l2_part, c
                                     int nsplit, int pages_per_split, cudaStream_t stream) {
   const int heads = S * Hq;
   const int blocks = (heads + 3) / 4;
+  // Programmatic dependent launch: the grid may be scheduled while the split
+  // kernel before it in the stream finishes; the kernel waits for that grid.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+  cudaError_t err;
   if (d == 128)
-    decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(o_part, l2_part, seq_lens,
-                                                           static_cast<__nv_bfloat16 *>(o), lse, S,
-                                                           Hq, max_blocks, nsplit, pages_per_split);
+    err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, o_part, l2_part, seq_lens, ob, lse,
+                             S, Hq, max_blocks, nsplit, pages_per_split);
   else if (d == 64)
-    decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(o_part, l2_part, seq_lens,
-                                                          static_cast<__nv_bfloat16 *>(o), lse, S,
-                                                          Hq, max_blocks, nsplit, pages_per_split);
+    err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, o_part, l2_part, seq_lens, ob, lse,
+                             S, Hq, max_blocks, nsplit, pages_per_split);
   else
     return ATTN_ERR_UNSUPPORTED;
+  if (err != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -194,6 +194,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
                            float *__restrict__ o_part, float *__restrict__ l2_part, int Hq,
                            int Hkv, int max_blocks, int num_pages, float scale_log2, int nsplit,
                            int head_chunks, unsigned *status) {
+  grid_dependents_launch();  // the combine kernel may be scheduled behind this grid
   using C = Q8Cfg<HC, D>;
   constexpr int KS = D / 16;   // k-steps of the q.k MMA = M-tiles of the p.v MMA
   constexpr int KCH = D / 64;  // 16-byte chunks of a K row held by one thread
