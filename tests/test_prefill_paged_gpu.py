@@ -70,6 +70,20 @@ def test_prefill_paged_small(qlens, ctxs, Hq, Hkv, d):
     assert ea.device_status() == 0
 
 
+@pytest.mark.parametrize("qlens,ctxs", [
+    # Equal key counts (the work order breaks ties by sequence index).
+    ([9, 9, 30, 9, 30], [40, 40, 19, 40, 19]),
+    # More sequences than the kernel ranks (384): the grid keeps the given order.
+    ([3] * 400, [i % 37 for i in range(400)]),
+])
+def test_prefill_paged_work_order(qlens, ctxs):
+    cfg, inp = make(qlens, ctxs, 2, 1, 64, seed=len(qlens))
+    o_ref, l_ref = oracle_run(inp, cfg.scale)
+    o, l = gpu_run(inp, cfg.scale)
+    assert_bf16_parity(o, l, o_ref, l_ref, (len(qlens), "sequences"))
+    assert ea.device_status() == 0
+
+
 def test_prefill_paged_window_and_alibi():
     # Window and ALiBi measured from the chunk query's absolute position;
     # checked against rows ctx.. of the contiguous causal prefill's oracle.
