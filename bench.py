@@ -349,7 +349,14 @@ def timed_launches(items, flush, reps):
 
 
 def e2e_sweep(items, reps):
-    """The sweep through the public API with pinned host buffers (H2D + call + D2H)."""
+    """The sweep through the public API with pinned host buffers (H2D + call + D2H).
+
+    Every step copies each workload's q, k, v from pinned host memory, calls
+    attn_fwd on them and reads O and L back into pinned host memory.  The
+    copies in, the calls and the copies out run on three streams ordered by
+    events, so one workload's copy overlaps the previous one's kernel and the
+    read-back before that (host-device copies in both directions share the
+    link at once).  The event pair brackets all three streams."""
     import exact_io_aware_101_b200 as ea
     host = []
     for it in items:
@@ -358,23 +365,45 @@ def e2e_sweep(items, reps):
                          l=torch.empty(it.lse.shape, dtype=torch.float32).pin_memory()))
     h2d = sum(h["q"].nbytes + h["k"].nbytes + h["v"].nbytes for h in host)
     d2h = sum(h["o"].nbytes + h["l"].nbytes for h in host)
+    dev = [dict(q=torch.empty_like(it.q), k=torch.empty_like(it.k), v=torch.empty_like(it.v))
+           for it in items]
+    s_run = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in items]
+    ev_run = [torch.cuda.Event() for _ in items]
+    ran = [False] * len(items)
 
     def once():
-        for it, h in zip(items, host):
-            q = h["q"].to("cuda", non_blocking=True)
-            k = h["k"].to("cuda", non_blocking=True)
-            v = h["v"].to("cuda", non_blocking=True)
-            o, l = ea.attn_fwd(q, k, v, causal=it.cfg.causal, scale=it.cfg.scale)
-            h["o"].copy_(o, non_blocking=True)
-            h["l"].copy_(l, non_blocking=True)
+        for i, (it, h, d) in enumerate(zip(items, host, dev)):
+            if ran[i]:
+                s_in.wait_event(ev_run[i])  # the last call on these buffers is done
+            with torch.cuda.stream(s_in):
+                d["q"].copy_(h["q"], non_blocking=True)
+                d["k"].copy_(h["k"], non_blocking=True)
+                d["v"].copy_(h["v"], non_blocking=True)
+                ev_in[i].record(s_in)
+            s_run.wait_event(ev_in[i])
+            o, l = ea.attn_fwd(d["q"], d["k"], d["v"], causal=it.cfg.causal, scale=it.cfg.scale)
+            ev_run[i].record(s_run)
+            s_out.wait_event(ev_run[i])
+            with torch.cuda.stream(s_out):
+                h["o"].copy_(o, non_blocking=True)
+                h["l"].copy_(l, non_blocking=True)
+            o.record_stream(s_out)
+            l.record_stream(s_out)
+            ran[i] = True
 
     once()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(s_run)
+    s_in.wait_stream(s_run)
+    s_out.wait_stream(s_run)
     for _ in range(reps):
         once()
-    e1.record()
+    s_run.wait_stream(s_in)
+    s_run.wait_stream(s_out)
+    e1.record(s_run)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / reps, h2d, d2h
 
