@@ -35,10 +35,12 @@
 // 128, contiguous in the pool).  The box is 128-byte swizzled (64-byte for d =
 // 64), which makes both fragment patterns conflict-free: K rows read along d,
 // and V read across token rows at one column.  Each consumer warp owns one
-// K/V head, walks every page of the chunk with a running max / sum (online
-// softmax, lazily rescaled), and writes its heads' normalised partials; the
-// combine kernel of decode_paged.cu merges the chunks exactly as for the
-// 16-bit cache.
+// K/V head and walks the chunk's pages two at a time with a running max / sum
+// (online softmax, lazily rescaled): the two pages' loads, conversions and
+// MMAs are independent and branch-free, so they interleave, and the softmax
+// bookkeeping runs once per 32 tokens.  It writes its heads' normalised
+// partials; the combine kernel of decode_paged.cu merges the chunks exactly as
+// for the 16-bit cache.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -343,109 +345,138 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     const int src0 = 8 * c + (g >> 1), src1 = src0 + 4;
     const uint32_t psel = (g & 1) ? 0x7632u : 0x5410u;
 
-    for (int i = 0; i < npg; ++i) {
-      const int st = i % C::NST;
-      const bool ok = mbar_wait(&full[st], (i / C::NST) & 1, &sm_abort, status);
+    // S^T = K . Q^T of one page for tokens g and g+8, scaled to log2 units and
+    // masked past the page's live tokens.  Branch-free, so that two pages'
+    // loads, conversions and MMAs interleave: a page with no live token (a bad
+    // page id, or the missing partner of an odd last page) reads a stage whose
+    // last copy has completed and been consumed, and every score is masked.
+    auto page_scores = [&](const uint8_t *kt, int ntok, float ks, float (&sv)[4]) {
+      uint4 ka[KCH], kb[KCH];
+#pragma unroll
+      for (int h = 0; h < KCH; ++h) {
+        const uint32_t col = static_cast<uint32_t>((D / 4) * c + 16 * h);
+        ka[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>(g * D + col));
+        kb[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>((g + 8) * D + col));
+      }
+      float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int t = 0; t < KS; ++t) {
+        const uint4 &A = ka[t / 4], &B = kb[t / 4];
+        const uint32_t wa = (t % 4 == 0) ? A.x : (t % 4 == 1) ? A.y : (t % 4 == 2) ? A.z : A.w;
+        const uint32_t wb = (t % 4 == 0) ? B.x : (t % 4 == 1) ? B.y : (t % 4 == 2) ? B.z : B.w;
+        mma_f16((t & 1) ? sd : sc, codes_f16x2<FMT>(wa, 0), codes_f16x2<FMT>(wb, 0),
+                codes_f16x2<FMT>(wa, 1), codes_f16x2<FMT>(wb, 1), qb[t][0], qb[t][1]);
+      }
+      const float kq0 = ks * sq0, kq1 = ks * sq1;
+      sv[0] = g < ntok ? (sc[0] + sd[0]) * kq0 : -INFINITY;
+      sv[1] = g < ntok ? (sc[1] + sd[1]) * kq1 : -INFINITY;
+      sv[2] = g + 8 < ntok ? (sc[2] + sd[2]) * kq0 : -INFINITY;
+      sv[3] = g + 8 < ntok ? (sc[3] + sd[3]) * kq1 : -INFINITY;
+    };
+    auto p_frag = [&](const float (&pv)[4], float f0, float f1, uint32_t &pb0, uint32_t &pb1) {
+      const uint32_t P01 = pack_f16x2(pv[0] * f0, pv[1] * f1);
+      const uint32_t P23 = pack_f16x2(pv[2] * f0, pv[3] * f1);
+      const uint32_t x0 = __shfl_sync(0xffffffffu, P01, src0);
+      const uint32_t x1 = __shfl_sync(0xffffffffu, P01, src1);
+      const uint32_t y0 = __shfl_sync(0xffffffffu, P23, src0);
+      const uint32_t y1 = __shfl_sync(0xffffffffu, P23, src1);
+      pb0 = prmt(x0, x1, psel);
+      pb1 = prmt(y0, y1, psel);
+    };
+
+    for (int i = 0; i < npg; i += 2) {
+      const bool two = i + 1 < npg;
+      const int sta = i % C::NST, stb = (i + 1) % C::NST;
+      bool ok = mbar_wait(&full[sta], (i / C::NST) & 1, &sm_abort, status);
+      if (two) ok = ok && mbar_wait(&full[stb], ((i + 1) / C::NST) & 1, &sm_abort, status);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const int ntok = stage_ntok[st];
-      const float ks = __shfl_sync(0xffffffffu, ks_r, i);
-      const float vs = __shfl_sync(0xffffffffu, vs_r, i);
-      if (ntok > 0) {
-        const uint8_t *kt = ring + st * C::STAGE + warp * C::SLICE;
-        const uint8_t *vt = ring + st * C::STAGE + (HC + warp) * C::SLICE;
-        // ---- S^T = K . Q^T for tokens g and g+8.
-        uint4 ka[KCH], kb[KCH];
+      const int na = stage_ntok[sta];
+      const int nb = two ? stage_ntok[stb] : 0;
+      const float ksa = __shfl_sync(0xffffffffu, ks_r, i);
+      const float vsa = __shfl_sync(0xffffffffu, vs_r, i);
+      const float ksb = __shfl_sync(0xffffffffu, ks_r, (i + 1) & 31);
+      const float vsb_r = __shfl_sync(0xffffffffu, vs_r, (i + 1) & 31);
+      const float vsb = two ? vsb_r : 0.f;
+      const uint8_t *sga = ring + sta * C::STAGE, *sgb = ring + stb * C::STAGE;
+      float sa[4], sb[4];
+      page_scores(sga + warp * C::SLICE, na, ksa, sa);
+      page_scores(sgb + warp * C::SLICE, nb, ksb, sb);
+      const float lva = vsa > 0.f ? __log2f(vsa) : -INFINITY;
+      const float lvb = vsb > 0.f ? __log2f(vsb) : -INFINITY;
+      const float ma0 = fmaxf(sa[0], sa[2]), ma1 = fmaxf(sa[1], sa[3]);
+      const float mb0 = fmaxf(sb[0], sb[2]), mb1 = fmaxf(sb[1], sb[3]);
+      float mx0 = fmaxf(ma0, mb0), mx1 = fmaxf(ma1, mb1);
+      float cv0 = fmaxf(ma0 + lva, mb0 + lvb), cv1 = fmaxf(ma1 + lva, mb1 + lvb);
 #pragma unroll
-        for (int h = 0; h < KCH; ++h) {
-          const uint32_t col = static_cast<uint32_t>((D / 4) * c + 16 * h);
-          ka[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>(g * D + col));
-          kb[h] = *reinterpret_cast<const uint4 *>(kt + swz<D>((g + 8) * D + col));
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        cv0 = fmaxf(cv0, __shfl_xor_sync(0xffffffffu, cv0, o));
+        cv1 = fmaxf(cv1, __shfl_xor_sync(0xffffffffu, cv1, o));
+      }
+      if (__any_sync(0xffffffffu, (mx0 > m0 + kRescaleLog2) || (mx1 > m1 + kRescaleLog2))) {
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        l0 *= ex2(m0 - n0);
+        l1 *= ex2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+      }
+      float pa[4], pb[4];
+      pa[0] = ex2(sa[0] - m0), pa[1] = ex2(sa[1] - m1), pa[2] = ex2(sa[2] - m0), pa[3] = ex2(sa[3] - m1);
+      pb[0] = ex2(sb[0] - m0), pb[1] = ex2(sb[1] - m1), pb[2] = ex2(sb[2] - m0), pb[3] = ex2(sb[3] - m1);
+      l0 += (pa[0] + pa[2]) + (pb[0] + pb[2]);
+      l1 += (pa[1] + pa[3]) + (pb[1] + pb[3]);
+      if (__any_sync(0xffffffffu, (cv0 > mv0 + kRescaleLog2) || (cv1 > mv1 + kRescaleLog2))) {
+        const float n0 = fmaxf(mv0, cv0), n1 = fmaxf(mv1, cv1);
+        const float a0 = ex2(mv0 - n0), a1 = ex2(mv1 - n1);
+#pragma unroll
+        for (int i2 = 0; i2 < KS; ++i2) {
+          acc[i2][0] *= a0;
+          acc[i2][1] *= a1;
+          acc[i2][2] *= a0;
+          acc[i2][3] *= a1;
         }
-        // Two accumulator chains (even / odd k-steps) halve the MMA latency chain.
-        float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
+        mv0 = n0;
+        mv1 = n1;
+      }
+      const float e0 = mv0 == -INFINITY ? 0.f : ex2(m0 - mv0);
+      const float e1 = mv1 == -INFINITY ? 0.f : ex2(m1 - mv1);
+      uint32_t pa0, pa1, pb0, pb1;
+      p_frag(pa, vsa * e0, vsa * e1, pa0, pa1);
+      p_frag(pb, vsb * e0, vsb * e1, pb0, pb1);
+      const uint8_t *vta = sga + (HC + warp) * C::SLICE, *vtb = sgb + (HC + warp) * C::SLICE;
+      const VRow<D> va = load_vrow<D>(vta, 2 * c, g, 2 * c < na);
+      const VRow<D> vb = load_vrow<D>(vta, 2 * c + 1, g, 2 * c + 1 < na);
+      const VRow<D> vc = load_vrow<D>(vta, 2 * c + 8, g, 2 * c + 8 < na);
+      const VRow<D> vd = load_vrow<D>(vta, 2 * c + 9, g, 2 * c + 9 < na);
+      const VRow<D> wa = load_vrow<D>(vtb, 2 * c, g, 2 * c < nb);
+      const VRow<D> wb = load_vrow<D>(vtb, 2 * c + 1, g, 2 * c + 1 < nb);
+      const VRow<D> wc = load_vrow<D>(vtb, 2 * c + 8, g, 2 * c + 8 < nb);
+      const VRow<D> wd = load_vrow<D>(vtb, 2 * c + 9, g, 2 * c + 9 < nb);
 #pragma unroll
-        for (int t = 0; t < KS; ++t) {
-          const uint4 &A = ka[t / 4], &B = kb[t / 4];
-          const uint32_t wa = (t % 4 == 0) ? A.x : (t % 4 == 1) ? A.y : (t % 4 == 2) ? A.z : A.w;
-          const uint32_t wb = (t % 4 == 0) ? B.x : (t % 4 == 1) ? B.y : (t % 4 == 2) ? B.z : B.w;
-          mma_f16((t & 1) ? sd : sc, codes_f16x2<FMT>(wa, 0), codes_f16x2<FMT>(wb, 0),
-                  codes_f16x2<FMT>(wa, 1), codes_f16x2<FMT>(wb, 1), qb[t][0], qb[t][1]);
-        }
+      for (int w = 0; w < D / 32; ++w) {
+        uint32_t lo[4], hi[4], lo2[4], hi2[4];
+        vpairs<FMT>(va.w[w], vb.w[w], lo);
+        vpairs<FMT>(vc.w[w], vd.w[w], hi);
+        vpairs<FMT>(wa.w[w], wb.w[w], lo2);
+        vpairs<FMT>(wc.w[w], wd.w[w], hi2);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sc[e] += sd[e];
-        const float kq0 = ks * sq0, kq1 = ks * sq1;
-        float s0 = sc[0] * kq0, s1 = sc[1] * kq1, s2 = sc[2] * kq0, s3 = sc[3] * kq1;
-        if (ntok < kPage) {
-          if (g >= ntok) s0 = s1 = -INFINITY;
-          if (g + 8 >= ntok) s2 = s3 = -INFINITY;
-        }
-        // ---- online softmax per head (column), over the page's 16 tokens.
-        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        if (__any_sync(0xffffffffu, (mx0 > m0 + kRescaleLog2) || (mx1 > m1 + kRescaleLog2))) {
-          const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-          l0 *= ex2(m0 - n0);
-          l1 *= ex2(m1 - n1);
-          m0 = n0;
-          m1 = n1;
-        }
-        const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
-        l0 += p0 + p2;
-        l1 += p1 + p3;
-        // ---- contribution scale of the page: its score max plus log2(V scale).
-        const float lvs = vs > 0.f ? __log2f(vs) : -INFINITY;
-        const float cv0 = mx0 + lvs, cv1 = mx1 + lvs;
-        if (__any_sync(0xffffffffu, (cv0 > mv0 + kRescaleLog2) || (cv1 > mv1 + kRescaleLog2))) {
-          const float n0 = fmaxf(mv0, cv0), n1 = fmaxf(mv1, cv1);
-          const float a0 = ex2(mv0 - n0), a1 = ex2(mv1 - n1);  // 0 while mv was -inf
-#pragma unroll
-          for (int i2 = 0; i2 < KS; ++i2) {
-            acc[i2][0] *= a0;
-            acc[i2][1] *= a1;
-            acc[i2][2] *= a0;
-            acc[i2][3] *= a1;
-          }
-          mv0 = n0;
-          mv1 = n1;
-        }
-        // f16 operand: p * vscale * 2^(m - mv) = 2^(s + log2 vscale - mv).
-        const float f0 = mv0 == -INFINITY ? 0.f : vs * ex2(m0 - mv0);
-        const float f1 = mv1 == -INFINITY ? 0.f : vs * ex2(m1 - mv1);
-        // ---- P^T fragment: (P[head g][tok 2c], [2c+1]) and tokens 2c+8, 2c+9.
-        const uint32_t P01 = pack_f16x2(p0 * f0, p1 * f1), P23 = pack_f16x2(p2 * f0, p3 * f1);
-        const uint32_t x0 = __shfl_sync(0xffffffffu, P01, src0);
-        const uint32_t x1 = __shfl_sync(0xffffffffu, P01, src1);
-        const uint32_t y0 = __shfl_sync(0xffffffffu, P23, src0);
-        const uint32_t y1 = __shfl_sync(0xffffffffu, P23, src1);
-        const uint32_t pb0 = prmt(x0, x1, psel), pb1 = prmt(y0, y1, psel);
-        // ---- O^T += V^T . P^T.  Rows past the sequence end read as zero.
-        const VRow<D> va = load_vrow<D>(vt, 2 * c, g, 2 * c < ntok);
-        const VRow<D> vb = load_vrow<D>(vt, 2 * c + 1, g, 2 * c + 1 < ntok);
-        const VRow<D> vc = load_vrow<D>(vt, 2 * c + 8, g, 2 * c + 8 < ntok);
-        const VRow<D> vd = load_vrow<D>(vt, 2 * c + 9, g, 2 * c + 9 < ntok);
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) {
-          uint32_t lo[4], hi[4];
-          vpairs<FMT>(va.w[w], vb.w[w], lo);
-          vpairs<FMT>(vc.w[w], vd.w[w], hi);
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            float t4[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_f16(t4, lo[2 * e2], lo[2 * e2 + 1], hi[2 * e2], hi[2 * e2 + 1], pb0, pb1);
-            float(&a)[4] = acc[2 * w + e2];
-            a[0] += t4[0];
-            a[1] += t4[1];
-            a[2] += t4[2];
-            a[3] += t4[3];
-          }
+        for (int e2 = 0; e2 < 2; ++e2) {
+          float t4[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_f16(t4, lo[2 * e2], lo[2 * e2 + 1], hi[2 * e2], hi[2 * e2 + 1], pa0, pa1);
+          mma_f16(t4, lo2[2 * e2], lo2[2 * e2 + 1], hi2[2 * e2], hi2[2 * e2 + 1], pb0, pb1);
+          float(&a)[4] = acc[2 * w + e2];
+          a[0] += t4[0];
+          a[1] += t4[1];
+          a[2] += t4[2];
+          a[3] += t4[3];
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
+      if (lane == 0) {
+        mbar_arrive(&empty[sta]);
+        if (two) mbar_arrive(&empty[stb]);
+      }
     }
 
     // Sums over the page tokens (lanes sharing c hold the same heads).
