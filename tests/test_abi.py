@@ -54,6 +54,17 @@ def test_only_the_c_abi_is_exported(lib):
     assert {s for s in exported if s.startswith("attn_")} == declared_functions()
 
 
+def test_device_status_bits_match_the_header():
+    text = open(os.path.join(ROOT, "include", "exattn.h")).read()
+    bits = {name: int(val, 16) for name, val in
+            re.findall(r"#define\s+(ATTN_DEV_[A-Z_]+)\s+(0x[0-9a-fA-F]+)u", text)}
+    assert set(bits) == {"ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "ATTN_DEV_LAYOUT"}
+    for name, val in bits.items():
+        assert getattr(ea, name) == val, name
+    assert len(set(bits.values())) == len(bits)  # distinct bits
+    assert all(v & (v - 1) == 0 for v in bits.values())  # one bit each
+
+
 def test_version_and_status_strings(lib):
     assert "sm_100a" in ea.version()
     assert ea.status_string(0) == "ATTN_OK"
