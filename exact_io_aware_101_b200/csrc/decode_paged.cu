@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kPageSize = 16;
 constexpr int kPagesPerSplit = 32;  // 512 tokens per chunk
+constexpr float kRescaleLog2 = 8.f;  // lazy rescale: move the max only when it grows by > 2^8
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -231,15 +232,21 @@ __global__ void __launch_bounds__((HC + 1) * 32)
         for (int it = 1; it < IT; ++it) mx = fmaxf(mx, sc[it]);
 #pragma unroll
         for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float m_new = fmaxf(m, mx);  // finite: row 0 of a page is always visible
-        const float alpha = ex2f(m - m_new);
-        m = m_new;
-        l *= alpha;
+        // Lazy rescale: the reference m moves (and l, acc are rescaled) only
+        // when a score exceeds it by more than 2^8, so P <= 2^8 in fp32 and
+        // most pages skip the rescale.  mx is finite: row 0 of a page is
+        // always visible.
+        if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+          const float m_new = fmaxf(m, mx);
+          const float alpha = ex2f(m - m_new);  // 0 on the first page (m = -inf)
+          m = m_new;
+          l *= alpha;
 #pragma unroll
-        for (int hh = 0; hh < GB; ++hh) {
-          const float a = __shfl_sync(0xffffffffu, alpha, hh * (LPT / GB));
+          for (int hh = 0; hh < GB; ++hh) {
+            const float a = __shfl_sync(0xffffffffu, alpha, hh * (LPT / GB));
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[hh][e] = make_float2(acc[hh][e].x * a, acc[hh][e].y * a);
+            for (int e = 0; e < 4; ++e) acc[hh][e] = make_float2(acc[hh][e].x * a, acc[hh][e].y * a);
+          }
         }
         // P V: each lane needs every head's weight for its rows.
 #pragma unroll
