@@ -14,7 +14,8 @@ The JSON line also carries, measured in the same run:
     peak; the chunked prefill over the paged cache (16 sequences, a 512-token
     chunk after U[0, 7680] cached tokens) in TFLOP/s; and the backward (dQ,
     dK, dV) of the N=8192 MHA and causal workloads in TFLOP/s of the
-    algorithm's five products;
+    algorithm's five products.  Each component is the median of its flushed
+    launches (the mean is kept beside it as ``ms_mean``);
   * ``roofline`` for the prefill kernel (tensor-bound);
   * ``e2e``: the same sweep through the public API with pinned host buffers,
     host->device and device->host copies inside the timed region;
@@ -348,6 +349,16 @@ def timed_launches(items, flush, reps):
     return [[a.elapsed_time(b) for a, b in row] for row in times], launches
 
 
+def component_time(ms_list):
+    """Median (seconds) and mean (ms) of one component's flushed launch times: the
+    median is the reported figure, robust to a slow launch while clocks or power
+    settle after the previous component; the mean is kept beside it."""
+    ts = sorted(ms_list)
+    n = len(ts)
+    med = ts[n // 2] if n % 2 else 0.5 * (ts[n // 2 - 1] + ts[n // 2])
+    return med / 1e3, sum(ts) / n
+
+
 def e2e_sweep(items, reps):
     """The sweep through the public API with pinned host buffers (H2D + call + D2H).
 
@@ -537,39 +548,40 @@ def run_ours(args):
         line["clocks"] = clocks
 
     if not args.skip_components:
-        comps = {}
+        comps = {"_timing": "per component: 3 warm-up launches, then args.component_reps "
+                            "launches each after an L2 flush; ms = median, ms_mean = mean"}
         for cfg in (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI):
             it = Prefill(cfg, lib)
             timed_launches([it], flush, 3)
             t, _ = timed_launches([it], flush, args.component_reps)
-            sec = sum(t[0]) / len(t[0]) / 1e3
+            sec, mean_ms = component_time(t[0])
             tf = cfg.flops / sec / 1e12
-            comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3}
+            comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3, "ms_mean": mean_ms}
             del it
         it = ChunkedPrefill(syn.CHUNKED, lib)
         timed_launches([it], flush, 3)
         t, _ = timed_launches([it], flush, args.component_reps)
-        sec = sum(t[0]) / len(t[0]) / 1e3
+        sec, mean_ms = component_time(t[0])
         tf = it.flops / sec / 1e12
-        comps[syn.CHUNKED.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3,
+        comps[syn.CHUNKED.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3, "ms_mean": mean_ms,
                                    "flops": it.flops, "flops_counted": "4*d per visible pair"}
         del it
         for cfg in (syn.MHA_SWEEP[-1], syn.CAUSAL):
             it = Backward(cfg, lib)
             timed_launches([it], flush, 3)
             t, _ = timed_launches([it], flush, args.component_reps)
-            sec = sum(t[0]) / len(t[0]) / 1e3
+            sec, mean_ms = component_time(t[0])
             tf = it.flops / sec / 1e12
             comps["bwd_" + cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf,
-                                        "ms": sec * 1e3, "flops": it.flops,
+                                        "ms": sec * 1e3, "ms_mean": mean_ms, "flops": it.flops,
                                         "flops_counted": "5 products of the algorithm (2.5x fwd)"}
             del it
         dec = Decode(syn.DECODE, lib)
         timed_launches([dec], flush, 3)
         t, _ = timed_launches([dec], flush, args.component_reps)
-        sec = sum(t[0]) / len(t[0]) / 1e3
+        sec, mean_ms = component_time(t[0])
         gbs = dec.bytes / sec / 1e9
-        comps["decode_paged_gqa"] = {"gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3,
+        comps["decode_paged_gqa"] = {"gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3, "ms_mean": mean_ms,
                                      "algorithmic_bytes": dec.bytes,
                                      "peak_gbs": peak_hbm,
                                      "traffic": profiled_traffic("decode_paged_gqa.md",
@@ -580,10 +592,10 @@ def run_ours(args):
             dq = DecodeQ8(syn.DECODE, lib, fmt)
             timed_launches([dq], flush, 3)
             t, _ = timed_launches([dq], flush, args.component_reps)
-            sec = sum(t[0]) / len(t[0]) / 1e3
+            sec, mean_ms = component_time(t[0])
             gbs = dq.bytes / sec / 1e9
             comps["decode_paged_gqa_" + fmt] = {
-                "gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3,
+                "gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3, "ms_mean": mean_ms,
                 "algorithmic_bytes": dq.bytes, "peak_gbs": peak_hbm,
                 "traffic": profiled_traffic("decode_q8_gqa.md", "decode_q8.cu"), "bound": "hbm"}
             del dq
