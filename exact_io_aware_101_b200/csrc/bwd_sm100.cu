@@ -26,15 +26,18 @@
 // scatters dQ with atomic adds (7 instead of 5); the FLOP rate reported counts
 // the 5 of the algorithm.
 //
-// Scheduling.  All MMAs are 128 wide.  Each tile uses one 128-column TMEM
-// buffer twice: the score tile S (S^T) is written there, the elementwise warps
-// load it into registers and say so, and the tensor pipe then writes dP (dP^T)
-// over it; the warps finally store their bf16 results (P^T and dS^T, or dS)
-// into the same columns.  Two such buffers next to the 128-column
-// accumulators (dV and dK, or dQ) keep two tiles in flight, and the two
-// elementwise warpgroups take alternate tiles.  Per tile the MMA issuer runs
-// dP(i), then the gradient products of tile i-1 and the scores of tile i+1,
-// so the exponentials of one tile overlap the other tile's products.  The
+// Scheduling.  All MMAs are 128 wide, and the two elementwise warpgroups take
+// alternate tiles.  dK/dV kernel: each tile uses one 128-column TMEM buffer
+// twice: the score tile S^T is written there, the tile's warpgroup loads it
+// into registers and says so, and the tensor pipe then writes dP^T over it;
+// the warps finally store their bf16 P^T and dS^T into the same columns.  Two
+// such buffers next to dV and dK keep two tiles in flight; per tile the MMA
+// issuer runs dP(i), then the gradient products of tile i-1 and the scores of
+// tile i+1, so the exponentials of one tile overlap the other's products.
+// dQ kernel: with one accumulator, TMEM has room for a dP buffer of its own
+// beside the two score buffers, so no product waits for a score tile to be
+// read: per tile j it runs dP(j+1) (once warpgroup j has read dP(j)), dQ(j)
+// (once dS(j) is in the score buffer), then S(j+2) into that buffer.  The
 // streamed tile whose product comes last (Q for dK, K for dQ) is live for
 // three iterations and gets a three-slot ring; the other (dO, V) two slots.
 //
@@ -66,12 +69,15 @@ constexpr int CHUNK = BT * 128;  // 128 rows x 128 bytes: one 64-column block of
 constexpr int NA = 3;            // slots of the three-iteration ring (Q or K)
 constexpr int NB = 2;            // slots of the two-iteration ring (dO + vectors, or V)
 
-// TMEM: two 128-column tile buffers, then the accumulators.  In a buffer the
-// bf16 results sit at columns [0, 64) (P^T, or dS) and [64, 128) (dS^T): the
-// 128 values of a row, two per column.
+// TMEM: two 128-column tile buffers, then the accumulators (dK/dV kernel) or
+// the dP buffer and the accumulator (dQ kernel).  In a tile buffer the bf16
+// results sit at columns [0, 64) (P^T, or dS) and [64, 128) (dS^T): the 128
+// values of a row, two per column.
 __device__ __forceinline__ uint32_t col_x(int buf) { return static_cast<uint32_t>(buf) * 128; }
-constexpr uint32_t kColAcc0 = 256;  // dV (dK/dV kernel) or dQ (dQ kernel)
+constexpr uint32_t kColAcc0 = 256;  // dV (dK/dV kernel)
 constexpr uint32_t kColAcc1 = 384;  // dK (dK/dV kernel)
+constexpr uint32_t kColDP = 256;    // dP (dQ kernel): a buffer of its own
+constexpr uint32_t kColDQ = 384;    // dQ (dQ kernel)
 
 template <int D>
 struct BCfg {
@@ -107,7 +113,8 @@ struct BBars {
   uint64_t b_full[NB], b_empty[NB];  // dO + vectors, or V ring
   uint64_t res_full;                 // the resident tiles
   uint64_t s_full[2];    // buffer w holds S (S^T) of its tile
-  uint64_t s_read[2];    // warpgroup w has loaded it into registers (count 128)
+  uint64_t s_read[2];    // warpgroup w has loaded its tile into registers (count 128):
+                         // S^T (dK/dV kernel) or dP (dQ kernel)
   uint64_t dp_full[2];   // buffer w holds dP (dP^T)
   uint64_t p_full[2];    // warpgroup w's bf16 results are in buffer w (count 128)
   uint64_t mma_done;
@@ -701,8 +708,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_commit(&bars->s_full[j & 1]);
       };
-      auto issue_dp = [&](int j) {  // dP = dO V^T over S (already read)
-        const uint32_t d = tmem + col_x(j & 1);
+      auto issue_dp = [&](int j) {  // dP = dO V^T into the dP buffer
+        const uint32_t d = tmem + kColDP;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t off = ((ks >> 2) * CHUNK + (ks & 3) * 32) >> 4;
@@ -715,39 +722,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t x = tmem + col_x(j & 1);
 #pragma unroll
         for (int ks = 0; ks < BT / 16; ++ks)
-          mma_ts(tmem + kColAcc0, x + ks * 8, kmn0 + a_off(j) + ((ks * 2048) >> 4), C::IDESC_G,
+          mma_ts(tmem + kColDQ, x + ks * 8, kmn0 + a_off(j) + ((ks * 2048) >> 4), C::IDESC_G,
                  (j > 0 || ks > 0) ? 1u : 0u);
         tc_commit(&bars->a_empty[j % NA]);  // K(j) consumed
       };
+      // dP has its own buffer, so no product waits for a score tile to be
+      // read: per tile j, dP(j+1) once warpgroup j has read dP(j), then dQ(j)
+      // once dS(j) is in, then S(j+2) into the buffer dQ(j) just read.
       bool ok = mbar_wait(&bars->res_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < 2 && j < n_items; ++j) {
         if (!(ok = wait_a(j))) break;
         tc_fence_after();
         issue_s(j);
       }
+      if (ok && n_items > 0 && (ok = wait_b(0))) {
+        tc_fence_after();
+        issue_dp(0);
+      }
       for (int j = 0; ok && j < n_items; ++j) {
         const int bb = j & 1;
-        if (!(ok = mbar_wait(&bars->s_read[bb], (j >> 1) & 1, abort_flag, p.status) && wait_b(j)))
-          break;
-        tc_fence_after();
-        issue_dp(j);
-        if (j >= 1) {
-          if (!(ok = mbar_wait(&bars->p_full[bb ^ 1], ((j - 1) >> 1) & 1, abort_flag, p.status)))
+        if (j + 1 < n_items) {
+          if (!(ok = mbar_wait(&bars->s_read[bb], (j >> 1) & 1, abort_flag, p.status) &&
+                     wait_b(j + 1)))
             break;
           tc_fence_after();
-          issue_dq(j - 1);
-          if (j + 1 < n_items) {
-            if (!(ok = wait_a(j + 1))) break;
-            tc_fence_after();
-            issue_s(j + 1);  // in order after dQ(j-1), which read this buffer
-          }
+          issue_dp(j + 1);  // warpgroup j has read dP(j)
         }
-      }
-      if (ok && n_items > 0 &&
-          (ok = mbar_wait(&bars->p_full[(n_items - 1) & 1], ((n_items - 1) >> 1) & 1, abort_flag,
-                          p.status))) {
+        if (!(ok = mbar_wait(&bars->p_full[bb], (j >> 1) & 1, abort_flag, p.status))) break;
         tc_fence_after();
-        issue_dq(n_items - 1);
+        issue_dq(j);
+        if (j + 2 < n_items) {
+          if (!(ok = wait_a(j + 2))) break;
+          tc_fence_after();
+          issue_s(j + 2);  // in order after dQ(j), which read this buffer
+        }
       }
       tc_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, p.status);
@@ -763,6 +771,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = row0 + r;  // query row; rows >= N have l2 = +inf, so P = 0
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tX = tmem + lane_off + col_x(wg);
+    const uint32_t tDP = tmem + lane_off + kColDP;
     const float c = p.scale_log2;
     const float l2s = p.l2[static_cast<size_t>(bh) * p.Npad + row];
     const float dds = p.dvec[static_cast<size_t>(bh) * p.Npad + row];
@@ -775,8 +784,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t sv[128];
       tmem_ld128(tX, sv);
       tmem_ld_wait128(sv);
-      tc_fence_before();
-      mbar_arrive(&bars->s_read[wg]);  // the tensor pipe may now write dP here
       const int kb0 = (js + j) * BT;     // first key of the tile
       uint32_t pk[64];
 #pragma unroll
@@ -800,15 +807,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ds[64];
       {
         uint32_t dp[64];
-        tmem_ld64(tX, dp);  // keys 0..63
+        tmem_ld64(tDP, dp);  // keys 0..63
         tmem_ld_wait64(dp);
         ds_cols(pk, dp, nullptr, dds, false, ds);
         ds_cols(pk + 16, dp + 32, nullptr, dds, false, ds + 16);
       }
       {
         uint32_t dp[64];
-        tmem_ld64(tX + 64, dp);  // keys 64..127
+        tmem_ld64(tDP + 64, dp);  // keys 64..127
         tmem_ld_wait64(dp);
+        tc_fence_before();
+        mbar_arrive(&bars->s_read[wg]);  // dP(j) is read: the buffer may take dP(j+1)
         ds_cols(pk + 32, dp, nullptr, dds, false, ds + 32);
         ds_cols(pk + 48, dp + 32, nullptr, dds, false, ds + 48);
       }
@@ -832,7 +841,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int cc = wg * (D / 64); cc < (wg + 1) * (D / 64); ++cc) {
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + kColAcc0 + cc * 32, v);
+          tmem_ld32(tmem + lane_off + kColDQ + cc * 32, v);
           tmem_ld_wait(v);
           uint32_t pkd[16];
 #pragma unroll
