@@ -143,3 +143,103 @@ def test_python_binding_rejects_cpu_tensors():
         ea.attn_fwd(q, q, q)
     with pytest.raises(TypeError):
         ea.attn_fwd(q.float(), q.float(), q.float())
+
+
+def dec_q8(lib, ws_bytes=None, **kw):
+    a = dict(q=A, kp=A, vp=A, ks=A, vs=A, fmt=0, bt=A, sl=A, o=A, lse=A, S=4, Hq=8, Hkv=2, d=128,
+             ps=16, maxb=8, npages=100, scale=0.1, ws=A)
+    a.update(kw)
+    need = lib.attn_decode_workspace_bytes(a["S"], a["Hq"], a["d"], a["maxb"], 16) or 1 << 20
+    return lib.attn_decode_paged_q8(a["q"], a["kp"], a["vp"], a["ks"], a["vs"], a["fmt"], a["bt"],
+                                    a["sl"], a["o"], a["lse"], a["S"], a["Hq"], a["Hkv"], a["d"],
+                                    a["ps"], a["maxb"], a["npages"], a["scale"], a["ws"],
+                                    need if ws_bytes is None else ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(ks=None), INVALID), (dict(vs=A + 2), INVALID),
+    (dict(fmt=2), INVALID), (dict(fmt=-1), INVALID), (dict(S=0), INVALID),
+    (dict(Hq=6, Hkv=4), INVALID), (dict(npages=0), INVALID), (dict(scale=float("nan")), INVALID),
+    (dict(d=96), UNSUPPORTED), (dict(ps=32), UNSUPPORTED),
+])
+def test_decode_q8_argument_checks(lib, kw, code):
+    assert dec_q8(lib, **kw) == code
+
+
+def test_decode_q8_rejects_small_workspace(lib):
+    assert dec_q8(lib, ws_bytes=64) == INVALID
+
+
+def test_decode_noalloc_argument_checks(lib):
+    def call(**kw):
+        a = dict(q=A, kp=A, vp=A, bt=A, sl=A, o=A, lse=A, S=4, Hq=8, Hkv=2, d=128, ps=16, maxb=8,
+                 npages=100, scale=0.1)
+        a.update(kw)
+        return lib.attn_decode_paged_noalloc(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["o"],
+                                             a["lse"], a["S"], a["Hq"], a["Hkv"], a["d"], a["ps"],
+                                             a["maxb"], a["npages"], a["scale"], None)
+    assert call(q=None) == INVALID
+    assert call(Hq=6, Hkv=4) == INVALID
+    assert call(d=80) == UNSUPPORTED
+    # More partials than the fixed scratch holds.
+    assert call(S=4096, Hq=64, maxb=4096) == INVALID
+
+
+def paged(lib, **kw):
+    a = dict(q=A, kp=A, vp=A, bt=A, sl=A, cu=A, o=A, lse=A, S=2, Hq=8, Hkv=2, T=64, maxq=32,
+             d=128, ps=16, maxb=8, npages=100, scale=0.1, window=0, slopes=None)
+    a.update(kw)
+    return lib.attn_prefill_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["cu"], a["o"],
+                                  a["lse"], a["S"], a["Hq"], a["Hkv"], a["T"], a["maxq"], a["d"],
+                                  a["ps"], a["maxb"], a["npages"], a["scale"], a["window"],
+                                  a["slopes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(cu=A + 2), INVALID), (dict(o=A + 8), INVALID),
+    (dict(slopes=A + 1), INVALID), (dict(S=0), INVALID), (dict(Hq=6, Hkv=4), INVALID),
+    (dict(T=-1), INVALID), (dict(maxq=-1), INVALID), (dict(window=-1), INVALID),
+    (dict(scale=0.0), INVALID), (dict(d=96), UNSUPPORTED), (dict(ps=32), UNSUPPORTED),
+])
+def test_prefill_paged_argument_checks(lib, kw, code):
+    assert paged(lib, **kw) == code
+
+
+def test_prefill_paged_empty_is_a_no_op(lib):
+    # Nothing to compute: no device is touched.
+    assert paged(lib, T=0) == 0
+    assert paged(lib, maxq=0) == 0
+
+
+def test_bwd_workspace_size(lib):
+    # L*log2(e) and D, each [B*Hq][N padded to 128] fp32, each 256-byte aligned.
+    n = lib.attn_bwd_workspace_bytes(2, 16, 1000)
+    rows = 2 * 16 * 1024
+    assert n == 2 * ((rows * 4 + 255) // 256 * 256)
+    assert lib.attn_bwd_workspace_bytes(0, 16, 1000) == 0
+    assert lib.attn_bwd_workspace_bytes(2, 16, 0) == 0
+
+
+def bwd(lib, ws_bytes=None, **kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, do=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=1, N=16, d=128,
+             scale=0.1, causal=0, window=0, slopes=None, ws=A)
+    a.update(kw)
+    need = lib.attn_bwd_workspace_bytes(a["B"], a["Hq"], max(a["N"], 1)) or 1 << 20
+    return lib.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"],
+                        a["dv"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["scale"], a["causal"],
+                        a["window"], a["slopes"], a["ws"], need if ws_bytes is None else ws_bytes,
+                        None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(do=None), INVALID), (dict(dk=A + 8), INVALID),
+    (dict(ws=A + 4), INVALID), (dict(window=8, causal=0), INVALID), (dict(window=-1), INVALID),
+    (dict(slopes=A + 2), INVALID), (dict(N=0), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(scale=-1.0), INVALID), (dict(d=96), UNSUPPORTED),
+])
+def test_bwd_argument_checks(lib, kw, code):
+    assert bwd(lib, **kw) == code
+
+
+def test_bwd_rejects_small_workspace(lib):
+    assert bwd(lib, ws_bytes=64) == INVALID
