@@ -580,6 +580,9 @@ def run_ours(args):
         timed_launches([dec], flush, 3)
         t, _ = timed_launches([dec], flush, args.component_reps)
         sec, mean_ms = component_time(t[0])
+        torch.cuda.synchronize()
+        if ea.decode_read_status(dec.ws) != 0:
+            raise RuntimeError("decode status word set in the decode component")
         gbs = dec.bytes / sec / 1e9
         comps["decode_paged_gqa"] = {"gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3, "ms_mean": mean_ms,
                                      "algorithmic_bytes": dec.bytes,
@@ -593,6 +596,9 @@ def run_ours(args):
             timed_launches([dq], flush, 3)
             t, _ = timed_launches([dq], flush, args.component_reps)
             sec, mean_ms = component_time(t[0])
+            torch.cuda.synchronize()
+            if ea.decode_read_status(dq.ws) != 0:
+                raise RuntimeError("decode status word set in the %s decode component" % fmt)
             gbs = dq.bytes / sec / 1e9
             comps["decode_paged_gqa_" + fmt] = {
                 "gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3, "ms_mean": mean_ms,
@@ -645,6 +651,8 @@ def run_only(args):
         it.launch()
     torch.cuda.synchronize()
     st = ea.device_status()
+    if hasattr(it, "ws") and isinstance(it, (Decode, DecodeQ8)):
+        st |= ea.decode_read_status(it.ws)
     print("ran %s x%d, device status %d" % (args.only, args.reps, st))
     return 0 if st == 0 else 1
 

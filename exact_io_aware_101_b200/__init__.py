@@ -9,6 +9,11 @@ or the device is not sm_100, calls raise.
     o, lse = attn_fwd(q, k, v, causal=True)                  # bf16 prefill
     o, lse = attn_fwd_f32(q, k, v)                           # fp32 prefill
     o, lse = attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens)
+
+Device-side failures (a corrupt block table, a bounded wait that ran out) are
+reported as ATTN_DEV_* bits: a decode given a ``workspace`` reports into that
+workspace (``decode_read_status``), every other call into the device's word
+(``device_status``).
 """
 from __future__ import annotations
 
@@ -23,7 +28,7 @@ __all__ = [
     "attn_decode_paged_q8", "KV_FORMATS", "decode_workspace_bytes", "attn_bwd",
     "attn_prefill_paged",
     "bwd_workspace_bytes", "DECODE_NOALLOC_SCRATCH_BYTES",
-    "device_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
+    "device_status", "decode_read_status", "status_string", "version", "library", "LIB_PATH", "EXPORTED_SYMBOLS",
     "ATTN_DEV_BAD_PAGE", "ATTN_DEV_TIMEOUT", "ATTN_DEV_LAYOUT", "AttnError",
 ]
 
@@ -32,7 +37,7 @@ EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ext", "attn_fwd_f32_ex
                     "attn_bwd_workspace_bytes", "attn_bwd", "attn_prefill_paged",
                     "attn_decode_workspace_bytes",
                     "attn_decode_paged", "attn_decode_paged_noalloc", "attn_decode_paged_q8",
-                    "attn_device_status",
+                    "attn_decode_read_status", "attn_device_status",
                     "attn_status_string", "attn_version")
 # Size of the library's fixed per-device scratch used by attn_decode_paged_noalloc.
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -53,50 +58,60 @@ class AttnError(RuntimeError):
         self.code = code
 
 
+def load_library(path: str) -> ctypes.CDLL:
+    """Load a build of the C ABI at ``path`` and declare every entry point's types."""
+    if not os.path.exists(path):
+        raise ImportError("%s is not built; run `python -m exact_io_aware_101_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    _declare(lib)
+    return lib
+
+
 def library() -> ctypes.CDLL:
     """Load libexattn.so (built by ``python -m exact_io_aware_101_b200.build``)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError("libexattn.so is not built (%s); run "
-                              "`python -m exact_io_aware_101_b200.build`" % LIB_PATH)
-        lib = ctypes.CDLL(LIB_PATH)
-        vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
-        lib.attn_fwd.restype = ci
-        lib.attn_fwd_f32.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
-        lib.attn_fwd_f32.restype = ci
-        lib.attn_fwd_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
-        lib.attn_fwd_ext.restype = ci
-        lib.attn_fwd_f32_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
-        lib.attn_fwd_f32_ext.restype = ci
-        lib.attn_prefill_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci,
-                                           ci, ci, ci, cf, ci, vp, vp]
-        lib.attn_prefill_paged.restype = ci
-        lib.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci]
-        lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
-        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
-                                 vp, vp, ctypes.c_size_t, vp]
-        lib.attn_bwd.restype = ci
-        lib.attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
-        lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
-        lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
-                                          cf, vp, ctypes.c_size_t, vp]
-        lib.attn_decode_paged.restype = ci
-        lib.attn_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
-                                                  ci, ci, cf, vp]
-        lib.attn_decode_paged_noalloc.restype = ci
-        lib.attn_decode_paged_q8.argtypes = [vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, ci, ci, ci,
-                                             ci, ci, ci, ci, cf, vp, ctypes.c_size_t, vp]
-        lib.attn_decode_paged_q8.restype = ci
-        lib.attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
-        lib.attn_device_status.restype = ci
-        lib.attn_status_string.argtypes = [ci]
-        lib.attn_status_string.restype = ctypes.c_char_p
-        lib.attn_version.argtypes = []
-        lib.attn_version.restype = ctypes.c_char_p
-        _lib = lib
+        _lib = load_library(LIB_PATH)
     return _lib
+
+
+def _declare(lib: ctypes.CDLL) -> None:
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+    lib.attn_fwd.restype = ci
+    lib.attn_fwd_f32.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+    lib.attn_fwd_f32.restype = ci
+    lib.attn_fwd_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
+    lib.attn_fwd_ext.restype = ci
+    lib.attn_fwd_f32_ext.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]
+    lib.attn_fwd_f32_ext.restype = ci
+    lib.attn_prefill_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci,
+                                       ci, ci, ci, cf, ci, vp, vp]
+    lib.attn_prefill_paged.restype = ci
+    lib.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci]
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
+                             vp, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd.restype = ci
+    lib.attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+    lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
+                                      cf, vp, ctypes.c_size_t, vp]
+    lib.attn_decode_paged.restype = ci
+    lib.attn_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
+                                              ci, ci, cf, vp]
+    lib.attn_decode_paged_noalloc.restype = ci
+    lib.attn_decode_paged_q8.argtypes = [vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, ci, ci, ci,
+                                         ci, ci, ci, ci, cf, vp, ctypes.c_size_t, vp]
+    lib.attn_decode_paged_q8.restype = ci
+    lib.attn_decode_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.attn_decode_read_status.restype = ci
+    lib.attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci, vp]
+    lib.attn_device_status.restype = ci
+    lib.attn_status_string.argtypes = [ci]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = ctypes.c_char_p
 
 
 def status_string(code: int) -> str:
@@ -154,12 +169,14 @@ def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype, window=0, alibi_
                 raise ValueError("alibi_slopes needs one value per query head")
             slopes_ptr = alibi_slopes.data_ptr()
         ext = getattr(library(), fn.__name__ + "_ext")
-        rc = ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                 B, Hq, Hkv, N, d, float(scale), int(bool(causal)), int(window), slopes_ptr,
-                 _stream(q))
+        with torch.cuda.device(q.device):
+            rc = ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     B, Hq, Hkv, N, d, float(scale), int(bool(causal)), int(window), slopes_ptr,
+                     _stream(q))
     else:
-        rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _stream(q))
+        with torch.cuda.device(q.device):
+            rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                    B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _stream(q))
     _raise(rc, what)
     return out, lse
 
@@ -217,11 +234,13 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, cu_q, max_q: 
         if alibi_slopes.numel() != Hq:
             raise ValueError("alibi_slopes needs one value per query head")
         slopes_ptr = alibi_slopes.data_ptr()
-    rc = library().attn_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
-                                      block_table.data_ptr(), seq_lens.data_ptr(), cu_q.data_ptr(),
-                                      out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, T, int(max_q), d,
-                                      page_size, block_table.shape[1], num_pages, float(scale),
-                                      int(window), slopes_ptr, _stream(q))
+    with torch.cuda.device(q.device):
+        rc = library().attn_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                          block_table.data_ptr(), seq_lens.data_ptr(),
+                                          cu_q.data_ptr(), out.data_ptr(), lse.data_ptr(), S, Hq,
+                                          Hkv, T, int(max_q), d, page_size, block_table.shape[1],
+                                          num_pages, float(scale), int(window), slopes_ptr,
+                                          _stream(q))
     _raise(rc, "attn_prefill_paged")
     return out, lse
 
@@ -269,16 +288,50 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, 1)
-    rc = library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq,
-                            Hkv, N, d, float(scale), int(bool(causal)), int(window), slopes_ptr,
-                            workspace.data_ptr(), workspace.numel(), _stream(q))
+    with torch.cuda.device(q.device):
+        rc = library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                dv.data_ptr(), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                                int(window), slopes_ptr, workspace.data_ptr(), workspace.numel(),
+                                _stream(q))
     _raise(rc, "attn_bwd")
     return dq, dk, dv
 
 
 def decode_workspace_bytes(S: int, Hq: int, d: int, max_blocks: int, page_size: int = 16) -> int:
     return int(library().attn_decode_workspace_bytes(S, Hq, d, max_blocks, page_size))
+
+
+def _decode_dims(q, k_pages, v_pages, block_table, seq_lens):
+    """Shapes of a paged decode's tensors, checked against one another before any
+    dtype or device check: the library gets no tensor sizes, so a block_table or
+    seq_lens with fewer than S rows would be read past its end on the device."""
+    for name, t, nd in (("q", q, 3), ("k_pages", k_pages, 4), ("v_pages", v_pages, 4),
+                        ("block_table", block_table, 2), ("seq_lens", seq_lens, 1)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError("%s must be a torch.Tensor" % name)
+        if t.dim() != nd:
+            raise ValueError("%s must have %d dims, got shape %s" % (name, nd, tuple(t.shape)))
+    S, Hq, d = q.shape
+    num_pages, Hkv, page_size, d2 = k_pages.shape
+    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("page pools must be [num_pages, Hkv, page_size, d] with q's d, and "
+                         "v_pages must match k_pages")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table/seq_lens must have S rows")
+    return S, Hq, d, num_pages, Hkv, page_size, block_table.shape[1]
+
+
+def _decode_outputs(q, S, Hq, out, lse):
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 3)
+    _check(lse, "lse", torch.float32, 2)
+    if tuple(out.shape) != tuple(q.shape) or tuple(lse.shape) != (S, Hq):
+        raise ValueError("out must be [S, Hq, d] and lse [S, Hq]")
+    return out, lse
 
 
 def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float | None = None,
@@ -288,37 +341,29 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float |
     q [S,Hq,d] bf16; k_pages/v_pages [num_pages,Hkv,page_size,d] bf16;
     block_table [S,max_blocks] int32; seq_lens [S] int32 (all on the GPU).
     Returns (O bf16 [S,Hq,d], L fp32 [S,Hq]).  ``workspace`` (uint8, at least
-    decode_workspace_bytes(...) bytes) is allocated when not given.
+    decode_workspace_bytes(...) bytes) is allocated when not given; pass one to
+    read the call's status afterwards with ``decode_read_status(workspace)``.
     """
+    S, Hq, d, num_pages, Hkv, page_size, max_blocks = _decode_dims(q, k_pages, v_pages,
+                                                                   block_table, seq_lens)
     _check(q, "q", torch.bfloat16, 3)
     _check(k_pages, "k_pages", torch.bfloat16, 4)
     _check(v_pages, "v_pages", torch.bfloat16, 4)
     _check(block_table, "block_table", torch.int32, 2)
     _check(seq_lens, "seq_lens", torch.int32, 1)
-    S, Hq, d = q.shape
-    num_pages, Hkv, page_size, d2 = k_pages.shape
-    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
-        raise ValueError("page pools must be [num_pages, Hkv, page_size, d]")
-    if block_table.shape[0] != S or seq_lens.shape[0] != S:
-        raise ValueError("block_table/seq_lens must have S rows")
-    max_blocks = block_table.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
-    _check(out, "out", torch.bfloat16, 3)
-    _check(lse, "lse", torch.float32, 2)
+    out, lse = _decode_outputs(q, S, Hq, out, lse)
     need = decode_workspace_bytes(S, Hq, d, max_blocks, page_size)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, 1)
-    rc = library().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
-                                     block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
-                                     lse.data_ptr(), S, Hq, Hkv, d, page_size, max_blocks,
-                                     num_pages, float(scale), workspace.data_ptr(),
-                                     workspace.numel(), _stream(q))
+    with torch.cuda.device(q.device):
+        rc = library().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                         block_table.data_ptr(), seq_lens.data_ptr(),
+                                         out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, page_size,
+                                         max_blocks, num_pages, float(scale), workspace.data_ptr(),
+                                         workspace.numel(), _stream(q))
     _raise(rc, "attn_decode_paged")
     return out, lse
 
@@ -331,13 +376,16 @@ def attn_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, block_table, s
     k_pages/v_pages [num_pages,Hkv,page_size,d]: E4M3 codes (torch.float8_e4m3fn,
     or their bytes as uint8) for kv_format "e4m3", torch.int8 for "int8";
     k_scales/v_scales [num_pages,Hkv] float32, one per (page, K/V head): the
-    element is scale * code.  Everything else as attn_decode_paged.
+    element is scale * code.  Everything else (the workspace and its status
+    word included) as attn_decode_paged.
     """
     if kv_format not in KV_FORMATS:
         raise ValueError("kv_format must be one of %s" % sorted(KV_FORMATS))
+    S, Hq, d, num_pages, Hkv, page_size, max_blocks = _decode_dims(q, k_pages, v_pages,
+                                                                   block_table, seq_lens)
     _check(q, "q", torch.bfloat16, 3)
     for name, t in (("k_pages", k_pages), ("v_pages", v_pages)):
-        if not isinstance(t, torch.Tensor) or t.dtype not in _KV_DTYPES[kv_format]:
+        if t.dtype not in _KV_DTYPES[kv_format]:
             raise TypeError("%s must be one of %s for kv_format %r"
                             % (name, _KV_DTYPES[kv_format], kv_format))
         _check(t, name, t.dtype, 4)
@@ -345,33 +393,23 @@ def attn_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, block_table, s
     _check(v_scales, "v_scales", torch.float32, 2)
     _check(block_table, "block_table", torch.int32, 2)
     _check(seq_lens, "seq_lens", torch.int32, 1)
-    S, Hq, d = q.shape
-    num_pages, Hkv, page_size, d2 = k_pages.shape
-    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
-        raise ValueError("page pools must be [num_pages, Hkv, page_size, d]")
     if tuple(k_scales.shape) != (num_pages, Hkv) or tuple(v_scales.shape) != (num_pages, Hkv):
         raise ValueError("scales must be [num_pages, Hkv]")
-    if block_table.shape[0] != S or seq_lens.shape[0] != S:
-        raise ValueError("block_table/seq_lens must have S rows")
-    max_blocks = block_table.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
-    _check(out, "out", torch.bfloat16, 3)
-    _check(lse, "lse", torch.float32, 2)
+    out, lse = _decode_outputs(q, S, Hq, out, lse)
     need = decode_workspace_bytes(S, Hq, d, max_blocks, page_size)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, 1)
-    rc = library().attn_decode_paged_q8(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
-                                        k_scales.data_ptr(), v_scales.data_ptr(),
-                                        KV_FORMATS[kv_format], block_table.data_ptr(),
-                                        seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), S,
-                                        Hq, Hkv, d, page_size, max_blocks, num_pages, float(scale),
-                                        workspace.data_ptr(), workspace.numel(), _stream(q))
+    with torch.cuda.device(q.device):
+        rc = library().attn_decode_paged_q8(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                            k_scales.data_ptr(), v_scales.data_ptr(),
+                                            KV_FORMATS[kv_format], block_table.data_ptr(),
+                                            seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), S,
+                                            Hq, Hkv, d, page_size, max_blocks, num_pages,
+                                            float(scale), workspace.data_ptr(), workspace.numel(),
+                                            _stream(q))
     _raise(rc, "attn_decode_paged_q8")
     return out, lse
 
@@ -385,33 +423,50 @@ def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens,
     allocator): the chunk partials live in the library's fixed per-device scratch
     (DECODE_NOALLOC_SCRATCH_BYTES), shared by every such call on the device, so
     calls that overlap on the GPU race.  Pass ``out`` and ``lse`` to avoid torch
-    allocating the outputs here.  Arguments as for attn_decode_paged.
+    allocating the outputs here.  Arguments as for attn_decode_paged; a bad page
+    id or length is reported in the device's word (``device_status``).
     """
+    S, Hq, d, num_pages, Hkv, page_size, max_blocks = _decode_dims(q, k_pages, v_pages,
+                                                                   block_table, seq_lens)
     _check(q, "q", torch.bfloat16, 3)
     _check(k_pages, "k_pages", torch.bfloat16, 4)
     _check(v_pages, "v_pages", torch.bfloat16, 4)
     _check(block_table, "block_table", torch.int32, 2)
     _check(seq_lens, "seq_lens", torch.int32, 1)
-    S, Hq, d = q.shape
-    num_pages, Hkv, page_size, _ = k_pages.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
-    _check(out, "out", torch.bfloat16, 3)
-    _check(lse, "lse", torch.float32, 2)
-    rc = library().attn_decode_paged_noalloc(
-        q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
-        seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, page_size,
-        block_table.shape[1], num_pages, float(scale), _stream(q))
+    out, lse = _decode_outputs(q, S, Hq, out, lse)
+    with torch.cuda.device(q.device):
+        rc = library().attn_decode_paged_noalloc(
+            q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+            seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, page_size,
+            max_blocks, num_pages, float(scale), _stream(q))
     _raise(rc, "attn_decode_paged_noalloc")
     return out, lse
 
 
-def device_status(clear: bool = False) -> int:
-    """Status bits (ATTN_DEV_*) raised by kernels on the current device; syncs the device."""
+def decode_read_status(workspace: torch.Tensor) -> int:
+    """ATTN_DEV_* bits of the last workspace decode that used ``workspace`` (0: none).
+
+    Synchronises nothing: first synchronise the stream the decode ran on (or an
+    event recorded after it)."""
+    _check(workspace, "workspace", torch.uint8, 1)
     st = ctypes.c_uint(0)
-    _raise(library().attn_device_status(ctypes.byref(st), int(bool(clear))), "attn_device_status")
+    with torch.cuda.device(workspace.device):
+        rc = library().attn_decode_read_status(workspace.data_ptr(), ctypes.byref(st))
+    _raise(rc, "attn_decode_read_status")
+    return int(st.value)
+
+
+def device_status(clear: bool = False, device=None) -> int:
+    """Status bits (ATTN_DEV_*) that calls without a decode workspace raised on a device.
+
+    Waits for the work enqueued so far on that device's current stream (and only
+    for it)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_uint(0)
+    with torch.cuda.device(dev):
+        rc = library().attn_device_status(ctypes.byref(st), int(bool(clear)),
+                                          torch.cuda.current_stream(dev).cuda_stream)
+    _raise(rc, "attn_device_status")
     return int(st.value)

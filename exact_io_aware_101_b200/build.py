@@ -3,19 +3,32 @@
 Usage: ``python -m exact_io_aware_101_b200.build [--force] [--verbose]``.
 The library links the CUDA runtime statically and reaches the driver's tensor
 map encoder through cudaGetDriverEntryPoint, so it needs only the NVIDIA
-driver at run time.
+driver at run time.  Each kernel file compiles to its own object (in parallel,
+in a temporary directory), then one link makes the library.
+
+``build_test_lib()`` makes a second library, used only by tests: the same
+sources with every wait limited to TEST_WAIT_CYCLES instead of about 1.5 s,
+with the producers of the prefill and decode kernels stopping before ring index
+TEST_WITHHOLD (so that the kernels' waits run out on purpose and their abort
+paths run), and with the probes of csrc/testbuild_probes.cu (device functions
+evaluated on their own).  The product library is never built with these
+switches.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import glob
 import os
 import subprocess
 import sys
+import tempfile
 
 HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libexattn.so")
-INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+TEST_LIB = os.path.join(HERE, "libexattn_testbuild.so")
+INCLUDE = os.path.join(ROOT, "include")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -23,6 +36,12 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--expt-relaxed-constexpr",
 ]
+# The test build: ~1 ms waits, producers stop before ring index 2 (the
+# prefill's second K tile; the decode's third page of a chunk), probes compiled.
+TEST_WAIT_CYCLES = 2000000
+TEST_WITHHOLD = 2
+TEST_FLAGS = ["-DEXATTN_WAIT_LIMIT_CYCLES=%dLL" % TEST_WAIT_CYCLES,
+              "-DEXATTN_TEST_WITHHOLD=%d" % TEST_WITHHOLD, "-DEXATTN_TEST_BUILD=1"]
 
 
 def _sources():
@@ -41,22 +60,55 @@ def nvcc() -> str:
     return "nvcc"
 
 
+def _up_to_date(target: str) -> bool:
+    if not os.path.exists(target):
+        return False
+    t = os.path.getmtime(target)
+    return all(os.path.getmtime(p) <= t for p in _deps())
+
+
+def _link(target: str, flags, verbose: bool) -> str:
+    with tempfile.TemporaryDirectory(prefix="exattn_build_") as objdir:
+        return _compile_and_link(target, flags, objdir, verbose)
+
+
+def _compile_and_link(target: str, flags, objdir: str, verbose: bool) -> str:
+    base = [nvcc()] + NVCC_FLAGS + list(flags)
+    if verbose:
+        base.insert(1, "-Xptxas=-v")
+
+    def compile_one(src):
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+        cmd = base + ["-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.check_call(cmd)
+        return obj
+
+    workers = max(1, min(len(_sources()), os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(workers) as ex:
+        objs = list(ex.map(compile_one, _sources()))
+    tmp = target + ".tmp%d" % os.getpid()
+    subprocess.check_call([nvcc()] + NVCC_FLAGS[:2] + ["-shared", "-o", tmp] + objs)
+    os.replace(tmp, target)
+    return target
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     """Compile every kernel file and the C ABI into libexattn.so; returns its path."""
-    if not force and os.path.exists(LIB):
-        t = os.path.getmtime(LIB)
-        if all(os.path.getmtime(p) <= t for p in _deps()):
-            return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc()] + NVCC_FLAGS + list(extra) + ["-shared", "-o", tmp] + _sources()
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    if not force and not extra and _up_to_date(LIB):
+        return LIB
+    return _link(LIB, extra, verbose)
+
+
+def build_test_lib(force: bool = False, verbose: bool = False) -> str:
+    """The test build of the library (see the module docstring); returns its path."""
+    if not force and _up_to_date(TEST_LIB):
+        return TEST_LIB
+    return _link(TEST_LIB, TEST_FLAGS, verbose)
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    force, verbose = "--force" in sys.argv, "--verbose" in sys.argv
+    print(build(force=force, verbose=verbose))
+    print(build_test_lib(force=force, verbose=verbose))

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/exattn.h: argument checks, device
-// checks and the per-device status word, then a launch of the right kernel.
-// Nothing here allocates, frees or synchronises (except attn_device_status).
+// checks and the status words, then a launch of the right kernel.  Nothing here
+// allocates or frees; only the two status reads wait, each for the one copy (or
+// the one stream) it reads through.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -13,7 +14,9 @@
 namespace exattn {
 namespace {
 
-// Status bits raised by kernels on this device (ATTN_DEV_*).
+// Status bits raised by the prefill, chunked-prefill and backward kernels (and
+// the workspace-free decode) on this device (ATTN_DEV_*).  The decodes that take
+// a workspace report into a word of that workspace instead.
 __device__ unsigned g_status = 0;
 
 constexpr int kMaxDevices = 64;
@@ -23,6 +26,7 @@ int g_is_sm100[kMaxDevices] = {};  // 0 unknown, 1 yes, -1 no
 
 // Device address of this device's status word, looked up once per device
 // (a __device__ variable's address is only meaningful on the device side).
+// The cache assumes the device is not reset while the library is loaded.
 bool device_state(unsigned **status, bool *sm100) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
@@ -187,9 +191,10 @@ attn_status_t attn_decode_paged(const void *q, const void *k_pages, const void *
   bool sm100 = false;
   if (!device_state(&status, &sm100)) return ATTN_ERR_CUDA;
   if (!sm100) return ATTN_ERR_UNSUPPORTED;
+  // The call's status goes to its own workspace word only.
   return launch_decode_paged(q, k_pages, v_pages, block_table, seq_lens, o, lse, S, Hq, Hkv, d,
                              max_blocks, num_pages, scale, workspace,
-                             reinterpret_cast<cudaStream_t>(stream), status);
+                             reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 attn_status_t attn_decode_paged_q8(const void *q, const void *k_pages, const void *v_pages,
@@ -216,7 +221,7 @@ attn_status_t attn_decode_paged_q8(const void *q, const void *k_pages, const voi
   if (!sm100) return ATTN_ERR_UNSUPPORTED;
   return launch_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, kv_format, block_table,
                                 seq_lens, o, lse, S, Hq, Hkv, d, max_blocks, num_pages, scale,
-                                workspace, reinterpret_cast<cudaStream_t>(stream), status);
+                                workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // The workspace-free decode: same checks and kernels as attn_decode_paged, with
@@ -243,21 +248,45 @@ attn_status_t attn_decode_paged_noalloc(const void *q, const void *k_pages, cons
   void *scratch = nullptr;
   attn_status_t st = noalloc_scratch_address(&scratch);
   if (st != ATTN_OK) return st;
+  // The scratch is shared, so its status word belongs to no caller: the bits
+  // also go to the per-device word that attn_device_status reads.
   return launch_decode_paged(q, k_pages, v_pages, block_table, seq_lens, o, lse, S, Hq, Hkv, d,
                              max_blocks, num_pages, scale, scratch,
                              reinterpret_cast<cudaStream_t>(stream), status);
 }
 
-attn_status_t attn_device_status(unsigned *status, int clear) {
+attn_status_t attn_decode_read_status(const void *workspace, unsigned *dev_status) {
+  if (!aligned16(workspace) || !dev_status) return ATTN_ERR_INVALID_ARG;
+  // One 4-byte copy through this thread's own default stream: it waits for
+  // nothing the caller enqueued on other streams (the caller has synchronised
+  // the decode's stream already).  cudaMemcpyDefault lets the workspace live
+  // on any device.
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(unsigned), cudaMemcpyDefault,
+                      cudaStreamPerThread) != cudaSuccess ||
+      cudaStreamSynchronize(cudaStreamPerThread) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  *dev_status = word;
+  return ATTN_OK;
+}
+
+attn_status_t attn_device_status(unsigned *status, int clear, attn_stream_t stream) {
   if (!status) return ATTN_ERR_INVALID_ARG;
   unsigned *dev_ptr = nullptr;
   bool sm100 = false;
   if (!device_state(&dev_ptr, &sm100)) return ATTN_ERR_CUDA;
-  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
-  if (cudaMemcpy(status, dev_ptr, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+  // Everything enqueued on `stream` before this call finishes first (the copy is
+  // ordered behind it); other streams are not waited for.
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, dev_ptr, sizeof(unsigned), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  if (clear && cudaMemset(dev_ptr, 0, sizeof(unsigned)) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (clear && cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (clear && (cudaMemsetAsync(dev_ptr, 0, sizeof(unsigned), st) != cudaSuccess ||
+                cudaStreamSynchronize(st) != cudaSuccess))
+    return ATTN_ERR_CUDA;
+  *status = word;
   return ATTN_OK;
 }
 

@@ -4,8 +4,8 @@
 // mbarriers with bounded waits, TMA tile loads (no multicast anywhere), and the
 // tcgen05 tensor-memory instructions (alloc/dealloc, mma, commit, ld/st,
 // fences).  Every wait in this library is bounded: after kWaitLimitCycles it
-// gives up, raises the abort flag of its CTA and the device status word, and
-// lets the caller unwind without trapping.
+// gives up, raises the abort flag of its CTA and ATTN_DEV_TIMEOUT in the status
+// word it was given, and lets the caller unwind without trapping.
 #pragma once
 
 #include <cuda.h>
@@ -17,8 +17,13 @@
 
 namespace exattn {
 
-// ~1.5 s at 1.9 GHz: far above any legitimate wait inside one kernel.
-constexpr long long kWaitLimitCycles = 3000000000LL;
+// ~1.5 s at 1.9 GHz: far above any legitimate wait inside one kernel.  A
+// separate test build of the library shortens it (EXATTN_WAIT_LIMIT_CYCLES) so
+// that a test can make a wait run out quickly; the product build never sets it.
+#ifndef EXATTN_WAIT_LIMIT_CYCLES
+#define EXATTN_WAIT_LIMIT_CYCLES 3000000000LL
+#endif
+constexpr long long kWaitLimitCycles = EXATTN_WAIT_LIMIT_CYCLES;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,7 +68,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed.  Returns false if
 // the CTA's abort flag is raised or the wait runs out (which raises it, and sets
-// ATTN_DEV_TIMEOUT in the device status word).
+// ATTN_DEV_TIMEOUT in *status: a global status word, or a word in the CTA's
+// shared memory that the kernel reports later).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           unsigned *status) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -360,6 +366,19 @@ __device__ __forceinline__ void grid_dependency_wait() {
 }
 __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// A split-decode chunk that failed (a bad page id or length, or a wait that ran
+// out) stores, instead of its log2-sum-exp, a quiet NaN whose low byte holds
+// its ATTN_DEV_* bits and whose upper 24 bits are the tag 0x7fe500.  The
+// combine kernel turns the NaN into NaN outputs and the bits into the call's
+// status word.  A NaN that arithmetic produced carries no tag, hence no bits.
+__device__ __forceinline__ float failed_partial(unsigned bits) {
+  return __uint_as_float(0x7fe50000u | (bits & 0xffu));
+}
+__device__ __forceinline__ unsigned failed_partial_bits(float x) {
+  const unsigned u = __float_as_uint(x);
+  return (u & 0xffffff00u) == 0x7fe50000u ? (u & 0xffu) : 0u;
 }
 
 // Round two floats to bf16 (nearest-even) and pack: lo in bits [0,16).

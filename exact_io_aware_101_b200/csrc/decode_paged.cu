@@ -20,6 +20,10 @@
 //  * combine kernel: per (sequence, head), merges the chunks' partials with
 //    weights 2^(L_r - L) -- the same rescaling rule applied across chunks --
 //    and writes O (bf16) and L (natural log, float32).
+//  * status: each call owns the status word at the start of its workspace.
+//    The split grid's first CTA clears it; a chunk that fails records its
+//    ATTN_DEV_* bits in its partial (failed_partial); the combine kernel, which
+//    starts only once the whole split grid is done, ORs them into the word.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -66,8 +70,10 @@ struct DecCfg {
   static constexpr int SMEM = NST * STAGE;
 };
 
-// Workspace: o_part [S][Hq][nsplit][D] f32 (normalised), l2_part [S][Hq][nsplit]
-// f32 (log2-sum-exp of scale*log2(e)*scores over the chunk; NaN marks a bad sequence).
+// Workspace (decode_ws_layout): the call's status word, then o_part
+// [S][Hq][nsplit][D] f32 (normalised) and l2_part [S][Hq][nsplit] f32
+// (log2-sum-exp of scale*log2(e)*scores over the chunk; a tagged NaN marks a
+// failed chunk).
 template <int D, int GB, int HC>
 __global__ void __launch_bounds__((HC + 1) * 32)
     decode_split_kernel(const __nv_bfloat16 *__restrict__ q,
@@ -76,7 +82,10 @@ __global__ void __launch_bounds__((HC + 1) * 32)
                         const int *__restrict__ block_table, const int *__restrict__ seq_lens,
                         float *__restrict__ o_part, float *__restrict__ l2_part, int Hq, int Hkv,
                         int max_blocks, int num_pages, float scale_log2, int nsplit,
-                        int head_chunks, unsigned *status) {
+                        int head_chunks, unsigned *call_status) {
+  // The call's status word starts clear; only the combine kernel, which waits
+  // for this whole grid, sets bits in it.
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *call_status = 0;
   grid_dependents_launch();  // the combine kernel may be scheduled behind this grid
   using C = DecCfg<HC, D>;
   constexpr int LPT = D / 8;           // lanes per token row (8 bf16 = 16 B each)
@@ -105,6 +114,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
   __shared__ int stage_ntok[C::NST];
   __shared__ int sm_pid[kPagesPerSplit];
   __shared__ int sm_bad, sm_abort;
+  __shared__ unsigned sm_status;  // ATTN_DEV_* bits of this CTA's bounded waits
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(&full[i], 1);
@@ -112,6 +122,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     }
     sm_bad = bad_len ? 1 : 0;
     sm_abort = 0;
+    sm_status = 0;
     fence_mbar_init();
   }
   if (warp == HC && lane < npg)
@@ -124,8 +135,13 @@ __global__ void __launch_bounds__((HC + 1) * 32)
       int issued = 0;
       for (int i = 0; i < npg; ++i) {
         const int st = i % C::NST;
-        if (i >= C::NST && !mbar_wait(&empty[st], ((i / C::NST) - 1) & 1, &sm_abort, status))
+        if (i >= C::NST && !mbar_wait(&empty[st], ((i / C::NST) - 1) & 1, &sm_abort, &sm_status))
           break;
+#ifdef EXATTN_TEST_WITHHOLD
+        // Test build only: stop before page EXATTN_TEST_WITHHOLD, arriving on
+        // nothing and copying nothing, so the compute warps' wait runs out.
+        if (i == EXATTN_TEST_WITHHOLD) break;
+#endif
         const int pid = sm_pid[i];
         if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
           sm_bad = 1;
@@ -145,7 +161,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
       }
       // Let every copy land before the CTA (and its shared memory) goes away.
       for (int i = max(0, issued - C::NST); i < issued; ++i)
-        mbar_wait_drain(&full[i % C::NST], (i / C::NST) & 1, status);
+        mbar_wait_drain(&full[i % C::NST], (i / C::NST) & 1, &sm_status);
     }
   } else {
     // ------------------------------------------------------------ compute
@@ -184,7 +200,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
 
     for (int i = 0; i < npg; ++i) {
       const int st = i % C::NST;
-      bool ok = mbar_wait(&full[st], (i / C::NST) & 1, &sm_abort, status);
+      bool ok = mbar_wait(&full[st], (i / C::NST) & 1, &sm_abort, &sm_status);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int ntok = stage_ntok[st];
       if (ntok > 0) {
@@ -287,9 +303,13 @@ __global__ void __launch_bounds__((HC + 1) * 32)
         }
     }
     // The warp's partial is the chunk's for its heads: normalise and write.
-    // sm_bad / sm_abort are final once every page has been consumed.
+    // sm_bad / sm_abort are final once every page has been consumed (or the
+    // warp gave up); a failed chunk's partial carries its status bits.
     const bool bad = *reinterpret_cast<volatile int *>(&sm_bad) != 0 ||
                      *reinterpret_cast<volatile int *>(&sm_abort) != 0;
+    unsigned bits = *reinterpret_cast<volatile unsigned *>(&sm_status) |
+                    (*reinterpret_cast<volatile int *>(&sm_bad) ? ATTN_DEV_BAD_PAGE : 0u);
+    if (bad && bits == 0) bits = ATTN_DEV_TIMEOUT;  // aborted by a wait that timed out
 #pragma unroll
     for (int hh = 0; hh < GB; ++hh) {
       const float mh = __shfl_sync(0xffffffffu, m, hh * (LPT / GB));
@@ -305,11 +325,9 @@ __global__ void __launch_bounds__((HC + 1) * 32)
                      : make_float4(acc[hh][2].x * inv, acc[hh][2].y * inv, acc[hh][3].x * inv,
                                    acc[hh][3].y * inv);
       }
-      if (lane == 0) l2_part[slot] = bad ? NAN : mh + log2f(lh);
+      if (lane == 0) l2_part[slot] = bad ? failed_partial(bits) : mh + log2f(lh);
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
 }
 
 // One warp per (sequence, head): merge the chunk partials.  The lanes read the
@@ -318,13 +336,16 @@ __global__ void __launch_bounds__((HC + 1) * 32)
 // rows are then summed eight chunks at a time with their loads issued
 // together.  Launched as a programmatic dependent of the split kernel: it may
 // start while the split kernel's last CTAs run, and waits for that grid to
-// finish (and its writes to be visible) before it reads a partial.
+// finish (and its writes to be visible) before it reads a partial.  A failed
+// sequence (a bad length, or a chunk whose partial is a tagged NaN) gets NaN
+// outputs and its bits are ORed into the call's status word (and into
+// dev_status when that is given).
 template <int D>
 __global__ void __launch_bounds__(128)
     decode_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ l2_part,
                           const int *__restrict__ seq_lens, __nv_bfloat16 *__restrict__ o,
                           float *__restrict__ lse, int S, int Hq, int max_blocks, int nsplit,
-                          int pages_per_split) {
+                          int pages_per_split, unsigned *call_status, unsigned *dev_status) {
   constexpr int DPL = D / 32;
   constexpr int kBatch = 8;
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -346,19 +367,30 @@ __global__ void __launch_bounds__(128)
       bad_len ? 0 : ((len + kPageSize - 1) / kPageSize + pages_per_split - 1) / pages_per_split;
   const float *lp = l2_part + head * nsplit;
   bool bad = bad_len;
+  unsigned bits = bad_len ? ATTN_DEV_BAD_PAGE : 0u;
   float M = -INFINITY;
   for (int r = lane; r < nparts; r += 32) {
     const float x = lp[r];
-    bad |= isnan(x);
+    if (isnan(x)) {
+      bad = true;
+      bits |= failed_partial_bits(x);
+    }
     M = fmaxf(M, x);
   }
   bad = __any_sync(0xffffffffu, bad);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   if (bad) {
+    bits = __reduce_or_sync(0xffffffffu, bits);
 #pragma unroll
     for (int e = 0; e < DPL; ++e) orow[lane + 32 * e] = __float2bfloat16_rn(NAN);
-    if (lane == 0) lse[head] = NAN;
+    if (lane == 0) {
+      lse[head] = NAN;
+      if (bits) {
+        atomicOr(call_status, bits);
+        if (dev_status) atomicOr(dev_status, bits);
+      }
+    }
     return;
   }
   float acc[DPL];
@@ -470,27 +502,35 @@ attn_status_t noalloc_scratch_address(void **addr) {
 
 int decode_max_splits(int max_blocks) { return (max_blocks + kPagesPerSplit - 1) / kPagesPerSplit; }
 
+// [status block | o_part (256-byte padded) | l2_part (256-byte padded)].
 size_t decode_workspace_bytes(int S, int Hq, int d, int max_blocks) {
   const size_t parts = static_cast<size_t>(S) * Hq * decode_max_splits(max_blocks);
   const size_t o_bytes = (parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
-  return o_bytes + ((parts * sizeof(float) + 255) & ~static_cast<size_t>(255));
+  return kDecodeStatusBytes + o_bytes + ((parts * sizeof(float) + 255) & ~static_cast<size_t>(255));
+}
+
+DecodeWs decode_ws_layout(void *workspace, int S, int Hq, int d, int max_blocks) {
+  const size_t parts = static_cast<size_t>(S) * Hq * decode_max_splits(max_blocks);
+  uint8_t *base = static_cast<uint8_t *>(workspace);
+  DecodeWs ws;
+  ws.status = reinterpret_cast<unsigned *>(base);
+  ws.o_part = reinterpret_cast<float *>(base + kDecodeStatusBytes);
+  ws.l2_part = reinterpret_cast<float *>(
+      base + kDecodeStatusBytes + ((parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+  return ws;
 }
 
 attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void *v_pages,
                                   const int *block_table, const int *seq_lens, void *o, float *lse,
                                   int S, int Hq, int Hkv, int d, int max_blocks, int num_pages,
                                   float scale, void *workspace, cudaStream_t stream,
-                                  unsigned *status) {
+                                  unsigned *dev_status) {
   const int G = Hq / Hkv;
   const int GB = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
   const int head_chunks = G / GB;
   const int HC = (Hkv % 8 == 0) ? 8 : (Hkv % 4 == 0) ? 4 : (Hkv % 2 == 0) ? 2 : 1;
   const int nsplit = decode_max_splits(max_blocks);
-  const size_t parts = static_cast<size_t>(S) * Hq * nsplit;
-  float *o_part = static_cast<float *>(workspace);
-  float *l2_part = reinterpret_cast<float *>(
-      static_cast<uint8_t *>(workspace) +
-      ((parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+  const DecodeWs ws = decode_ws_layout(workspace, S, Hq, d, max_blocks);
   if (static_cast<long long>(Hkv / HC) * head_chunks > 65535 || S > 65535)
     return ATTN_ERR_UNSUPPORTED;
   dim3 grid(nsplit, S, (Hkv / HC) * head_chunks);
@@ -498,22 +538,23 @@ attn_status_t launch_decode_paged(const void *q, const void *k_pages, const void
   bool ok;
   if (d == 128)
     ok = dispatch_split<128>(HC, GB, grid, stream, q, k_pages, v_pages, block_table, seq_lens,
-                             o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit,
-                             head_chunks, status);
+                             ws.o_part, ws.l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit,
+                             head_chunks, ws.status);
   else if (d == 64)
     ok = dispatch_split<64>(HC, GB, grid, stream, q, k_pages, v_pages, block_table, seq_lens,
-                            o_part, l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit,
-                            head_chunks, status);
+                            ws.o_part, ws.l2_part, Hq, Hkv, max_blocks, num_pages, sl2, nsplit,
+                            head_chunks, ws.status);
   else
     return ATTN_ERR_UNSUPPORTED;
   if (!ok) return ATTN_ERR_UNSUPPORTED;
-  return launch_decode_combine(o_part, l2_part, seq_lens, o, lse, S, Hq, d, max_blocks, nsplit,
-                               kPagesPerSplit, stream);
+  return launch_decode_combine(ws, seq_lens, o, lse, S, Hq, d, max_blocks, nsplit,
+                               kPagesPerSplit, stream, dev_status);
 }
 
-attn_status_t launch_decode_combine(const float *o_part, const float *l2_part, const int *seq_lens,
-                                    void *o, float *lse, int S, int Hq, int d, int max_blocks,
-                                    int nsplit, int pages_per_split, cudaStream_t stream) {
+attn_status_t launch_decode_combine(const DecodeWs &ws, const int *seq_lens, void *o, float *lse,
+                                    int S, int Hq, int d, int max_blocks, int nsplit,
+                                    int pages_per_split, cudaStream_t stream,
+                                    unsigned *dev_status) {
   const int heads = S * Hq;
   const int blocks = (heads + 3) / 4;
   // Programmatic dependent launch: the grid may be scheduled while the split
@@ -531,11 +572,13 @@ attn_status_t launch_decode_combine(const float *o_part, const float *l2_part, c
   __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
   cudaError_t err;
   if (d == 128)
-    err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, o_part, l2_part, seq_lens, ob, lse,
-                             S, Hq, max_blocks, nsplit, pages_per_split);
+    err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, ws.o_part, ws.l2_part, seq_lens,
+                             ob, lse, S, Hq, max_blocks, nsplit, pages_per_split, ws.status,
+                             dev_status);
   else if (d == 64)
-    err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, o_part, l2_part, seq_lens, ob, lse,
-                             S, Hq, max_blocks, nsplit, pages_per_split);
+    err = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, ws.o_part, ws.l2_part, seq_lens,
+                             ob, lse, S, Hq, max_blocks, nsplit, pages_per_split, ws.status,
+                             dev_status);
   else
     return ATTN_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return ATTN_ERR_CUDA;

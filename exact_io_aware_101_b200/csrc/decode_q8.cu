@@ -165,9 +165,10 @@ __device__ __forceinline__ VRow<D> load_vrow(const uint8_t *tile, int row, int g
   return r;
 }
 
-// Workspace and partial layout as in decode_paged.cu: o_part [S][Hq][nsplit][D]
-// f32 (normalised), l2_part [S][Hq][nsplit] f32 (log2-sum-exp; NaN marks a bad
-// sequence).
+// Workspace and partial layout as in decode_paged.cu (decode_ws_layout): the
+// call's status word, o_part [S][Hq][nsplit][D] f32 (normalised), l2_part
+// [S][Hq][nsplit] f32 (log2-sum-exp; a tagged NaN marks a failed chunk and
+// carries its status bits, which the combine kernel reports).
 //
 // One CTA per (chunk of kPagesPerSplitQ8 pages, sequence, group of HC K/V
 // heads, chunk of GB query heads per K/V head).  Warp HC is the producer: its
@@ -195,7 +196,10 @@ __global__ void __launch_bounds__((HC + 1) * 32)
                            const int *__restrict__ block_table, const int *__restrict__ seq_lens,
                            float *__restrict__ o_part, float *__restrict__ l2_part, int Hq,
                            int Hkv, int max_blocks, int num_pages, float scale_log2, int nsplit,
-                           int head_chunks, unsigned *status) {
+                           int head_chunks, unsigned *call_status) {
+  // The call's status word starts clear; only the combine kernel, which waits
+  // for this whole grid, sets bits in it.
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *call_status = 0;
   grid_dependents_launch();  // the combine kernel may be scheduled behind this grid
   using C = Q8Cfg<HC, D>;
   constexpr int KS = D / 16;   // k-steps of the q.k MMA = M-tiles of the p.v MMA
@@ -225,6 +229,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
   __shared__ int stage_ntok[C::NST];
   __shared__ int sm_pid[kPagesPerSplitQ8];
   __shared__ int sm_bad, sm_abort;
+  __shared__ unsigned sm_status;  // ATTN_DEV_* bits of this CTA's bounded waits
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(&full[i], 1);
@@ -232,6 +237,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     }
     sm_bad = bad_len ? 1 : 0;
     sm_abort = 0;
+    sm_status = 0;
     fence_mbar_init();
   }
   if (warp == HC && lane < npg)
@@ -244,8 +250,13 @@ __global__ void __launch_bounds__((HC + 1) * 32)
       int issued = 0;
       for (int i = 0; i < npg; ++i) {
         const int st = i % C::NST;
-        if (i >= C::NST && !mbar_wait(&empty[st], ((i / C::NST) - 1) & 1, &sm_abort, status))
+        if (i >= C::NST && !mbar_wait(&empty[st], ((i / C::NST) - 1) & 1, &sm_abort, &sm_status))
           break;
+#ifdef EXATTN_TEST_WITHHOLD
+        // Test build only: stop before page EXATTN_TEST_WITHHOLD, arriving on
+        // nothing and copying nothing, so the compute warps' wait runs out.
+        if (i == EXATTN_TEST_WITHHOLD) break;
+#endif
         const int pid = sm_pid[i];
         if (pid < 0 || pid >= num_pages) {  // never dereference a bad page id
           sm_bad = 1;
@@ -263,7 +274,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
       }
       // Let every copy land before the CTA (and its shared memory) goes away.
       for (int i = max(0, issued - C::NST); i < issued; ++i)
-        mbar_wait_drain(&full[i % C::NST], (i / C::NST) & 1, status);
+        mbar_wait_drain(&full[i % C::NST], (i / C::NST) & 1, &sm_status);
     }
   } else {
     // ------------------------------------------------------------ compute
@@ -387,8 +398,8 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     for (int i = 0; i < npg; i += 2) {
       const bool two = i + 1 < npg;
       const int sta = i % C::NST, stb = (i + 1) % C::NST;
-      bool ok = mbar_wait(&full[sta], (i / C::NST) & 1, &sm_abort, status);
-      if (two) ok = ok && mbar_wait(&full[stb], ((i + 1) / C::NST) & 1, &sm_abort, status);
+      bool ok = mbar_wait(&full[sta], (i / C::NST) & 1, &sm_abort, &sm_status);
+      if (two) ok = ok && mbar_wait(&full[stb], ((i + 1) / C::NST) & 1, &sm_abort, &sm_status);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int na = stage_ntok[sta];
       const int nb = two ? stage_ntok[stb] : 0;
@@ -489,6 +500,9 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     __syncwarp();
     const bool bad = *reinterpret_cast<volatile int *>(&sm_bad) != 0 ||
                      *reinterpret_cast<volatile int *>(&sm_abort) != 0;
+    unsigned bits = *reinterpret_cast<volatile unsigned *>(&sm_status) |
+                    (*reinterpret_cast<volatile int *>(&sm_bad) ? ATTN_DEV_BAD_PAGE : 0u);
+    if (bad && bits == 0) bits = ATTN_DEV_TIMEOUT;  // aborted by a wait that timed out
     // O = acc * 2^(mv - m) / l.
     const float inv0 = (mv0 == -INFINITY ? 0.f : ex2(mv0 - m0)) / l0;
     const float inv1 = (mv1 == -INFINITY ? 0.f : ex2(mv1 - m1)) / l1;
@@ -506,12 +520,10 @@ __global__ void __launch_bounds__((HC + 1) * 32)
             bad ? make_float2(NAN, NAN) : make_float2(acc[i][1] * inv1, acc[i][3] * inv1);
     }
     if (g == 0) {
-      if (hA < GB) l2_part[slotA] = bad ? NAN : m0 + log2f(l0);
-      if (hB < GB) l2_part[slotB] = bad ? NAN : m1 + log2f(l1);
+      if (hA < GB) l2_part[slotA] = bad ? failed_partial(bits) : m0 + log2f(l0);
+      if (hB < GB) l2_part[slotB] = bad ? failed_partial(bits) : m1 + log2f(l1);
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0 && sm_bad) atomicOr(status, ATTN_DEV_BAD_PAGE);
 }
 
 // Page pool [num_pages][Hkv][16][D] bytes as a 3-D tensor (D, 16, num_pages*Hkv);
@@ -587,17 +599,17 @@ attn_status_t launch_decode_paged_q8(const void *q, const void *k_pages, const v
                                      const int *block_table, const int *seq_lens, void *o,
                                      float *lse, int S, int Hq, int Hkv, int d, int max_blocks,
                                      int num_pages, float scale, void *workspace,
-                                     cudaStream_t stream, unsigned *status) {
+                                     cudaStream_t stream) {
   const int G = Hq / Hkv;
   const int GB = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
   const int head_chunks = G / GB;
   const int HC = (Hkv % 8 == 0) ? 8 : (Hkv % 4 == 0) ? 4 : (Hkv % 2 == 0) ? 2 : 1;
-  const int nsplit = (max_blocks + kPagesPerSplitQ8 - 1) / kPagesPerSplitQ8;
-  const size_t parts = static_cast<size_t>(S) * Hq * nsplit;
-  float *o_part = static_cast<float *>(workspace);
-  float *l2_part = reinterpret_cast<float *>(
-      static_cast<uint8_t *>(workspace) +
-      ((parts * d * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+  static_assert(kPagesPerSplitQ8 == 32, "chunks of the shared decode workspace layout");
+  const int nsplit = decode_max_splits(max_blocks);
+  const DecodeWs ws = decode_ws_layout(workspace, S, Hq, d, max_blocks);
+  float *o_part = ws.o_part;
+  float *l2_part = ws.l2_part;
+  unsigned *status = ws.status;
   if (static_cast<long long>(Hkv / HC) * head_chunks > 65535 || S > 65535)
     return ATTN_ERR_UNSUPPORTED;
   CUtensorMap mk, mv;
@@ -618,8 +630,8 @@ attn_status_t launch_decode_paged_q8(const void *q, const void *k_pages, const v
   else
     return ATTN_ERR_UNSUPPORTED;
   if (st != ATTN_OK) return st;
-  return launch_decode_combine(o_part, l2_part, seq_lens, o, lse, S, Hq, d, max_blocks, nsplit,
-                               kPagesPerSplitQ8, stream);
+  return launch_decode_combine(ws, seq_lens, o, lse, S, Hq, d, max_blocks, nsplit,
+                               kPagesPerSplitQ8, stream, nullptr);
 }
 
 }  // namespace exattn

@@ -322,6 +322,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0 && round > 0)
           go = mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status);
         if (!__shfl_sync(0xffffffffu, go, 0)) break;
+#ifdef EXATTN_TEST_WITHHOLD
+        // Test build only: stop before ring index EXATTN_TEST_WITHHOLD, arriving
+        // on nothing and copying nothing, so the consumers' waits run out.
+        if (i == EXATTN_TEST_WITHHOLD) break;
+#endif
         if (lane == 0) mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
         __syncwarp();
         if (lane < BN / 16) {
@@ -372,6 +377,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int round = i / C::NST;
         if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status))
           break;
+#ifdef EXATTN_TEST_WITHHOLD
+        // Test build only: stop before ring index EXATTN_TEST_WITHHOLD, arriving
+        // on nothing and copying nothing, so the consumers' waits run out.
+        if (i == EXATTN_TEST_WITHHOLD) break;
+#endif
         mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
         const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
         for (int c = 0; c < C::CH; ++c)

@@ -16,15 +16,25 @@
  *
  * Conventions for every entry point:
  *  - All tensor arguments are DEVICE pointers to dense, row-major (C order)
- *    arrays owned by the caller.  The library never allocates, frees or
- *    synchronises; work is enqueued on `stream` (0 = legacy default stream) and
- *    the call returns before it finishes.
+ *    arrays owned by the caller.  The library never allocates or frees device
+ *    memory; work is enqueued on `stream` (0 = legacy default stream) and the
+ *    call returns before it finishes.  `stream` must belong to the current
+ *    device, and the tensors must live on it.  Only the two status reads below
+ *    wait for anything: attn_decode_read_status for its own 4-byte copy,
+ *    attn_device_status for the stream it is given.
  *  - Pointers must be 16-byte aligned.
  *  - Errors are reported only through the return value; nothing is written when
  *    a call returns anything but ATTN_OK.  No call aborts or traps.
  *  - Device-side conditions that the host cannot see in advance (a block-table
- *    entry outside the page pool, a bounded wait that ran out) set bits in a
- *    per-device status word read with attn_device_status().
+ *    entry outside the page pool, a bounded wait that ran out) set ATTN_DEV_*
+ *    bits in a status word.  A decode that takes a workspace (attn_decode_paged,
+ *    attn_decode_paged_q8) owns the word at the start of that workspace: each
+ *    such call clears it and reports only its own conditions there, read with
+ *    attn_decode_read_status().  Every other call ORs its bits into one word
+ *    per device, read (and cleared) with attn_device_status().
+ *  - The library looks up a few device addresses once per device and keeps
+ *    them; it does not support cudaDeviceReset (or a reset of the primary
+ *    context) while it is loaded.
  *  - `causal` means key j is visible to query i iff j <= i (queries and keys
  *    share positions 0..N-1).
  *  - L is the natural logarithm of sum_j exp(scale * q_i . k_j) over the
@@ -59,12 +69,13 @@ typedef enum {
     ATTN_ERR_CUDA = 3           /* a CUDA runtime or driver call failed */
 } attn_status_t;
 
-/* Bits of the per-device status word (attn_device_status). */
+/* Status bits (attn_decode_read_status, attn_device_status). */
 #define ATTN_DEV_BAD_PAGE 0x1u  /* a decode sequence referenced a page outside the pool or
                                    had a length outside [0, max_blocks*page_size]; its
                                    outputs are NaN */
-#define ATTN_DEV_TIMEOUT 0x2u   /* a bounded wait inside the prefill kernel expired; the
-                                   kernel returned early and its outputs are undefined */
+#define ATTN_DEV_TIMEOUT 0x2u   /* a bounded wait inside a kernel expired; the kernel
+                                   returned early and the outputs it owed are undefined
+                                   (a decode writes NaN for the sequences concerned) */
 #define ATTN_DEV_LAYOUT 0x4u    /* a backward kernel found its dynamic shared memory not
                                    1024-byte aligned and returned at once; the gradients
                                    are undefined */
@@ -184,8 +195,11 @@ EXATTN_API attn_status_t attn_bwd(const void *q, const void *k, const void *v, c
 
 /*
  * attn_decode_workspace_bytes -- bytes of device workspace attn_decode_paged
- * needs for S sequences, Hq query heads, head dim d and at most max_blocks
- * pages per sequence.  Returns 0 for invalid sizes.
+ * (and attn_decode_paged_q8) needs for S sequences, Hq query heads, head dim d
+ * and at most max_blocks pages per sequence.  The workspace starts with a
+ * 256-byte block whose first 32-bit word is the call's status word (see
+ * attn_decode_read_status); the chunk partials follow.  Returns 0 for invalid
+ * sizes.
  */
 EXATTN_API size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_blocks, int page_size);
 
@@ -204,11 +218,14 @@ EXATTN_API size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_bloc
  *   seq_lens     [S] int32, each in [0, max_blocks * page_size]
  *   o            [S, Hq, d] bf16 (out)      lse [S, Hq] float32 (out)
  *   workspace    device scratch of at least attn_decode_workspace_bytes(...) bytes,
- *                owned by the caller; its contents need no initialisation.
+ *                owned by the caller; its contents need no initialisation.  It
+ *                holds the call's status word until the next call that uses it.
  * d in {64, 128}; page_size == 16; Hq / Hkv in {1, 2, 4, 8, 16, 32, ...} (any divisor).
  * A sequence of length 0 gets O = 0 and L = -inf.  A sequence with a page id
  * outside [0, num_pages) or an out-of-range length gets NaN outputs and sets
- * ATTN_DEV_BAD_PAGE; no out-of-range address is ever dereferenced.
+ * ATTN_DEV_BAD_PAGE in the workspace's status word; no out-of-range address is
+ * ever dereferenced.  Calls on different workspaces never share a status word,
+ * so concurrent decodes on several streams each report only their own faults.
  */
 EXATTN_API attn_status_t attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
                                 const int32_t *block_table, const int32_t *seq_lens,
@@ -270,7 +287,10 @@ EXATTN_API attn_status_t attn_decode_paged_q8(const void *q, const void *k_pages
  *   until the process exits.
  * - The first call on a device looks up the scratch's device address (with that
  *   device current) and caches it; make that first call before any stream
- *   capture.
+ *   capture.  `stream` must belong to the current device.
+ * - The scratch's status word is shared too, so this call reports a bad page id
+ *   or length (ATTN_DEV_BAD_PAGE) in the per-device word of attn_device_status,
+ *   not through attn_decode_read_status.
  * - All calls on a device share the one array and leave their partials in it.
  *   Calls whose kernels overlap on the GPU (different streams, no ordering
  *   between them) race on it; order them on one stream or use attn_decode_paged
@@ -292,11 +312,27 @@ EXATTN_API attn_status_t attn_decode_paged_noalloc(const void *q, const void *k_
                                                    attn_stream_t stream);
 
 /*
- * attn_device_status -- read (and, if clear != 0, reset) the status word of the
- * current device.  Synchronises the device first, so call it between steps, not
- * inside stream capture.
+ * attn_decode_read_status -- the ATTN_DEV_* bits of the last attn_decode_paged
+ * or attn_decode_paged_q8 call that used `workspace` (0: no sequence failed).
+ * The paged decode's only device-side failure is the Lab 03 step 4 one: a
+ * block-table entry (the indirection table) naming a page outside the pool, or
+ * a length the table cannot hold (ATTN_DEV_BAD_PAGE); a wait that ran out gives
+ * ATTN_DEV_TIMEOUT.  Synchronises nothing: the caller first synchronises the
+ * stream the decode ran on (or waits on an event recorded after it); the call
+ * then copies the one word to the host through a stream of its own, waiting only
+ * for that copy.  `workspace` is the device pointer given to the decode.
+ * ATTN_ERR_INVALID_ARG for a null or misaligned workspace or a null dev_status.
  */
-EXATTN_API attn_status_t attn_device_status(unsigned *status, int clear);
+EXATTN_API attn_status_t attn_decode_read_status(const void *workspace, unsigned *dev_status);
+
+/*
+ * attn_device_status -- read (and, if clear != 0, reset) the status word of the
+ * current device, which every call other than the workspace decodes reports
+ * into.  Waits for the work enqueued on `stream` so far, and only for that:
+ * pass the stream the calls of interest ran on (kernels still running on other
+ * streams may set bits later).  Not for use inside stream capture.
+ */
+EXATTN_API attn_status_t attn_device_status(unsigned *status, int clear, attn_stream_t stream);
 
 /* attn_status_string -- a static, human-readable name for a status code. */
 EXATTN_API const char *attn_status_string(attn_status_t status);

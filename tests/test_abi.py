@@ -102,10 +102,11 @@ def test_window_alibi_argument_checks(lib, window, causal, slopes, code):
 
 
 def test_decode_workspace_size(lib):
-    # 512 pages of 16 tokens in chunks of 32 pages -> 16 chunks per sequence.
+    # 512 pages of 16 tokens in chunks of 32 pages -> 16 chunks per sequence;
+    # a 256-byte status block precedes the partials.
     n = ea.decode_workspace_bytes(64, 32, 128, 512)
     parts = 64 * 32 * 16
-    assert n >= parts * 129 * 4 and n % 256 == 0 and n < parts * 129 * 4 + 512
+    assert n >= 256 + parts * 129 * 4 and n % 256 == 0 and n < 256 + parts * 129 * 4 + 512
     assert ea.decode_workspace_bytes(64, 32, 96, 512) == 0
     assert ea.decode_workspace_bytes(64, 32, 128, 512, page_size=32) == 0
     assert ea.decode_workspace_bytes(0, 32, 128, 512) == 0
@@ -134,6 +135,48 @@ def test_decode_argument_checks(lib, kw, code):
 
 def test_decode_rejects_small_workspace(lib):
     assert dec(lib, ws_bytes=64) == INVALID
+
+
+def test_decode_read_status_argument_checks(lib):
+    import ctypes
+    st = ctypes.c_uint(7)
+    assert lib.attn_decode_read_status(None, ctypes.byref(st)) == INVALID
+    assert lib.attn_decode_read_status(A + 8, ctypes.byref(st)) == INVALID
+    assert lib.attn_decode_read_status(A, None) == INVALID
+    assert st.value == 7  # nothing written on an error
+    assert lib.attn_device_status(None, 0, None) == INVALID
+
+
+@pytest.mark.parametrize("which", ["paged", "q8", "noalloc"])
+def test_decode_binding_checks_shapes_before_the_library(which):
+    # The C side gets no tensor sizes, so the binding must reject a block table
+    # or length vector with fewer rows than q has sequences, and pools that do
+    # not agree, before any call (these CPU tensors never reach the library).
+    import torch
+    S, Hq, Hkv, d, P = 3, 8, 2, 128, 10
+    q = torch.zeros(S, Hq, d, dtype=torch.bfloat16)
+    kp = torch.zeros(P, Hkv, 16, d, dtype=torch.bfloat16)
+    bt = torch.zeros(S, 4, dtype=torch.int32)
+    sl = torch.zeros(S, dtype=torch.int32)
+    sc = torch.ones(P, Hkv)
+
+    def call(q=q, kp=kp, vp=kp, bt=bt, sl=sl):
+        if which == "paged":
+            return ea.attn_decode_paged(q, kp, vp, bt, sl)
+        if which == "noalloc":
+            return ea.attn_decode_paged_noalloc(q, kp, vp, bt, sl)
+        return ea.attn_decode_paged_q8(q, kp.to(torch.int8), vp.to(torch.int8), sc, sc, bt, sl,
+                                       kv_format="int8")
+    with pytest.raises(ValueError, match="S rows"):
+        call(bt=bt[:2])
+    with pytest.raises(ValueError, match="S rows"):
+        call(sl=sl[:1])
+    with pytest.raises(ValueError, match="page pools"):
+        call(vp=kp[:, :1].contiguous())
+    with pytest.raises(ValueError, match="page pools"):
+        call(q=torch.zeros(S, Hq, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="dims"):
+        call(bt=bt[0])
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -5,8 +5,10 @@ Covers lengths at and around page and chunk boundaries (0, 1, 15, 16, 17,
 511, 512, 513, ...), MHA / GQA / MQA head sharing, both head dims, placement
 invariance (the same tokens on other pages give bit-identical results), the
 autoregressive check against the causal prefill, a corrupt block table (status
-bit and NaN outputs, no out-of-range access), and the full-size workload in
-the launch configuration bench.py times.
+bit in the call's own workspace and NaN outputs, no out-of-range access), two
+concurrent decodes on two streams that each report only their own status, and
+the full-size workload (every sequence) in the launch configuration bench.py
+times.
 """
 from __future__ import annotations
 
@@ -41,12 +43,18 @@ def oracle_decode(inp, scale, seq_ids=None):
                                inp["seq_lens"].numpy(), scale=scale, seq_ids=seq_ids)
 
 
-def gpu_decode(inp, scale):
+def gpu_decode(inp, scale, workspace=None):
     d = {k: v.to(DEV) for k, v in inp.items()}
     o, l = ea.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],
-                                d["seq_lens"], scale=scale)
+                                d["seq_lens"], scale=scale, workspace=workspace)
     torch.cuda.synchronize()
     return o, l
+
+
+def workspace_for(inp):
+    S, Hq, d = inp["q"].shape
+    n = ea.decode_workspace_bytes(S, Hq, d, inp["block_table"].shape[1])
+    return torch.empty(n, dtype=torch.uint8, device=DEV)
 
 
 CASES = [
@@ -124,29 +132,81 @@ def test_decode_matches_causal_prefill_rows():
 
 def test_decode_bad_page_sets_status_and_nan():
     cfg, inp = make_case([40, 40], 8, 2, 128, num_pages=12, max_blocks=4, seed=5)
-    bt = inp["block_table"].clone()
+    good_bt = inp["block_table"]
+    bt = good_bt.clone()
     bt[1, 1] = 12          # one past the pool: must not be dereferenced
     inp = dict(inp, block_table=bt)
-    ea.device_status(clear=True)
-    o, l = gpu_decode(inp, cfg.scale)
-    assert ea.device_status(clear=True) & ea.ATTN_DEV_BAD_PAGE
+    assert ea.device_status(clear=True) == 0
+    ws = workspace_for(inp)
+    o, l = gpu_decode(inp, cfg.scale, workspace=ws)
+    # The call's own status word holds the bit; the per-device word stays clear.
+    assert ea.decode_read_status(ws) == ea.ATTN_DEV_BAD_PAGE
+    assert ea.device_status() == 0
     assert torch.isnan(o[1].float()).all() and torch.isnan(l[1]).all()
     o_ref, l_ref = oracle_decode(inp, cfg.scale, seq_ids=[0])
     assert_bf16_parity(o[0:1], l[0:1], o_ref, l_ref)
+    # The next call on the same workspace clears the word it inherited.
+    o2, l2 = gpu_decode(dict(inp, block_table=good_bt), cfg.scale, workspace=ws)
+    assert ea.decode_read_status(ws) == 0
+    assert torch.isfinite(o2.float()).all() and torch.isfinite(l2).all()
+
+
+def test_decode_bad_length_sets_status():
+    # A length past max_blocks * 16 is caught on the device too (the table
+    # cannot hold it); the other sequence is unaffected.
+    cfg, inp = make_case([40, 40], 8, 2, 128, num_pages=12, max_blocks=4, seed=6)
+    inp = dict(inp, seq_lens=torch.tensor([40, 4 * 16 + 1], dtype=torch.int32))
+    ws = workspace_for(inp)
+    o, l = gpu_decode(inp, cfg.scale, workspace=ws)
+    assert ea.decode_read_status(ws) == ea.ATTN_DEV_BAD_PAGE
+    assert torch.isnan(o[1].float()).all() and torch.isnan(l[1]).all()
+    o_ref, l_ref = oracle_decode(inp, cfg.scale, seq_ids=[0])
+    assert_bf16_parity(o[0:1], l[0:1], o_ref, l_ref)
+
+
+def test_decode_status_is_per_call_on_two_streams():
+    # Two decodes run concurrently on two streams with their own workspaces;
+    # only the one whose block table is corrupt reports ATTN_DEV_BAD_PAGE, and
+    # neither touches the per-device word.
+    cfg, inp = make_case([900, 40, 3000], 8, 2, 128, num_pages=300, max_blocks=200, seed=8)
+    bad_bt = inp["block_table"].clone()
+    bad_bt[2, 150] = -7
+    dev_good = {k: v.to(DEV) for k, v in inp.items()}
+    dev_bad = dict(dev_good, block_table=bad_bt.to(DEV))
+    ws_good, ws_bad = workspace_for(inp), workspace_for(inp)
+    assert ea.device_status(clear=True) == 0
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    outs = {}
+    for name, st, dv, ws in (("good", s1, dev_good, ws_good), ("bad", s2, dev_bad, ws_bad)):
+        with torch.cuda.stream(st):
+            outs[name] = ea.attn_decode_paged(dv["q"], dv["k_pages"], dv["v_pages"],
+                                              dv["block_table"], dv["seq_lens"],
+                                              scale=cfg.scale, workspace=ws)
+    s1.synchronize()
+    assert ea.decode_read_status(ws_good) == 0
+    s2.synchronize()
+    assert ea.decode_read_status(ws_bad) == ea.ATTN_DEV_BAD_PAGE
     assert ea.device_status() == 0
+    o_ref, l_ref = oracle_decode(inp, cfg.scale)
+    assert_bf16_parity(outs["good"][0], outs["good"][1], o_ref, l_ref, "good stream")
+    ob, lb = outs["bad"]
+    assert torch.isnan(ob[2].float()).all() and torch.isnan(lb[2]).all()
+    assert_bf16_parity(ob[:2], lb[:2], o_ref[:2], l_ref[:2], "bad stream, good sequences")
 
 
 def test_decode_full_size_workload():
     cfg = syn.DECODE
     inp = syn.decode_inputs(cfg, device=DEV)
+    ws = workspace_for(inp)
     o, l = ea.attn_decode_paged(inp["q"], inp["k_pages"], inp["v_pages"], inp["block_table"],
-                                inp["seq_lens"], scale=cfg.scale)
+                                inp["seq_lens"], scale=cfg.scale, workspace=ws)
     torch.cuda.synchronize()
-    assert ea.device_status() == 0
+    assert ea.decode_read_status(ws) == 0 and ea.device_status() == 0
     assert torch.isfinite(o.float()).all() and torch.isfinite(l).all()
-    # Compare 16 sampled sequences (all heads) with the oracle; gather only the
-    # pages they use so the host copy stays small.
-    seqs = [0, 1, 5, 17, 31, 32, 40, 47, 50, 55, 58, 60, 61, 62, 63, 33]
+    # Compare every sequence (all heads) with the oracle; gather only the pages
+    # they use so the host copy holds no unused page.
+    seqs = list(range(cfg.S))
     bt = inp["block_table"][seqs]
     used = torch.unique(bt[bt >= 0])
     remap = torch.full((cfg.num_pages,), -1, dtype=torch.int32, device=DEV)

@@ -117,6 +117,9 @@ def test_fp32_shapes(B, Hq, Hkv, N, d, causal):
 
 
 def sample_rows(B, Hq, N, n_random, seed):
+    """Flat row indices: tile-edge and random rows of random heads, plus every
+    row of the last (batch, head) -- a whole head covers every Q-tile position
+    of the grid's last CTAs."""
     rng = np.random.default_rng(seed)
     fixed = [0, 1, 127, 128, 129, 255, 256, N // 2, N - 129, N - 128, N - 2, N - 1]
     rows = []
@@ -125,7 +128,8 @@ def sample_rows(B, Hq, N, n_random, seed):
             rows.append((int(rng.integers(B)), int(rng.integers(Hq)), r))
     for _ in range(n_random):
         rows.append((int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(N))))
-    return np.array([(b * Hq + h) * N + i for b, h, i in rows], dtype=np.int64)
+    rows += [(B - 1, Hq - 1, i) for i in range(N)]
+    return np.unique(np.array([(b * Hq + h) * N + i for b, h, i in rows], dtype=np.int64))
 
 
 def full_size_check(cfg, n_random=64):

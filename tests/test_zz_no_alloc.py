@@ -10,19 +10,45 @@ The GPU test calls the new entry point through the C ABI, twice in a row (the
 scratch keeps the previous call's partials, which must not leak into the next
 result), and checks both outputs against attn_decode_paged with a separately
 allocated workspace, within the bf16 tolerances the other decode tests use.
+Before the second call the scratch is filled with NaN partials from a longer
+problem of the same shape, so a result that read a stale slot would show it;
+the small case is also checked against the fp64 oracle.
 This file is named to be collected last, so a run that stops at the first
 failure has already run every other test.
 """
 from __future__ import annotations
 
-import ctypes
-
+import numpy as np
 import pytest
 import torch
 
 import exact_io_aware_101_b200 as ea
+import oracle
 from exact_io_aware_101_b200 import synthetic as syn
-from parity_helpers import BF16_MAX_L, BF16_MAX_O, BF16_MEAN_O
+from parity_helpers import BF16_MAX_L, BF16_MAX_O, BF16_MEAN_O, assert_bf16_parity
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _poison_scratch(lib, cfg, inp):
+    """A noalloc call on NaN pages with every sequence at the longest length the
+    block table allows: it leaves a NaN partial in every scratch slot that a
+    problem of this shape (S, Hq, d, max_blocks) can use."""
+    npg = cfg.S * cfg.max_blocks
+    kp = torch.full((npg, cfg.Hkv, cfg.page_size, cfg.d), float("nan"), dtype=torch.bfloat16,
+                    device="cuda")
+    bt = torch.arange(npg, dtype=torch.int32, device="cuda").view(cfg.S, cfg.max_blocks)
+    sl = torch.full((cfg.S,), cfg.max_blocks * cfg.page_size, dtype=torch.int32, device="cuda")
+    poison = dict(q=inp["q"], k_pages=kp, v_pages=kp, block_table=bt, seq_lens=sl)
+    cfg_p = syn.Decode(name="poison", S=cfg.S, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, num_pages=npg,
+                       max_blocks=cfg.max_blocks, seed=0)
+    o = torch.empty_like(inp["q"])
+    l = torch.empty(cfg.S, cfg.Hq, dtype=torch.float32, device="cuda")
+    assert _noalloc(lib, poison, cfg_p, o, l) == 0
+    torch.cuda.synchronize()
+    assert torch.isnan(l).all()
 
 
 def _noalloc(lib, inp, cfg, o, lse):
@@ -68,11 +94,38 @@ def test_noalloc_matches_workspace_decode_twice(which):
     l_ref = torch.empty(cfg.S, cfg.Hq, dtype=torch.float32, device="cuda")
     assert _with_workspace(lib, inp, cfg, o_ref, l_ref) == 0
     for call in range(2):
+        if call == 1 and which == "small":
+            _poison_scratch(lib, cfg, inp)
         o = torch.full_like(inp["q"], float("nan"))
         l = torch.full((cfg.S, cfg.Hq), float("nan"), device="cuda")
         assert _noalloc(lib, inp, cfg, o, l) == 0, call
         torch.cuda.synchronize()
         _close(o, l, o_ref, l_ref)
+        if which == "small":
+            host = {k: v.cpu() for k, v in inp.items()}
+            o_or, l_or = oracle.decode_paged(host["q"].float().numpy(), _bits(host["k_pages"]),
+                                             _bits(host["v_pages"]), host["block_table"].numpy(),
+                                             host["seq_lens"].numpy(), scale=cfg.scale)
+            assert_bf16_parity(o, l, o_or, l_or, "noalloc vs oracle, call %d" % call)
+    assert ea.device_status() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_bad_page_reports_in_the_device_word():
+    # The scratch (and its status word) is shared, so this entry point reports a
+    # corrupt block table in the per-device word.
+    lib = ea.library()
+    cfg = syn.Decode(name="noalloc_bad", S=2, Hq=8, Hkv=2, d=128, num_pages=12, max_blocks=4,
+                     seed=5)
+    inp = syn.decode_inputs(cfg, device="cuda", seq_lens=[40, 40])
+    inp["block_table"][1, 1] = 12  # one past the pool
+    assert ea.device_status(clear=True) == 0
+    o = torch.empty_like(inp["q"])
+    l = torch.empty(cfg.S, cfg.Hq, dtype=torch.float32, device="cuda")
+    assert _noalloc(lib, inp, cfg, o, l) == 0
+    torch.cuda.synchronize()
+    assert ea.device_status(clear=True) == ea.ATTN_DEV_BAD_PAGE
+    assert torch.isnan(l[1]).all() and torch.isfinite(l[0]).all()
     assert ea.device_status() == 0
 
 
