@@ -30,13 +30,9 @@
 //    special-function unit is not the bottleneck.
 //  * Causal: KV tiles above the diagonal are never loaded or multiplied; only
 //    diagonal tiles are masked (Concepts: causal masking; Lab 01 step 4).
-//  * Work items are (Q-tile pair, batch*head).  Consecutive items share K/V
+//  * Grid: one CTA per (Q-tile pair, batch*head).  Consecutive CTAs share K/V
 //    (same head, or the query heads of one K/V group), so re-reads hit L2;
-//    causal items go heaviest pair first within groups of 8 heads.  The CTAs
-//    are persistent, one per SM: the next item's Q and first K/V tiles load,
-//    and its first score MMAs run, while the current item's last tiles and
-//    epilogue finish, so a CTA's start-up cost is paid once, not per item.
-//    (The chunked-prefill variant keeps one item per CTA.)
+//    causal grids go heaviest pair first within groups of 8 heads.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -81,11 +77,9 @@ struct Bars {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t q_full;
-  uint64_t q_empty;      // the last score MMA of an item has read Q (one commit)
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
-  uint64_t o_empty[2];   // a Q tile's epilogue has read O out of TMEM (128 arrivals)
   uint64_t mrg_full;     // split item: warpgroup 1's O, m, l are final (128 arrivals)
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -98,7 +92,7 @@ struct Params {
   unsigned *status;
   int B, Hq, Hkv, N;
   int pairs;  // ceil(N / 256)
-  int split_pairs;  // the last split_pairs pair items run as 2 split items each
+  int whole_pairs;  // split kernel: pair items [whole_pairs, ...) run as two split CTAs each
   float scale_log2;
   int causal;
   int window;            // > 0: key j visible to query i only if i - j < window
@@ -139,101 +133,7 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float c, flo
   return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
 }
 
-// One work item: a pair of 128-row Q tiles of one (batch, head) -- or, in the
-// chunked-prefill variant, of one sequence's chunk -- and the KV tiles each
-// of the two Q tiles walks.
-struct Item {
-  bool valid;        // false: a split item of a Q tile past the rows (skipped)
-  bool split;        // one Q tile, its KV tiles [jlo, mid) and [mid, jhi) on the
-                     // two warpgroups (tiles 0 and 1 share rows), merged at the end
-  int mid;
-  int b, hq, hkv;
-  int row0;          // first query row of the pair (within the head or chunk)
-  int nq, nk;        // query rows and keys of the head (chunk: its rows, its keys)
-  int ctx, qrow0;    // position of row 0 among the keys; chunk: first token row
-  int js0, je0, js1, je1;  // KV tiles [js_t, je_t) of Q tile t (empty past the rows)
-  int jlo, jhi;
-};
-
-// KV tile ranges of an item whose (b, hq, row0, nq, nk, ctx) are set: the
-// causal diagonal caps the end, a sliding window moves the start, and a Q tile
-// past the rows has none.
-__device__ __forceinline__ void item_ranges(const Params &p, Item &it) {
-  const int nkv = (it.nk + BN - 1) / BN;
-  const bool rows1 = it.row0 + BM < it.nq;
-  const int last0 = min(it.row0 + BM, it.nq) - 1, last1 = min(it.row0 + 2 * BM, it.nq) - 1;
-  it.je0 = p.causal ? min((it.ctx + last0) / BN + 1, nkv) : nkv;
-  it.je1 = !rows1 ? 0 : (p.causal ? min((it.ctx + last1) / BN + 1, nkv) : nkv);
-  it.js0 = p.window > 0 ? max(0, it.ctx + it.row0 - p.window + 1) / BN : 0;
-  it.js1 = (!rows1 || p.window <= 0) ? 0 : max(0, it.ctx + it.row0 + BM - p.window + 1) / BN;
-  it.jlo = it.js0;
-  it.jhi = max(it.je0, it.je1);
-}
-
-// Self-attention work item `lin` (0 <= lin < pairs * B * Hq).  Non-causal:
-// head-major, so the items in flight at one time share a few heads' K/V in L2.
-// Causal: groups of kHeadGroup heads, heaviest pairs first inside each group
-// (load balance) while a group's K/V stays in L2.
-__device__ __forceinline__ Item self_item(const Params &p, int lin) {
-  const int BH = p.B * p.Hq;
-  const int whole = p.pairs * BH - p.split_pairs;  // pair items that stay whole
-  int split_tile = -1;  // split item: which Q tile of its pair
-  if (lin >= whole) {
-    split_tile = (lin - whole) & 1;
-    lin = whole + ((lin - whole) >> 1);
-  }
-  int pair, bh;
-  if (!p.causal) {
-    bh = lin / p.pairs;
-    pair = lin % p.pairs;
-  } else {
-    const int grp = lin / (kHeadGroup * p.pairs);
-    const int first = grp * kHeadGroup;
-    const int hg = min(kHeadGroup, BH - first);
-    const int rr = lin - grp * kHeadGroup * p.pairs;
-    pair = p.pairs - 1 - rr / hg;
-    bh = first + rr % hg;
-  }
-  Item it;
-  it.valid = true;
-  it.split = false;
-  it.mid = 0;
-  it.b = bh / p.Hq;
-  it.hq = bh % p.Hq;
-  it.hkv = it.hq / (p.Hq / p.Hkv);
-  it.row0 = pair * 2 * BM;
-  it.nq = p.N;
-  it.nk = p.N;
-  it.ctx = 0;
-  it.qrow0 = 0;
-  if (split_tile >= 0) {
-    // One Q tile: its own KV range, cut in two halves (the first one the
-    // larger) for the two warpgroups; a single KV tile stays on warpgroup 0.
-    it.row0 += split_tile * BM;
-    it.valid = it.row0 < it.nq;
-    const int save = it.nq;
-    it.nq = min(save, it.row0 + BM);  // rows1 false: tile 1 gets no range here
-    item_ranges(p, it);
-    it.nq = save;
-    const int n = it.je0 - it.js0;
-    it.jlo = it.js0;
-    it.jhi = it.je0;
-    if (n >= 2) {
-      it.split = true;
-      it.mid = it.js0 + (n + 1) / 2;
-      it.je0 = it.mid;
-      it.js1 = it.mid;
-      it.je1 = it.jhi;
-    } else {
-      it.js1 = it.je1 = 0;
-    }
-    return it;
-  }
-  item_ranges(p, it);
-  return it;
-}
-
-template <int D, bool kAlibi, bool kPaged>
+template <int D, bool kAlibi, bool kPaged, bool kSplit>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -241,6 +141,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_k1,
                         const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   using C = Cfg<D>;
+  // The split CTAs of a launch come as a second grid, programmatically
+  // dependent on this one: it may be scheduled on the SMs this grid frees.
+  if constexpr (!kPaged && !kSplit) grid_dependents_launch();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -252,25 +155,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work items.  Self-attention: the CTA is persistent; round r gives it
-  // item r*G + c (even r) or r*G + G-1-c (odd r) for CTA c of G, so each round
-  // covers the next G items in order (the L2 locality of the order above) and
-  // the snake evens out the heaviest-first causal items across CTAs.  Every
-  // role walks the same item sequence; the barriers' phases run on across
-  // items.  Chunked prefill: one item per CTA, validated here first.
-  Item first{};
+  // ---- work item: Q-tile pair and (batch, head).  Non-causal: head-major, so
+  // the CTAs resident at one time share a few heads' K/V in L2.  Causal: groups
+  // of kHeadGroup heads, heaviest pairs first inside each group (load balance)
+  // while a group's K/V stays in L2.
+  const int BH = p.B * p.Hq;
+  int pair, bh;
+  // The split variant (kSplit) runs split CTAs only: one Q tile (split_tile
+  // of its pair) whose KV tiles are halved over the two softmax warpgroups --
+  // both hold the same rows -- and merged at the end.  It is launched behind
+  // the whole pairs for the pairs that did not fill a last wave (see launch).
+  int split_tile = -1;
   if constexpr (kPaged) {
-    // A CTA's work grows with its sequence's key count, which varies by up to
-    // the longest context over the shortest.  The grid takes the sequences
-    // longest first (ranked here by key count, ties by index), each one's
-    // heaviest pair first, all heads of a pair together, so that the last wave
-    // holds the short ones.  Past kRankMax sequences the order stays as given
-    // (the grid is then large enough to balance by itself).
+    // Chunked prefill: a CTA's work grows with its sequence's key count, which
+    // varies by up to the longest context over the shortest.  The grid takes
+    // the sequences longest first (ranked here by key count, ties by index),
+    // each one's heaviest pair first, all heads of a pair together, so that
+    // the last wave holds the short ones.  Past kRankMax sequences the order
+    // stays as given (the grid is then large enough to balance by itself).
     const int lin = static_cast<int>(blockIdx.x);
     const int per_seq = p.pairs * p.Hq;
     const int r = lin / per_seq;
     const int rem = lin - r * per_seq;
-    const int pair = p.pairs - 1 - rem / p.Hq;
+    pair = p.pairs - 1 - rem / p.Hq;
     int seq = r;
     if (p.B <= kRankMax) {
       __shared__ int s_len[kRankMax];
@@ -287,42 +194,97 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncthreads();
       seq = s_seq;
     }
-    first.b = seq;
-    first.hq = rem % p.Hq;
-    first.hkv = first.hq / (p.Hq / p.Hkv);
-    first.row0 = pair * 2 * BM;
-    // Rows of the sequence's chunk (nq) and its keys (nk); the chunk's queries
-    // are the last nq of the sequence's nk positions.  (p.N is the caller's
-    // bound max_q on every chunk length; the grid covers it.)
-    const int q0 = p.cu_q[seq], q1 = p.cu_q[seq + 1];
-    first.nk = p.seq_lens[seq];
-    first.nq = q1 - q0;
-    first.qrow0 = q0;
-    const bool bad_len = q0 < 0 || first.nq < 0 || q1 > p.T || first.nk < first.nq ||
-                         first.nk > p.max_blocks * 16 || first.nq > p.N;
+    bh = seq * p.Hq + rem % p.Hq;
+  } else {
+    int lin = static_cast<int>(blockIdx.x);
+    if constexpr (kSplit) {
+      split_tile = lin & 1;
+      lin = p.whole_pairs + (lin >> 1);
+    }
+    if (!p.causal) {
+      bh = lin / p.pairs;
+      pair = lin % p.pairs;
+    } else {
+      const int grp = lin / (kHeadGroup * p.pairs);
+      const int first = grp * kHeadGroup;
+      const int hg = min(kHeadGroup, BH - first);
+      const int rr = lin - grp * kHeadGroup * p.pairs;
+      pair = p.pairs - 1 - rr / hg;
+      bh = first + rr % hg;
+    }
+  }
+  const int b = bh / p.Hq;
+  const int hq = bh % p.Hq;
+  const int hkv = hq / (p.Hq / p.Hkv);
+  const int row0 = pair * 2 * BM + (split_tile > 0 ? BM : 0);
+  // Rows of this (batch, head) or sequence chunk (nq), keys (nk), and the
+  // position of row 0 among the keys (ctx: 0 for self-attention; for a chunk,
+  // its queries are the last nq of the sequence's nk positions).
+  int nq = p.N, nk = p.N, ctx = 0, qrow0 = 0;
+  if constexpr (kPaged) {
+    const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1];
+    nk = p.seq_lens[b];
+    nq = q1 - q0;
+    qrow0 = q0;
+    // (For a chunk, p.N is the caller's bound max_q on every chunk length; the
+    // grid covers it.)
+    const bool bad_len = q0 < 0 || nq < 0 || q1 > p.T || nk < nq || nk > p.max_blocks * 16 ||
+                         nq > p.N;
     if (bad_len) {
-      if (threadIdx.x == 0 && pair == 0 && first.hq == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
+      if (threadIdx.x == 0 && pair == 0 && hq == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
       return;
     }
-    if (first.row0 >= first.nq) return;  // pair past the chunk: nothing to do
-    first.ctx = first.nk - first.nq;
-    item_ranges(p, first);
+    if (row0 >= nq) return;  // pair past the chunk: nothing to do
+    ctx = nk - nq;
+  }
+  if (split_tile >= 0 && row0 >= nq) return;  // split CTA of a Q tile past the rows
+  const int nkv = (nk + BN - 1) / BN;
+  // KV tiles [js_t, je_t) of each Q tile: the causal diagonal caps the end,
+  // a sliding window moves the start; a Q tile past the rows has none.
+  // (Scalars, not arrays: the issuing thread reads them every iteration.)
+  const bool rows1 = split_tile < 0 && row0 + BM < nq;
+  int je0, je1, js0, js1;
+  if constexpr (kPaged) {  // the diagonal sits ctx keys to the right
+    const int last0 = min(row0 + BM, nq) - 1, last1 = min(row0 + 2 * BM, nq) - 1;
+    je0 = p.causal ? min((ctx + last0) / BN + 1, nkv) : nkv;
+    je1 = !rows1 ? 0 : (p.causal ? min((ctx + last1) / BN + 1, nkv) : nkv);
+    js0 = p.window > 0 ? max(0, ctx + row0 - p.window + 1) / BN : 0;
+    js1 = (!rows1 || p.window <= 0) ? 0 : max(0, ctx + row0 + BM - p.window + 1) / BN;
+  } else {
+    je0 = p.causal ? min(row0 / BN + 1, nkv) : nkv;
+    je1 = !rows1 ? 0 : (p.causal ? min((row0 + BM) / BN + 1, nkv) : nkv);
+    js0 = p.window > 0 ? max(0, row0 - p.window + 1) / BN : 0;
+    js1 = (!rows1 || p.window <= 0) ? 0 : max(0, row0 + BM - p.window + 1) / BN;
+  }
+  // A split CTA's one Q tile: its KV range halved (the first half the larger);
+  // a single KV tile stays on warpgroup 0.
+  bool split = false;  // (always false in the whole-pair kernel)
+  int mid = 0;
+  if (kSplit && je0 - js0 >= 2) {
+    split = true;
+    mid = js0 + (je0 - js0 + 1) / 2;
+    js1 = mid;
+    je1 = je0;
+    je0 = mid;
+  }
+  const int jlo = js0;
+  const int jhi = max(je0, je1);
+  if constexpr (kPaged) {
     // Every page the tiles [jlo, jhi) read must be in the pool; a sequence
     // with a bad entry gets NaN rows and the status bit, and no copy is issued.
-    const int pg_end = min(first.jhi * (BN / 16), (first.nk + 15) / 16);
+    const int pg_end = min(jhi * (BN / 16), (nk + 15) / 16);
     bool bad = false;
-    for (int i = first.jlo * (BN / 16) + static_cast<int>(threadIdx.x); i < pg_end;
-         i += NUM_THREADS) {
-      const int pid = p.block_table[static_cast<size_t>(seq) * p.max_blocks + i];
+    for (int i = jlo * (BN / 16) + static_cast<int>(threadIdx.x); i < pg_end; i += NUM_THREADS) {
+      const int pid = p.block_table[static_cast<size_t>(b) * p.max_blocks + i];
       bad |= pid < 0 || pid >= p.num_pages;
     }
     if (__syncthreads_or(bad)) {
       if (threadIdx.x == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
       for (int idx = threadIdx.x; idx < 2 * BM * (D + 1); idx += NUM_THREADS) {
-        const int r2 = idx / (D + 1), c = idx % (D + 1);
-        const int row = first.row0 + r2;
-        if (row >= first.nq) continue;
-        const size_t tok = static_cast<size_t>(first.qrow0 + row) * p.Hq + first.hq;
+        const int r = idx / (D + 1), c = idx % (D + 1);
+        const int row = row0 + r;
+        if (row >= nq) continue;
+        const size_t tok = static_cast<size_t>(qrow0 + row) * p.Hq + hq;
         if (c < D)
           reinterpret_cast<__nv_bfloat16 *>(p.o)[tok * D + c] = __float2bfloat16_rn(NAN);
         else
@@ -331,28 +293,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       return;
     }
   }
-  const int n_items = kPaged ? 1 : p.pairs * p.B * p.Hq + p.split_pairs;
-  const int G = static_cast<int>(gridDim.x);
-  const int cta = static_cast<int>(blockIdx.x);
-  // The CTA's next item from round r on (r advances past it), or false once the
-  // CTA's items are done.  Every role walks the same sequence.
-  auto fetch = [&](int &r, Item &it) -> bool {
-    if constexpr (kPaged) {
-      if (r > 0) return false;
-      it = first;
-      ++r;
-      return true;
-    } else {
-      while (true) {
-        if (static_cast<long long>(r) * G >= n_items) return false;
-        const int lin = r * G + ((r & 1) ? G - 1 - cta : cta);
-        ++r;
-        if (lin >= n_items) return false;  // (only in the last, partial round)
-        it = self_item(p, lin);
-        if (it.valid) return true;
-      }
-    }
-  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -360,12 +300,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&bars->empty[i], 1);
     }
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], BM);
       mbar_init(&bars->o_full[t], 1);
-      mbar_init(&bars->o_empty[t], BM);
     }
     mbar_init(&bars->mrg_full, BM);
     mbar_init(&bars->mma_done, 1);
@@ -386,16 +324,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    // Q of an item once (both tiles, after the previous item's last score MMA
-    // has read the buffer: q_empty), then its K0 V0 K1 V1 ... into the ring;
-    // the ring index runs on across items.
     regs_dec<kRegsLow>();
     if constexpr (kPaged) {
       // The whole warp gathers: lane 0 runs the barrier protocol and the Q
       // copies, lanes 0-7 each bring one page of every K/V tile, so the eight
       // block-table reads and sixteen or more box copies per tile proceed in
       // parallel.
-      const Item &it = first;
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -406,10 +340,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::CH; ++c)
             tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
-                        it.hq, it.qrow0 + it.row0 + t * BM);
+                        hq, qrow0 + row0 + t * BM);
       }
       int issued = 0;
-      for (int i = 0; i < 2 * (it.jhi - it.jlo); ++i) {
+      for (int i = 0; i < 2 * (jhi - jlo); ++i) {
         const int slot = i % C::NST;
         const int round = i / C::NST;
         bool go = true;
@@ -430,11 +364,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // shared memory, which a zero P could not cancel if it held a NaN).
           const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
           const CUtensorMap *map1 = (i & 1) ? &tm_v1 : &tm_k1;
-          const int key0 = (it.jlo + (i >> 1)) * BN + lane * 16;
-          const int ntok = min(16, it.nk - key0);
+          const int key0 = (jlo + (i >> 1)) * BN + lane * 16;
+          const int ntok = min(16, nk - key0);
           const int z = ntok > 0
-              ? p.block_table[static_cast<size_t>(it.b) * p.max_blocks + key0 / 16] * p.Hkv +
-                    it.hkv
+              ? p.block_table[static_cast<size_t>(b) * p.max_blocks + key0 / 16] * p.Hkv + hkv
               : -1;
           uint8_t *dst = sRing + slot * C::TILE_BYTES + lane * 16 * 128;
           for (int c = 0; c < C::CH; ++c) {
@@ -459,67 +392,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t ri = 0;  // ring entries issued, over all items
-      int nq_loads = 0;
-      bool go = true;
-      Item it;
-      for (int r = 0; go && fetch(r, it);) {
-        const int zq = it.b * p.Hq + it.hq;
-        const int zkv = it.b * p.Hkv + it.hkv;
-        if (nq_loads > 0 &&
-            !mbar_wait(&bars->q_empty, (nq_loads - 1) & 1, abort_flag, p.status))
-          break;
-        // Both Q slots; a split item's two warpgroups share one Q tile.
-        mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
-        for (int t = 0; t < 2; ++t)
-          for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
-                        it.row0 + (it.split ? 0 : t * BM), zq);
-        ++nq_loads;
-        int i = 0;  // ring entry of the item
-        // One ring entry: K (v = false) or V of KV tile kv.
-        auto emit = [&](bool v, int kv) {
-          const int slot = static_cast<int>(ri % C::NST);
-          const uint32_t round = ri / C::NST;
-          if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status))
-            return false;
-#ifdef EXATTN_TEST_WITHHOLD
-          // Test build only: stop before ring index EXATTN_TEST_WITHHOLD of
-          // the first item, arriving on nothing and copying nothing, so the
-          // consumers' waits run out.
-          if (nq_loads == 1 && i == EXATTN_TEST_WITHHOLD) return false;
-#endif
-          mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
-          const CUtensorMap *map = v ? &tm_v : &tm_k;
-          for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
-                        64 * c, kv * BN, zkv);
-          ++ri;
-          ++i;
-          return true;
-        };
-        if (!it.split) {
-          // K(jlo), then V(j) K(j+1) per KV tile j: both Q tiles use each.
-          for (int e = 0; go && e < 2 * (it.jhi - it.jlo); ++e)
-            go = emit(e & 1, it.jlo + (e >> 1));
-        } else {
-          // In the order the MMA issuer consumes them: K0(0) K1(0), then per
-          // step s: V0(s) K0(s+1) V1(s) K1(s+1) (tile t's KV tiles start at
-          // jlo and mid; the second half may be one tile shorter).
-          const int n0 = it.mid - it.jlo, n1 = it.jhi - it.mid;
-          go = emit(false, it.jlo) && emit(false, it.mid);
-          for (int st = 0; go && st < n0; ++st) {
-            go = emit(true, it.jlo + st);
-            if (go && st + 1 < n0) go = emit(false, it.jlo + st + 1);
-            if (go && st < n1) go = emit(true, it.mid + st);
-            if (go && st + 1 < n1) go = emit(false, it.mid + st + 1);
-          }
+      const int zq = b * p.Hq + hq;
+      const int zkv = b * p.Hkv + hkv;
+      // Both Q slots; a split CTA's two warpgroups share its one Q tile.
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
+                      row0 + (kSplit && split ? 0 : t * BM), zq);
+      // Ring entries in the order the MMA issuer consumes them.  Whole pair:
+      // K(jlo), then V(j) K(j+1) per KV tile j (both Q tiles use each).  Split:
+      // K0(0) K1(0), then per step s V0(s) K0(s+1) V1(s) K1(s+1), where tile 0
+      // walks the KV tiles from jlo and tile 1 from mid (one fewer, at most).
+      int sst = 0, sph = 0;  // split walk: step, and position within the step
+      auto entry = [&](int i, bool &v, int &kv) {
+        if (!split) {
+          v = (i & 1) != 0;
+          kv = jlo + (i >> 1);
+          return;
         }
+        if (i < 2) {
+          v = false;
+          kv = i == 0 ? jlo : mid;
+          return;
+        }
+        const int n0 = mid - jlo, n1 = jhi - mid;
+        while (true) {
+          const int st = sst, ph = sph;
+          if (++sph == 4) {
+            sph = 0;
+            ++sst;
+          }
+          if (ph == 0) { v = true; kv = jlo + st; return; }
+          if (ph == 1 && st + 1 < n0) { v = false; kv = jlo + st + 1; return; }
+          if (ph == 2 && st < n1) { v = true; kv = mid + st; return; }
+          if (ph == 3 && st + 1 < n1) { v = false; kv = mid + st + 1; return; }
+        }
+      };
+      int issued = 0;
+      for (int i = 0; i < 2 * (jhi - jlo); ++i) {
+        const int slot = i % C::NST;
+        const int round = i / C::NST;
+        if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status))
+          break;
+#ifdef EXATTN_TEST_WITHHOLD
+        // Test build only: stop before ring index EXATTN_TEST_WITHHOLD, arriving
+        // on nothing and copying nothing, so the consumers' waits run out.
+        if (i == EXATTN_TEST_WITHHOLD) break;
+#endif
+        mbar_arrive_expect_tx(&bars->full[slot], C::TILE_BYTES);
+        bool ev;
+        int kv;
+        entry(i, ev, kv);
+        const CUtensorMap *map = ev ? &tm_v : &tm_k;
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sRing + slot * C::TILE_BYTES + c * CHUNK_BYTES, map, &bars->full[slot],
+                      64 * c, kv * BN, zkv);
+        issued = i + 1;
       }
       // Drain: no copy may still be writing shared memory when the CTA exits.
       // Normally these phases completed long ago and each wait returns at once.
-      if (nq_loads > 0) mbar_wait_drain(&bars->q_full, (nq_loads - 1) & 1, p.status);
-      for (uint32_t i = ri > static_cast<uint32_t>(C::NST) ? ri - C::NST : 0; i < ri; ++i)
+      mbar_wait_drain(&bars->q_full, 0, p.status);
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
         mbar_wait_drain(&bars->full[i % C::NST], (i / C::NST) & 1, p.status);
     }
   } else if (warp == 1) {
@@ -528,6 +462,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t ring_base = smem_u32(sRing);
+      auto slot_of = [](int i) { return i % C::NST; };
+      auto wait_full = [&](int i) {
+        return mbar_wait(&bars->full[i % C::NST], (i / C::NST) & 1, abort_flag, p.status);
+      };
       // Descriptors are built once; per MMA only the start-address field moves
       // (smem addresses stay below 256 KB, so adding addr>>4 never carries out
       // of the 14-bit field).  This keeps the issuing thread's instruction
@@ -536,130 +474,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t kdesc0 = sdesc_sw128(ring_base, 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(ring_base, CHUNK_BYTES, 1024);
       const uint32_t idesc_qk = C::IDESC_QK, idesc_pv = C::IDESC_PV;
-      uint32_t base = 0;          // ring index of the current item's K(jlo)
-      uint32_t pcnt0 = 0, pcnt1 = 0;  // p_full phases consumed, per Q tile
-      uint32_t ecnt0 = 0, ecnt1 = 0;  // epilogues before the current item, per Q tile
-      int k = 0;                  // items so far
-      bool ok = true;
-      Item it;
-      for (int r = 0; ok && fetch(r, it); ++k) {
-        auto slot_of = [&](int i) { return static_cast<int>((base + i) % C::NST); };
-        auto wait_full = [&](int i) {
-          return mbar_wait(&bars->full[(base + i) % C::NST], ((base + i) / C::NST) & 1, abort_flag,
-                           p.status);
-        };
-        auto issue_s = [&](int t, int kidx) {  // S_t = Q_t K^T
-          const uint64_t qd = qdesc0 + ((t * C::TILE_BYTES) >> 4);
-          const uint64_t kd = kdesc0 + ((slot_of(kidx) * C::TILE_BYTES) >> 4);
-          const uint32_t d_tmem = tmem + t * 128;
+      auto issue_s = [&](int t, int kidx) {  // S_t = Q_t K^T
+        const uint64_t qd = qdesc0 + ((t * C::TILE_BYTES) >> 4);
+        const uint64_t kd = kdesc0 + ((slot_of(kidx) * C::TILE_BYTES) >> 4);
+        const uint32_t d_tmem = tmem + t * 128;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = ((ks >> 2) * CHUNK_BYTES + (ks & 3) * 32) >> 4;
-            mma_ss(d_tmem, qd + off, kd + off, idesc_qk, ks > 0);
-          }
-        };
-        auto issue_pv = [&](int t, int vidx, bool acc) {  // O_t (+)= P_t V
-          const uint64_t vd = vdesc0 + ((slot_of(vidx) * C::TILE_BYTES) >> 4);
-          const uint32_t d_tmem = tmem + 256 + t * 128, a_tmem = tmem + t * 128;
-#pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ts(d_tmem, a_tmem + ks * 8, vd + ((ks * 16 * 128) >> 4), idesc_pv,
-                   (acc || ks > 0) ? 1u : 0u);
-        };
-        // P_t(j) is in TMEM: wait for it; before the item's first PV of a Q
-        // tile (which overwrites O_t) also for that tile's previous epilogue.
-        auto wait_p = [&](int t, int j) {
-          if (t == 0) {
-            if (j == it.js0 && ecnt0 > 0 &&
-                !mbar_wait(&bars->o_empty[0], (ecnt0 - 1) & 1, abort_flag, p.status))
-              return false;
-            return mbar_wait(&bars->p_full[0], (pcnt0++) & 1, abort_flag, p.status);
-          }
-          if (j == it.js1 && ecnt1 > 0 &&
-              !mbar_wait(&bars->o_empty[1], (ecnt1 - 1) & 1, abort_flag, p.status))
-            return false;
-          return mbar_wait(&bars->p_full[1], (pcnt1++) & 1, abort_flag, p.status);
-        };
-        // K/V tile j of this item sits at ring index 2*(j - jlo) (K) and +1 (V).
-        auto has = [&](int t, int j) {
-          return t == 0 ? (j >= it.js0 && j < it.je0) : (j >= it.js1 && j < it.je1);
-        };
-        const int jlo = it.jlo, jhi = it.jhi;
-        ok = mbar_wait(&bars->q_full, k & 1, abort_flag, p.status);
-        ok = ok && wait_full(0);
-        if (!ok) break;
-        tc_fence_after();
-        if (it.split) {
-          // Split item: tile t walks its own half of the KV tiles, so each ring
-          // entry feeds one MMA group and is released right after it.  Entries
-          // come in the producer's order: K0(0) K1(0), then V0(s) K0(s+1) V1(s)
-          // K1(s+1) per step s.
-          const int n0 = it.mid - jlo, n1 = jhi - it.mid;
-          issue_s(0, 0);
-          tc_commit(&bars->s_full[0]);
-          tc_commit(&bars->empty[slot_of(0)]);
-          if (!(ok = wait_full(1))) break;
-          tc_fence_after();
-          issue_s(1, 1);
-          tc_commit(&bars->s_full[1]);
-          tc_commit(&bars->empty[slot_of(1)]);
-          if (n0 == 1) tc_commit(&bars->q_empty);  // no score MMA left on Q
-          int e = 2;
-          for (int st = 0; ok && st < n0; ++st) {
-            if (!(ok = wait_p(0, jlo + st) && wait_full(e))) break;
-            tc_fence_after();
-            issue_pv(0, e, st > 0);
-            tc_commit(&bars->o_full[0]);
-            tc_commit(&bars->empty[slot_of(e++)]);
-            if (st + 1 < n0) {
-              if (!(ok = wait_full(e))) break;
-              tc_fence_after();
-              issue_s(0, e);  // in order after PV0(st), which read P0 there
-              tc_commit(&bars->s_full[0]);
-              tc_commit(&bars->empty[slot_of(e++)]);
-            }
-            if (st < n1) {
-              if (!(ok = wait_p(1, it.mid + st) && wait_full(e))) break;
-              tc_fence_after();
-              issue_pv(1, e, st > 0);
-              tc_commit(&bars->o_full[1]);
-              tc_commit(&bars->empty[slot_of(e++)]);
-            }
-            if (st + 1 < n1) {
-              if (!(ok = wait_full(e))) break;
-              tc_fence_after();
-              issue_s(1, e);
-              tc_commit(&bars->s_full[1]);
-              tc_commit(&bars->empty[slot_of(e++)]);
-            }
-            if (st + 2 == n0) tc_commit(&bars->q_empty);  // the last score MMAs on Q
-          }
-          if (!ok) break;
-          base += 2 * (jhi - jlo);
-          ++ecnt0;
-          ++ecnt1;
-          continue;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = ((ks >> 2) * CHUNK_BYTES + (ks & 3) * 32) >> 4;
+          mma_ss(d_tmem, qd + off, kd + off, idesc_qk, ks > 0);
         }
-        // S0(jlo) and S1(jlo) overwrite the previous item's P tiles only after
-        // its last PVs, issued before them, have read them (in-order MMAs).
+      };
+      auto issue_pv = [&](int t, int vidx, bool acc) {  // O_t (+)= P_t V
+        const uint64_t vd = vdesc0 + ((slot_of(vidx) * C::TILE_BYTES) >> 4);
+        const uint32_t d_tmem = tmem + 256 + t * 128, a_tmem = tmem + t * 128;
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-          if (has(t, jlo)) {
-            issue_s(t, 0);
-            tc_commit(&bars->s_full[t]);
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(d_tmem, a_tmem + ks * 8, vd + ((ks * 16 * 128) >> 4), idesc_pv,
+                 (acc || ks > 0) ? 1u : 0u);
+      };
+
+      // K/V tile j of this CTA sits at ring index 2*(j - jlo) (K) and +1 (V).
+      auto has = [&](int t, int j) {
+        return t == 0 ? (j >= js0 && j < je0) : (j >= js1 && j < je1);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.status);
+      ok = ok && wait_full(0);
+      if (kSplit && split) {
+        // Split CTA: tile t walks its own half of the KV tiles, so each ring
+        // entry feeds one MMA group and is released right after it, in the
+        // producer's order: K0(0) K1(0), then V0(s) K0(s+1) V1(s) K1(s+1).
+        const int n0 = mid - jlo, n1 = jhi - mid;
+        int e = 0;
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, e);
+          tc_commit(&bars->s_full[0]);
+          tc_commit(&bars->empty[slot_of(e++)]);
+          ok = wait_full(e);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_s(1, e);
+          tc_commit(&bars->s_full[1]);
+          tc_commit(&bars->empty[slot_of(e++)]);
+        }
+        for (int st = 0; ok && st < n0; ++st) {
+          if (!(ok = mbar_wait(&bars->p_full[0], st & 1, abort_flag, p.status) && wait_full(e)))
+            break;
+          tc_fence_after();
+          issue_pv(0, e, st > 0);
+          tc_commit(&bars->o_full[0]);
+          tc_commit(&bars->empty[slot_of(e++)]);
+          if (st + 1 < n0) {
+            if (!(ok = wait_full(e))) break;
+            tc_fence_after();
+            issue_s(0, e);  // in order after PV0(st), which read P0 there
+            tc_commit(&bars->s_full[0]);
+            tc_commit(&bars->empty[slot_of(e++)]);
           }
-        tc_commit(&bars->empty[slot_of(0)]);
-        // Q may be replaced once the item's last score MMA has read it: the
-        // next item's Q then loads during this item's last KV step.
-        if (jhi - jlo == 1) tc_commit(&bars->q_empty);
+          if (st < n1) {
+            if (!(ok = mbar_wait(&bars->p_full[1], st & 1, abort_flag, p.status) && wait_full(e)))
+              break;
+            tc_fence_after();
+            issue_pv(1, e, st > 0);
+            tc_commit(&bars->o_full[1]);
+            tc_commit(&bars->empty[slot_of(e++)]);
+          }
+          if (st + 1 < n1) {
+            if (!(ok = wait_full(e))) break;
+            tc_fence_after();
+            issue_s(1, e);
+            tc_commit(&bars->s_full[1]);
+            tc_commit(&bars->empty[slot_of(e++)]);
+          }
+        }
+      } else {
+        if (ok) {
+          tc_fence_after();
+  #pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (has(t, jlo)) {
+              issue_s(t, 0);
+              tc_commit(&bars->s_full[t]);
+            }
+          tc_commit(&bars->empty[slot_of(0)]);
+        }
         for (int j = jlo; ok && j < jhi; ++j) {
           const int rj = j - jlo;
           bool v_ready = false;
           if (has(0, j)) {
-            if (!(ok = wait_p(0, j) && wait_full(2 * rj + 1))) break;
+            if (!(ok = mbar_wait(&bars->p_full[0], (j - js0) & 1, abort_flag, p.status) &&
+                       wait_full(2 * rj + 1)))
+              break;
             v_ready = true;
             tc_fence_after();
-            issue_pv(0, 2 * rj + 1, j > it.js0);
+            issue_pv(0, 2 * rj + 1, j > js0);
             tc_commit(&bars->o_full[0]);
           }
           if (j + 1 < jhi && !(ok = wait_full(2 * rj + 2))) break;
@@ -671,10 +580,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_commit(&bars->s_full[0]);
           }
           if (has(1, j)) {
-            if (!(ok = wait_p(1, j))) break;
+            if (!(ok = mbar_wait(&bars->p_full[1], (j - js1) & 1, abort_flag, p.status))) break;
             if (!v_ready && !(ok = wait_full(2 * rj + 1))) break;
             tc_fence_after();
-            issue_pv(1, 2 * rj + 1, j > it.js1);
+            issue_pv(1, 2 * rj + 1, j > js1);
             tc_commit(&bars->o_full[1]);
           }
           tc_commit(&bars->empty[slot_of(2 * rj + 1)]);  // V(j) no longer needed
@@ -683,12 +592,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_commit(&bars->s_full[1]);
           }
           if (j + 1 < jhi) tc_commit(&bars->empty[slot_of(2 * rj + 2)]);  // K(j+1) done
-          if (j + 2 == jhi) tc_commit(&bars->q_empty);  // S(jhi-1) was the last on Q
         }
-        if (!ok) break;
-        base += 2 * (jhi - jlo);
-        if (it.je0 > it.js0) ++ecnt0;
-        if (it.je1 > it.js1) ++ecnt1;
       }
       // Every MMA issued above must finish before TMEM is released.
       tc_commit(&bars->mma_done);
@@ -701,182 +605,169 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     regs_inc<kRegsHigh>();
     const int t = (warp - 4) >> 2;        // Q tile of this warpgroup
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
-    const int rr = quarter * 32 + lane;   // row within the Q tile
+    const int r = quarter * 32 + lane;    // row within the Q tile
+    // (In a split CTA both warpgroups hold the rows of its one Q tile.)
+    const int row = row0 + (kSplit && split ? 0 : t * BM) + r;
+    const int jst = t == 0 ? js0 : js1, jen = t == 0 ? je0 : je1;
+    const int nt = jen - jst;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + t * 128;
     const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
     const float c = p.scale_log2;
-    uint32_t scnt = 0;  // s_full phases consumed (score tiles of this Q tile, all items)
-    uint32_t ocnt = 0;  // o_full phases (PVs of this Q tile, all items)
-    uint32_t mcnt = 0;  // split items merged (warpgroup 0)
-    float2 *xfer = reinterpret_cast<float2 *>(smem + C::XFER_OFF);
+    // ALiBi slope in log2 units; the bias slope * (key - query) joins the score
+    // before the row max.
+    const float slope2 = kAlibi ? p.slopes[hq] * 1.4426950408889634f : 0.f;
+    float m = -INFINITY;  // reference max, in log2 units of scaled scores
+    float l = 0.f;
     bool ok = true;
-    Item it;
-    for (int r = 0; ok && fetch(r, it);) {
-      // (In a split item both warpgroups hold the same rows.)
-      const int row = it.row0 + (it.split ? 0 : t * BM) + rr;
-      const int jst = t == 0 ? it.js0 : it.js1, jen = t == 0 ? it.je0 : it.je1;
-      const int nt = jen - jst;
-      const int nk = it.nk, nq = it.nq, ctx = it.ctx;
-      // ALiBi slope in log2 units; the bias slope * (key - query) joins the score
-      // before the row max.
-      const float slope2 = kAlibi ? p.slopes[it.hq] * 1.4426950408889634f : 0.f;
-      float m = -INFINITY;  // reference max, in log2 units of scaled scores
-      float l = 0.f;
-      for (int j = jst; j < jen; ++j) {
-        ok = mbar_wait(&bars->s_full[t], (scnt++) & 1, abort_flag, p.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        // Visible columns [lo, hi) of this row in KV tile j: the end of the keys,
-        // the causal diagonal and the sliding window.
-        int hi = min(BN, nk - j * BN);
-        if (p.causal) hi = min(hi, ctx + row - j * BN + 1);
-        // (Rows past the last take the last real row's window so that they never
-        // force the masked path on a warp whose real rows need none.)
-        const int lo = p.window > 0 ? ctx + min(row, nq - 1) - p.window + 1 - j * BN : 0;
-        // The whole 128-column score row of this thread, in one TMEM load.
-        uint32_t sv[128];
-        tmem_ld128(s_addr, sv);
-        tmem_ld_wait128(sv);
-        float cx = c;  // factor still to apply to sv in the exponent
-        if (kAlibi) {
-          const float rb = slope2 * static_cast<float>(j * BN - (ctx + row));
-          const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2), rb2 = make_float2(rb, rb);
-#pragma unroll
-          for (int i = 0; i < 128; i += 2) {
-            const float2 bias = fma2(sl2, make_float2(static_cast<float>(i), static_cast<float>(i + 1)), rb2);
-            const float2 x = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, bias);
-            sv[i] = __float_as_uint(x.x);
-            sv[i + 1] = __float_as_uint(x.y);
-          }
-          cx = 1.0f;
-        }
-        // Only diagonal, window-edge and last tiles carry masked columns;
-        // elsewhere the warp takes the branch-free path.
-        const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= BN);
-        if (masked) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i < lo || i >= hi) sv[i] = 0xff800000u;  // -inf
-        }
-        float mx;
-        {
-          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 128; i += 8) {
-            m0 = fmax3(m0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
-            m1 = fmax3(m1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
-            m2 = fmax3(m2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
-            m3 = fmax3(m3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
-          }
-          mx = fmax3(m0, m1, fmaxf(m2, m3));
-        }
-        const float m_new = fmaxf(m, mx * cx);
-        const bool resc = m_new > m + 8.0f;
-        const float alpha = resc ? ex2(m - m_new) : 1.0f;
-        if (resc) m = m_new;
-        l *= alpha;
-        // A row that has seen no visible key yet (a window edge) keeps m = -inf;
-        // its masked scores must still give P = 0, not -inf - (-inf).
-        const float m_use = (m == -INFINITY) ? 0.f : m;
-        // P = 2^(s*c - m), rounded to bf16 and written over the (already read) S
-        // columns; the row sum stays in fp32.  Unmasked tiles compute one pair in
-        // four with the FMA-pipe polynomial to unload the special-function unit.
-        if (masked)
-          l += exp_row<false>(sv, cx, m_use, s_addr);
-        else
-          l += exp_row<true>(sv, cx, m_use, s_addr);
-        if (j > jst && __any_sync(0xffffffffu, resc)) {
-          // Lazy rescale of O (rare once the max settles).  O is stable here:
-          // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(o_addr + cc * 32, ov);
-            tmem_ld_wait(ov);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(o_addr + cc * 32, ov);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[t]);
-      }
-      if (!ok || nt <= 0) continue;
-      // The item's last PV: S(jen-1) completing implied PV(jen-2) completed, so
-      // o_full is at most one phase behind this wait.
-      ocnt += nt;
-      ok = mbar_wait(&bars->o_full[t], (ocnt - 1) & 1, abort_flag, p.status);
+    for (int j = jst; j < jen; ++j) {
+      ok = mbar_wait(&bars->s_full[t], (j - jst) & 1, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      if (it.split && t == 1) {
-        // Warpgroup 0 merges: it reads this O tile from TMEM itself (any
-        // warpgroup may address any column of its lane quarter), and m, l here.
-        xfer[rr] = make_float2(m, l);
+      // Visible columns [lo, hi) of this row in KV tile j: the end of the keys,
+      // the causal diagonal and the sliding window.
+      int hi = min(BN, nk - j * BN);
+      if (p.causal) hi = min(hi, ctx + row - j * BN + 1);
+      // (Rows past the last take the last real row's window so that they never
+      // force the masked path on a warp whose real rows need none.)
+      const int lo = p.window > 0 ? ctx + min(row, nq - 1) - p.window + 1 - j * BN : 0;
+      // The whole 128-column score row of this thread, in one TMEM load.
+      uint32_t sv[128];
+      tmem_ld128(s_addr, sv);
+      tmem_ld_wait128(sv);
+      float cx = c;  // factor still to apply to sv in the exponent
+      if (kAlibi) {
+        const float rb = slope2 * static_cast<float>(j * BN - (ctx + row));
+        const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2), rb2 = make_float2(rb, rb);
+#pragma unroll
+        for (int i = 0; i < 128; i += 2) {
+          const float2 bias = fma2(sl2, make_float2(static_cast<float>(i), static_cast<float>(i + 1)), rb2);
+          const float2 x = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, bias);
+          sv[i] = __float_as_uint(x.x);
+          sv[i + 1] = __float_as_uint(x.y);
+        }
+        cx = 1.0f;
+      }
+      // Only diagonal, window-edge and last tiles carry masked columns;
+      // elsewhere the warp takes the branch-free path.
+      const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= BN);
+      if (masked) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i < lo || i >= hi) sv[i] = 0xff800000u;  // -inf
+      }
+      float mx;
+      {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 8) {
+          m0 = fmax3(m0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          m1 = fmax3(m1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
+          m2 = fmax3(m2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
+          m3 = fmax3(m3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
+        }
+        mx = fmax3(m0, m1, fmaxf(m2, m3));
+      }
+      const float m_new = fmaxf(m, mx * cx);
+      const bool resc = m_new > m + 8.0f;
+      const float alpha = resc ? ex2(m - m_new) : 1.0f;
+      if (resc) m = m_new;
+      l *= alpha;
+      // A row that has seen no visible key yet (a window edge) keeps m = -inf;
+      // its masked scores must still give P = 0, not -inf - (-inf).
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      // P = 2^(s*c - m), rounded to bf16 and written over the (already read) S
+      // columns; the row sum stays in fp32.  Unmasked tiles compute one pair in
+      // four with the FMA-pipe polynomial to unload the special-function unit.
+      if (masked)
+        l += exp_row<false>(sv, cx, m_use, s_addr);
+      else
+        l += exp_row<true>(sv, cx, m_use, s_addr);
+      if (j > jst && __any_sync(0xffffffffu, resc)) {
+        // Lazy rescale of O (rare once the max settles).  O is stable here:
+        // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+          tmem_ld_wait(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(o_addr + cc * 32, ov);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[t]);
+    }
+    if (ok && nt > 0) {
+      ok = mbar_wait(&bars->o_full[t], (nt - 1) & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (kSplit && ok && split && t == 1) {
+        // Warpgroup 0 merges: it reads this O tile from TMEM itself (a warp may
+        // address every column of its lane quarter), and m, l from here.
+        reinterpret_cast<float2 *>(smem + C::XFER_OFF)[r] = make_float2(m, l);
         tc_fence_before();
         mbar_arrive(&bars->mrg_full);
-        continue;  // warpgroup 0 releases O1 (o_empty[1]) once it has read it
+        ok = false;  // nothing more for this warpgroup
       }
-      float a0 = 1.f, a1 = 0.f;  // weights of this O tile and (split) of O1
-      if (it.split) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->mrg_full, (mcnt++) & 1, abort_flag, p.status));
-        if (!ok) break;
+      float a0 = 1.f, a1 = 0.f;  // weights of this O tile and (split) of the other
+      if (kSplit && ok && split) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->mrg_full, 0, abort_flag, p.status));
+        if (ok) {
+          tc_fence_after();
+          // Two partial results of one row over disjoint keys: the joint max
+          // and sum, each accumulator weighted by 2^(its reference - the joint).
+          const float2 ml1 = reinterpret_cast<const float2 *>(smem + C::XFER_OFF)[r];
+          const float mm = fmaxf(m, ml1.x);
+          a0 = ex2(m - mm);
+          a1 = ex2(ml1.x - mm);
+          l = a0 * l + a1 * ml1.y;
+          m = mm;
+        }
+      }
+      if (ok) {
         tc_fence_after();
-        // Two partial results of one row over disjoint keys: the joint max and
-        // sum, and each accumulator weighted by 2^(its reference - the joint one).
-        const float2 ml1 = xfer[rr];
-        const float mm = fmaxf(m, ml1.x);
-        a0 = ex2(m - mm);
-        a1 = ex2(ml1.x - mm);
-        l = a0 * l + a1 * ml1.y;
-        m = mm;
-      }
-      const float inv_l = 1.0f / l;
-      a0 *= inv_l;
-      a1 *= inv_l;
-      const uint32_t o1_addr = tmem + lane_off + 256 + 128;
-      const bool valid = row < nq;
-      // Row of O and L: [B][Hq][N] for self-attention, [T][Hq] for a chunk.
-      const size_t orow_idx =
-          kPaged ? static_cast<size_t>(it.qrow0 + (valid ? row : 0)) * p.Hq + it.hq
-                 : (static_cast<size_t>(it.b) * p.Hq + it.hq) * p.N + (valid ? row : 0);
-      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + orow_idx * D;
+        const float inv_l = 1.0f / l;
+        a0 *= inv_l;
+        a1 *= inv_l;
+        const uint32_t o1_addr = tmem + lane_off + 256 + 128;
+        const bool valid = row < nq;
+        // Row of O and L: [B][Hq][N] for self-attention, [T][Hq] for a chunk.
+        const size_t orow_idx =
+            kPaged ? static_cast<size_t>(qrow0 + (valid ? row : 0)) * p.Hq + hq
+                   : (static_cast<size_t>(b) * p.Hq + hq) * p.N + (valid ? row : 0);
+        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + orow_idx * D;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(o_addr + cc * 32, ov);
-        tmem_ld_wait(ov);
-        uint32_t pk[16];
-        if (it.split) {
-          uint32_t ov1[32];
-          tmem_ld32(o1_addr + cc * 32, ov1);
-          tmem_ld_wait(ov1);
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+          tmem_ld_wait(ov);
+          uint32_t pk[16];
+          if (kSplit && split) {
+            uint32_t ov1[32];
+            tmem_ld32(o1_addr + cc * 32, ov1);
+            tmem_ld_wait(ov1);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            pk[i >> 1] = pack_bf16x2(
-                fmaf(__uint_as_float(ov[i]), a0, __uint_as_float(ov1[i]) * a1),
-                fmaf(__uint_as_float(ov[i + 1]), a0, __uint_as_float(ov1[i + 1]) * a1));
-        } else {
+            for (int i = 0; i < 32; i += 2)
+              pk[i >> 1] = pack_bf16x2(
+                  fmaf(__uint_as_float(ov[i]), a0, __uint_as_float(ov1[i]) * a1),
+                  fmaf(__uint_as_float(ov[i + 1]), a0, __uint_as_float(ov1[i + 1]) * a1));
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            pk[i >> 1] = pack_bf16x2(__uint_as_float(ov[i]) * a0, __uint_as_float(ov[i + 1]) * a0);
+            for (int i = 0; i < 32; i += 2)
+              pk[i >> 1] = pack_bf16x2(__uint_as_float(ov[i]) * a0, __uint_as_float(ov[i + 1]) * a0);
+          }
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
         }
-        if (valid) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
+        if (valid) p.lse[orow_idx] = (m + log2f(l)) * 0.6931471805599453f;
       }
-      if (valid) p.lse[orow_idx] = (m + log2f(l)) * 0.6931471805599453f;
-      // O_t (and in a split item O1) is read: the next item's first PV of the
-      // tile may overwrite it.
-      tc_fence_before();
-      mbar_arrive(&bars->o_empty[t]);
-      if (it.split) mbar_arrive(&bars->o_empty[1]);
     }
   }
 
@@ -887,6 +778,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // A split grid may run beside the whole-pair grid ahead of it; it does not
+  // finish before that grid has, so work behind it in the stream sees both.
+  if constexpr (kSplit) grid_dependency_wait();
 }
 
 // --------------------------------------------------------------- host side
@@ -954,23 +848,40 @@ bool make_tok_map(CUtensorMap *map, const void *base, int D, int Hq, int T) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool kAlibi, bool kPaged>
+template <int D, bool kAlibi, bool kPaged, bool kSplit>
 attn_status_t launch_kernel(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                             const CUtensorMap &mk1, const CUtensorMap &mv1, const Params &prm,
-                            long long ctas, cudaStream_t stream) {
+                            long long ctas, cudaStream_t stream, bool dependent = false) {
   using C = Cfg<D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D, kAlibi, kPaged>,
+    attr_err = cudaFuncSetAttribute(prefill_bf16_kernel<D, kAlibi, kPaged, kSplit>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
   if (ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   if (ctas == 0) return ATTN_OK;
-  prefill_bf16_kernel<D, kAlibi, kPaged>
-      <<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mk1, mv1,
-                                                                             prm);
+  if (!dependent) {
+    prefill_bf16_kernel<D, kAlibi, kPaged, kSplit>
+        <<<static_cast<unsigned>(ctas), NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mk1,
+                                                                               mv1, prm);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  // Programmatic dependent launch behind the grid before it in the stream.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, prefill_bf16_kernel<D, kAlibi, kPaged, kSplit>, mq, mk, mv, mk1,
+                         mv1, prm) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -1000,25 +911,30 @@ attn_status_t launch(const void *q, const void *k, const void *v, void *o, float
   if (!make_map(&mq, q, D, N, B * Hq) || !make_map(&mk, k, D, N, B * Hkv) ||
       !make_map(&mv, v, D, N, B * Hkv))
     return ATTN_ERR_CUDA;
+  if (window >= N) window = 0;  // a window of N or more keys is plain causal attention
   Params prm = base_params(o, lse, status, B, Hq, Hkv, N, scale, causal, window, slopes);
   const long long pairs = static_cast<long long>(prm.pairs) * B * Hq;
   if (pairs > 0x3fffffffLL) return ATTN_ERR_INVALID_ARG;
-  // Persistent CTAs: one per SM (the kernel holds all of an SM's tensor
-  // memory), each walking its share of the items.
+  // The pairs of the last, partial wave (all of them when there are fewer
+  // pairs than SMs) run as two split CTAs each -- one Q tile, its KV range
+  // halved over the two softmax warpgroups -- when the split CTAs fit in one
+  // wave: that wave then takes about half as long.  They are a second grid of
+  // the split variant, launched as a programmatic dependent of the whole
+  // pairs' grid, so the whole-pair kernel carries none of the split code.
+  // Not with a sliding window, whose halves could leave a row without a
+  // visible key.
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return ATTN_ERR_CUDA;
-  // The pairs of a last, partial round (all of them when there are fewer
-  // pairs than SMs) run as two split items each -- one Q tile, its KV range
-  // halved over the two warpgroups -- when the split items fit in one round:
-  // that round then takes about half as long.  Not with a sliding window,
-  // whose halves could leave a row without a visible key.
   const long long rem = pairs % sms;
-  prm.split_pairs = (window == 0 && rem > 0 && 2 * rem <= sms) ? static_cast<int>(rem) : 0;
-  const long long items = pairs + prm.split_pairs;
-  return launch_kernel<D, kAlibi, false>(mq, mk, mv, mk, mv, prm, items < sms ? items : sms,
-                                         stream);
+  const long long split_pairs = (window == 0 && rem > 0 && 2 * rem <= sms) ? rem : 0;
+  prm.whole_pairs = static_cast<int>(pairs - split_pairs);
+  attn_status_t st = launch_kernel<D, kAlibi, false, false>(mq, mk, mv, mk, mv, prm,
+                                                            prm.whole_pairs, stream);
+  if (st != ATTN_OK || split_pairs == 0) return st;
+  return launch_kernel<D, kAlibi, false, true>(mq, mk, mv, mk, mv, prm, 2 * split_pairs, stream,
+                                               prm.whole_pairs > 0);
 }
 
 template <int D, bool kAlibi>
@@ -1041,7 +957,7 @@ attn_status_t launch_paged(const void *q, const void *k_pages, const void *v_pag
   prm.num_pages = num_pages;
   prm.T = T;
   const long long ctas = static_cast<long long>(prm.pairs) * S * Hq;
-  return launch_kernel<D, kAlibi, true>(mq, mk, mv, mk1, mv1, prm, ctas, stream);
+  return launch_kernel<D, kAlibi, true, false>(mq, mk, mv, mk1, mv1, prm, ctas, stream);
 }
 
 }  // namespace
