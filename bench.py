@@ -528,7 +528,7 @@ def run_ours(args):
                 "frac": big_tf / peak_tf,
                 "traffic": profiled_traffic("prefill_bf16_mha_n8192.md", "prefill_sm100.cu"),
                 "peak_source": peak_kind + " bf16_tflops (burst)",
-                "kernel": "prefill_bf16_kernel<128>, %s launch (%.0f%% of the step)"
+                "kernel": "prefill_bf16_kernel<128, 0, 0, 0> (whole pairs), %s launch (%.0f%% of the step)"
                           % (sweep[big].cfg.name, 100.0 * sum(times[big]) / sum(sum(t) for t in times)),
                 "algorithmic": "4*B*H*N^2*d = %.4g FLOP per launch; %d bytes (Q,K,V read, O,L written)"
                                % (sweep[big].cfg.flops, sweep[big].cfg.bytes),
