@@ -64,6 +64,62 @@ def test_bf16_small_shapes(B, Hq, Hkv, N, d, causal):
     assert ea.device_status() == 0
 
 
+# Which grid a launch uses depends on its count of 256-row Q-tile pairs
+# (B * Hq * ceil(N / 256)) against the SM count: pairs that do not fill the
+# last wave, when they are at most half the SMs and no window is set, run as
+# two split CTAs each (one Q tile, its KV range halved over the two softmax
+# warpgroups) in a second grid behind the whole pairs.  The SMALL shapes above
+# all have at most 74 pairs, so on a 148-SM part they run split CTAs only.
+# These shapes reach the other two cases: whole pairs only, and a full wave of
+# whole pairs plus split CTAs for the rest.
+GRID_CASES = [
+    # label, B, Hq, Hkv, N, d, causal, alibi
+    ("whole", 1, 24, 6, 1100, 128, True, False),     # GQA, ragged last tile
+    ("whole", 2, 12, 1, 900, 64, False, False),      # MQA, d = 64
+    ("mixed", 1, 40, 8, 1000, 128, True, False),     # GQA causal
+    ("mixed", 1, 32, 32, 1200, 128, True, True),     # ALiBi causal
+    ("mixed", 2, 16, 4, 1280, 64, False, False),     # d = 64 non-causal
+]
+
+
+def grid_kind(B, Hq, N, sms, window=0):
+    pairs = B * Hq * ((N + 255) // 256)
+    rem = pairs % sms
+    split = window == 0 and rem > 0 and 2 * rem <= sms
+    if not split:
+        return "whole"
+    return "split" if pairs < sms else "mixed"
+
+
+@pytest.mark.parametrize("label,B,Hq,Hkv,N,d,causal,alibi", GRID_CASES)
+def test_bf16_whole_and_mixed_grids(label, B, Hq, Hkv, N, d, causal, alibi):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if grid_kind(B, Hq, N, sms) != label:
+        pytest.skip("this shape takes another grid on a %d-SM device" % sms)
+    q, k, v = syn.random_qkv(B, Hq, Hkv, N, d, seed=500 + N + d + Hq)
+    scale = 1.0 / math.sqrt(d)
+    sl = slopes_for(Hq) if alibi else None
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=scale, causal=causal,
+                                    alibi_slopes=None if sl is None else sl.numpy())
+    out = torch.full_like(q, float("nan"), device=DEV)
+    lse = torch.full((B, Hq, N), float("nan"), device=DEV)
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale, out=out,
+                       lse=lse, alibi_slopes=None if sl is None else sl.to(DEV))
+    torch.cuda.synchronize()
+    assert_bf16_parity(o, l, o_ref, l_ref, (label, B, Hq, Hkv, N, d, causal, alibi))
+    assert ea.device_status() == 0
+
+
+def test_grid_kinds_of_the_shapes():
+    # On a 148-SM B200 every GRID_CASES shape takes the grid its label names,
+    # and the SMALL shapes take split CTAs only.
+    for label, B, Hq, _, N, _, _, _ in GRID_CASES:
+        assert grid_kind(B, Hq, N, 148) == label
+    for B, Hq, _, N, _, _ in SMALL:
+        assert grid_kind(B, Hq, N, 148) == "split"
+
+
 def test_bf16_deterministic_and_gqa_equals_repeated_heads():
     B, Hq, Hkv, N, d = 2, 8, 2, 700, 128
     q, k, v = (t.to(DEV) for t in syn.random_qkv(B, Hq, Hkv, N, d, seed=7))
