@@ -35,6 +35,9 @@
  *  - The library looks up a few device addresses once per device and keeps
  *    them; it does not support cudaDeviceReset (or a reset of the primary
  *    context) while it is loaded.
+ *  - Every compute call may be captured into a CUDA graph once the same
+ *    entry point has run eagerly on the device (its one-time setup happens
+ *    then); the two status reads may not.
  *  - `causal` means key j is visible to query i iff j <= i (queries and keys
  *    share positions 0..N-1).
  *  - L is the natural logarithm of sum_j exp(scale * q_i . k_j) over the
