@@ -50,6 +50,8 @@ CASES = [
     (1, 4, 4, 256, 128, False, 0, False),
     (1, 2, 1, 390, 128, True, 100, False),
     (1, 2, 2, 300, 64, True, 0, True),
+    (1, 8, 2, 1000, 128, True, 257, True),   # GQA with a window and ALiBi together
+    (2, 6, 3, 700, 64, False, 0, True),      # group of 2, ALiBi without a mask
     (1, 4, 2, 257, 128, True, 64, True),
 ]
 

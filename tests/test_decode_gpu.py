@@ -65,6 +65,8 @@ CASES = [
     ([300, 5], 8, 1, 128),          # MQA: 8 heads share one K/V head
     ([1025, 96], 32, 1, 64),        # MQA with 32 query heads
     ([250, 17, 48], 6, 2, 128),     # group of 3
+    ([700, 33], 32, 16, 128),       # 16 K/V heads: two groups of 8 per CTA grid
+    ([400, 1500], 32, 2, 128),      # group of 16: two chunks of 8 query heads
 ]
 
 

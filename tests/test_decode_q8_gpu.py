@@ -69,6 +69,8 @@ CASES = [
     ([250, 17, 48], 6, 2, 128),     # group of 3
     ([129, 40], 16, 8, 64),         # group of 2
     ([1023, 1024, 1025, 2049], 16, 4, 128),  # around the 1024-token chunk boundary
+    ([700, 33], 32, 16, 128),       # 16 K/V heads: two groups of 8 per CTA grid
+    ([400, 1500], 32, 2, 128),      # group of 16: two chunks of 8 query heads
 ]
 
 
