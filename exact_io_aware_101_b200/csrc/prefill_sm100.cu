@@ -104,32 +104,49 @@ struct Params {
   int max_blocks, num_pages, T;
 };
 
-// One thread's 128-column score row -> P (bf16 pairs in TMEM at s_addr) and
-// the row sum of P.  x = s*c - m is one packed FMA per pair; with kEmu, pairs
-// 3, 7, 11, ... use the polynomial 2^x, the rest the special-function unit.
-template <bool kEmu>
+// Columns cc*32 .. cc*32+31 of one thread's score row -> 16 bf16 pairs of P
+// and their part of the row sum: x = s*c - m is one packed FMA per pair, 2^x
+// one special-function op per column.  That 2^x is +inf from x = 128 up and
+// NaN for a NaN x, so a sum stays finite only when every term is right.
+__device__ __forceinline__ void exp_chunk(const uint32_t (&sv)[128], int cc, float2 c2, float2 nm2,
+                                          uint32_t *pk, float2 &sum_a, float2 &sum_b) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const int col = cc * 32 + i;
+    const float2 x0 = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), c2, nm2);
+    const float2 x1 = fma2(make_float2(__uint_as_float(sv[col + 2]), __uint_as_float(sv[col + 3])), c2, nm2);
+    const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+    const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+    sum_a = add2(sum_a, p0);
+    sum_b = add2(sum_b, p1);
+    pk[i >> 1] = pack_bf16x2(p0.x, p0.y);
+    pk[(i >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+  }
+}
+
+// One thread's 128-column score row -> P (bf16 pairs in TMEM at s_addr, over
+// the first 64 of the row's S columns) and the row sum of P.
 __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float c, float m,
                                          uint32_t s_addr) {
-  const float2 c2 = make_float2(c, c);
-  const float2 nm2 = make_float2(-m, -m);
+  const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
   float2 sum_a = make_float2(0.f, 0.f), sum_b = make_float2(0.f, 0.f);
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      const int col = cc * 32 + i;
-      const float2 x0 = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), c2, nm2);
-      const float2 x1 = fma2(make_float2(__uint_as_float(sv[col + 2]), __uint_as_float(sv[col + 3])), c2, nm2);
-      const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
-      const float2 p1 = (kEmu && (col & 4)) ? exp2_poly2(x1) : make_float2(ex2(x1.x), ex2(x1.y));
-      sum_a = add2(sum_a, p0);
-      sum_b = add2(sum_b, p1);
-      pk[i >> 1] = pack_bf16x2(p0.x, p0.y);
-      pk[(i >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
-    }
+    exp_chunk(sv, cc, c2, nm2, pk, sum_a, sum_b);
     tmem_st16(s_addr + cc * 16, pk);
   }
+  return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
+}
+
+// The same P and row sum kept in registers: TMEM, and with it the S row, is
+// left untouched.
+__device__ __forceinline__ float exp_row_held(const uint32_t (&sv)[128], float c, float m,
+                                              uint32_t (&pk)[64]) {
+  const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
+  float2 sum_a = make_float2(0.f, 0.f), sum_b = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) exp_chunk(sv, cc, c2, nm2, pk + cc * 16, sum_a, sum_b);
   return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
 }
 
@@ -657,44 +674,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = 0; i < 128; ++i)
           if (i < lo || i >= hi) sv[i] = 0xff800000u;  // -inf
       }
-      float mx;
-      {
-        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+      // Once every row of the warp has a finite reference max, an unmasked tile
+      // first computes P against that max without looking for the tile's own
+      // max.  If every row's P sums to at most 255, every x = s*c - m is below
+      // 8 and no term overflowed: m stays the reference (the max-first step
+      // below would keep it too, as it moves m only past m + 8), and P and
+      // its sum are written to TMEM and l as they stand.  Otherwise the S row
+      // is read back from TMEM, which the attempt left untouched, and the tile
+      // takes the max-first step, which then also moves a row that missed up
+      // to its running max, so that a max left low by a window's first tile
+      // does not miss again.  Masked and ALiBi tiles take the max-first step
+      // at once: their scores in registers are no longer those in TMEM (and
+      // ALiBi's rise along the row, so the attempt would miss most tiles).
+      bool fast = false, missed = false;
+      if (!kAlibi && !masked && j > jst && __all_sync(0xffffffffu, m != -INFINITY)) {
+        uint32_t pk[64];
+        const float l_tile = exp_row_held(sv, cx, m, pk);
+        missed = !(l_tile <= 255.0f);
+        fast = !__any_sync(0xffffffffu, missed);
+        if (fast) {
+          l += l_tile;
 #pragma unroll
-        for (int i = 0; i < 128; i += 8) {
-          m0 = fmax3(m0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
-          m1 = fmax3(m1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
-          m2 = fmax3(m2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
-          m3 = fmax3(m3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
+          for (int cc = 0; cc < 4; ++cc)
+            tmem_st16(s_addr + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + cc * 16));
+          // The step below is skipped on this path: tell the compiler that the
+          // scores are dead here, so that it keeps no copy of them alive across
+          // the exponentials above.
+#pragma unroll
+          for (int i = 0; i < 128; ++i) asm("" : "=r"(sv[i]));
+        } else {
+          tmem_ld128(s_addr, sv);
+          tmem_ld_wait128(sv);
         }
-        mx = fmax3(m0, m1, fmaxf(m2, m3));
       }
-      const float m_new = fmaxf(m, mx * cx);
-      const bool resc = m_new > m + 8.0f;
-      const float alpha = resc ? ex2(m - m_new) : 1.0f;
-      if (resc) m = m_new;
-      l *= alpha;
-      // A row that has seen no visible key yet (a window edge) keeps m = -inf;
-      // its masked scores must still give P = 0, not -inf - (-inf).
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      // P = 2^(s*c - m), rounded to bf16 and written over the (already read) S
-      // columns; the row sum stays in fp32.  Unmasked tiles compute one pair in
-      // four with the FMA-pipe polynomial to unload the special-function unit.
-      if (masked)
-        l += exp_row<false>(sv, cx, m_use, s_addr);
-      else
-        l += exp_row<true>(sv, cx, m_use, s_addr);
-      if (j > jst && __any_sync(0xffffffffu, resc)) {
-        // Lazy rescale of O (rare once the max settles).  O is stable here:
-        // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
+      if (!fast) {
+        float mx;
+        {
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t ov[32];
-          tmem_ld32(o_addr + cc * 32, ov);
-          tmem_ld_wait(ov);
+          for (int i = 0; i < 128; i += 8) {
+            m0 = fmax3(m0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+            m1 = fmax3(m1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
+            m2 = fmax3(m2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
+            m3 = fmax3(m3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
+          }
+          mx = fmax3(m0, m1, fmaxf(m2, m3));
+        }
+        const float m_new = fmaxf(m, mx * cx);
+        const bool resc = m_new > m + 8.0f || (missed && m_new > m);
+        const float alpha = resc ? ex2(m - m_new) : 1.0f;
+        if (resc) m = m_new;
+        l *= alpha;
+        // A row that has seen no visible key yet (a window edge) keeps m = -inf;
+        // its masked scores must still give P = 0, not -inf - (-inf).
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+        // P = 2^(s*c - m), rounded to bf16 and written over the (already read) S
+        // columns; the row sum stays in fp32.
+        l += exp_row(sv, cx, m_use, s_addr);
+        if (j > jst && __any_sync(0xffffffffu, resc)) {
+          // Lazy rescale of O (rare once the max settles).  O is stable here:
+          // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(o_addr + cc * 32, ov);
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t ov[32];
+            tmem_ld32(o_addr + cc * 32, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(o_addr + cc * 32, ov);
+          }
         }
       }
       tmem_st_wait();

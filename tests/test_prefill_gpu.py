@@ -152,6 +152,40 @@ def test_bf16_large_scores_stay_finite(causal, d):
     assert np.abs(f32(o) - o_ref).max() <= 2e-2
 
 
+# An unmasked tile after the first may compute P against the running max
+# before it looks for the tile's own max, and keeps that P only when every
+# row's sum stays at most 255.  One key here scores far above every earlier
+# key for every query (all queries positive, that key constant): its x = s*c - m
+# lands just above 8, near 50, or near 200, in a column that goes to the
+# special-function exp2 (column 0 of a group of 8) or to the polynomial one
+# (column 6), whose exponent field would wrap above 128.  Each must fall back to
+# the max-first step and match the oracle.
+@pytest.mark.parametrize("col,a,causal", [(46, 16.0, False), (46, 16.0, True), (46, 4.0, False),
+                                          (46, 0.75, False), (40, 16.0, False), (47, 1.0, True)])
+def test_bf16_score_jump_after_the_first_tile(col, a, causal):
+    B, H, N, d = 1, 2, 640, 128
+    g = torch.Generator().manual_seed(1234)
+    q = torch.randn(B, H, N, d, generator=g).abs().to(torch.bfloat16)
+    k = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    J = 256 + col  # third KV tile
+    k[:, :, J, :] = a
+    scale = 1.0 / math.sqrt(d)
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=scale, causal=causal)
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    # The jump in log2 units over the best earlier key, for the rows that see J.
+    s = np.einsum("bhnd,bhkd->bhnk", q.double().numpy(), k.double().numpy()) * scale / math.log(2)
+    jump = s[:, :, J:, J] - s[:, :, J:, :J].max(-1)
+    assert jump.min() > {16.0: 150, 4.0: 30, 1.0: 5, 0.75: 2}[a]
+    # l_ref is near a * sum(q) * scale for rows past J: compare relative to |L|.
+    e = np.abs(f32(l) - l_ref) / np.maximum(1.0, np.abs(l_ref))
+    assert e.max() <= 5e-3
+    assert np.abs(f32(o) - o_ref).max() <= 2e-2
+    assert ea.device_status() == 0
+
+
 def test_fp32_tiny_workload():
     cfg = syn.TINY
     q, k, v = syn.prefill_inputs(cfg)
