@@ -10,9 +10,7 @@ in a temporary directory), then one link makes the library.
 sources with every wait limited to TEST_WAIT_CYCLES instead of about 1.5 s,
 with the producers of the prefill and decode kernels stopping before ring index
 TEST_WITHHOLD (so that the kernels' waits run out on purpose and their abort
-paths run), and with the probes of csrc/testbuild_probes.cu (device functions
-evaluated on their own).  The product library is never built with these
-switches.
+paths run).  The product library is never built with these switches.
 """
 from __future__ import annotations
 
@@ -37,11 +35,11 @@ NVCC_FLAGS = [
     "--expt-relaxed-constexpr",
 ]
 # The test build: ~1 ms waits, producers stop before ring index 2 (the
-# prefill's second K tile; the decode's third page of a chunk), probes compiled.
+# prefill's second K tile; the decode's third page of a chunk).
 TEST_WAIT_CYCLES = 2000000
 TEST_WITHHOLD = 2
 TEST_FLAGS = ["-DEXATTN_WAIT_LIMIT_CYCLES=%dLL" % TEST_WAIT_CYCLES,
-              "-DEXATTN_TEST_WITHHOLD=%d" % TEST_WITHHOLD, "-DEXATTN_TEST_BUILD=1"]
+              "-DEXATTN_TEST_WITHHOLD=%d" % TEST_WITHHOLD]
 
 
 def _sources():

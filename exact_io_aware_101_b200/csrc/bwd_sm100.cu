@@ -179,8 +179,7 @@ __global__ void __launch_bounds__(256)
 
 // P = 2^(s*c + bias - l2) for 32 columns (0 where vis(i) is false), packed to
 // bf16 pairs; bias = bias0 + bias_step * i (ALiBi); l2 per column (per_col) or
-// one value.  On unmasked columns one pair in four takes 2^x from the FMA-pipe
-// cubic (relative error < 2^-13, below the bf16 rounding that follows).
+// one value.
 template <bool kAlibi, bool kMasked, typename Vis>
 __device__ __forceinline__ void p_cols(const uint32_t *sv, const float *l2c, float l2s,
                                        bool per_col, float c, float bias0, float bias_step,
@@ -195,15 +194,10 @@ __device__ __forceinline__ void p_cols(const uint32_t *sv, const float *l2c, flo
       x = fma2(make_float2(bias_step, bias_step),
                make_float2(static_cast<float>(i), static_cast<float>(i + 1)),
                make_float2(x.x + bias0, x.y + bias0));
-    float2 e;
-    if (!kMasked && (i & 6) == 6) {
-      e = exp2_poly2(x);
-    } else {
-      e = make_float2(ex2(x.x), ex2(x.y));
-      if (kMasked) {
-        if (!vis(i)) e.x = 0.f;
-        if (!vis(i + 1)) e.y = 0.f;
-      }
+    float2 e = make_float2(ex2(x.x), ex2(x.y));
+    if (kMasked) {
+      if (!vis(i)) e.x = 0.f;
+      if (!vis(i + 1)) e.y = 0.f;
     }
     pk[i >> 1] = pack_bf16x2(e.x, e.y);
   }

@@ -316,42 +316,11 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return *reinterpret_cast<float2 *>(&d);
 }
 
-__device__ __forceinline__ float2 add2_rm(float2 a, float2 b) {  // rounded toward -inf
-  uint64_t d;
-  asm("add.rm.f32x2 %0, %1, %2;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
-  return *reinterpret_cast<float2 *>(&d);
-}
-
 // ------------------------------------------------------------------ numerics
 __device__ __forceinline__ float ex2(float x) {  // 2^x on the special-function unit
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x for a pair, on the FMA/ALU pipes instead of the special-function unit.
-// x = j + f with j = floor(x): adding 1.5*2^23 rounded toward -inf leaves j in
-// the low mantissa bits of the sum, so (bits << 23) is j shifted into the
-// exponent field; 2^f on [0,1) is a cubic (coefficients fitted by
-// exp2_poly.py, relative error < 2^-13); the result is the cubic's value with
-// j added to its exponent.  Inputs are clamped at -126 so that the exponent
-// field never wraps below zero (p(0) is just under 1); below the clamp the true
-// value is under 2^-126 and the result stays a tiny non-negative number.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kC0 = 0x1.fff63p-1f, kC1 = 0x1.64445ap-1f, kC2 = 0x1.cefc4p-3f,
-                  kC3 = 0x1.3f962p-4f;
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
-  const float2 t = add2_rm(x, make_float2(kShift, kShift));
-  const float2 j = add2(t, make_float2(-kShift, -kShift));
-  const float2 f = add2(x, make_float2(-j.x, -j.y));
-  float2 p = fma2(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
-  p = fma2(p, f, make_float2(kC1, kC1));
-  p = fma2(p, f, make_float2(kC0, kC0));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Programmatic dependent launch.  A kernel launched with the programmatic

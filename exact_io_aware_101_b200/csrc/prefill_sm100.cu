@@ -26,8 +26,9 @@
 //  * exp2-based online softmax with scale*log2(e) folded into one FMA and a
 //    lazy rescale: the reference max m only moves (and O is rescaled in TMEM)
 //    when a row's max grows by more than 8 in log2 units; O/l stays exact.
-//    A quarter of the exponentials run as a cubic on the FMA pipe so that the
-//    special-function unit is not the bottleneck.
+//    Once m is set, an unmasked tile first takes P against m as it stands and
+//    keeps it when the row sums stay at most 255, so most tiles never search
+//    for their own max.
 //  * Causal: KV tiles above the diagonal are never loaded or multiplied; only
 //    diagonal tiles are masked (Concepts: causal masking; Lab 01 step 4).
 //  * Grid: one CTA per (Q-tile pair, batch*head).  Consecutive CTAs share K/V

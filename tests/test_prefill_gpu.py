@@ -137,7 +137,7 @@ def test_bf16_deterministic_and_gqa_equals_repeated_heads():
 @pytest.mark.parametrize("d", [64, 128])
 def test_bf16_large_scores_stay_finite(causal, d):
     # Scores of several hundred: only the running-max shift keeps exp finite, and
-    # exponents far below -126 reach the polynomial exp2 of unmasked tiles.
+    # exponents far below -126 reach the exp2 of unmasked tiles.
     B, H, N = 1, 2, 300
     q, k, v = syn.random_qkv(B, H, H, N, d, seed=11)
     q = (q.float() * 8).to(torch.bfloat16)
@@ -156,10 +156,9 @@ def test_bf16_large_scores_stay_finite(causal, d):
 # before it looks for the tile's own max, and keeps that P only when every
 # row's sum stays at most 255.  One key here scores far above every earlier
 # key for every query (all queries positive, that key constant): its x = s*c - m
-# lands just above 8, near 50, or near 200, in a column that goes to the
-# special-function exp2 (column 0 of a group of 8) or to the polynomial one
-# (column 6), whose exponent field would wrap above 128.  Each must fall back to
-# the max-first step and match the oracle.
+# lands within 8 (the P stands), across 8 for some rows only, near 50, or near
+# 200 (where 2^x overflows fp32), at several columns of the tile.  A row that
+# misses must fall back to the max-first step; every case must match the oracle.
 @pytest.mark.parametrize("col,a,causal", [(46, 16.0, False), (46, 16.0, True), (46, 4.0, False),
                                           (46, 0.75, False), (40, 16.0, False), (47, 1.0, True)])
 def test_bf16_score_jump_after_the_first_tile(col, a, causal):
