@@ -579,17 +579,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int j = jlo; ok && j < jhi; ++j) {
           const int rj = j - jlo;
-          bool v_ready = false;
+          // The ring entries this iteration reads, V(j) and K(j+1), are checked
+          // before the waits for P: their barrier latency then falls in time
+          // the issuing thread spends waiting anyway, not between a P and the
+          // MMAs that consume it.
+          if (!(ok = wait_full(2 * rj + 1))) break;
+          if (j + 1 < jhi && !(ok = wait_full(2 * rj + 2))) break;
           if (has(0, j)) {
-            if (!(ok = mbar_wait(&bars->p_full[0], (j - js0) & 1, abort_flag, p.status) &&
-                       wait_full(2 * rj + 1)))
-              break;
-            v_ready = true;
+            if (!(ok = mbar_wait(&bars->p_full[0], (j - js0) & 1, abort_flag, p.status))) break;
             tc_fence_after();
             issue_pv(0, 2 * rj + 1, j > js0);
             tc_commit(&bars->o_full[0]);
           }
-          if (j + 1 < jhi && !(ok = wait_full(2 * rj + 2))) break;
           if (has(0, j + 1)) {
             // P0(j) aliases S0.  tcgen05.mma ops issued by one thread execute in
             // order, so S0(j+1) overwrites the P0(j) columns only after PV0(j),
@@ -599,7 +600,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (has(1, j)) {
             if (!(ok = mbar_wait(&bars->p_full[1], (j - js1) & 1, abort_flag, p.status))) break;
-            if (!v_ready && !(ok = wait_full(2 * rj + 1))) break;
             tc_fence_after();
             issue_pv(1, 2 * rj + 1, j > js1);
             tc_commit(&bars->o_full[1]);
@@ -639,17 +639,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float l = 0.f;
     bool ok = true;
     for (int j = jst; j < jen; ++j) {
-      ok = mbar_wait(&bars->s_full[t], (j - jst) & 1, abort_flag, p.status);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
       // Visible columns [lo, hi) of this row in KV tile j: the end of the keys,
-      // the causal diagonal and the sliding window.
+      // the causal diagonal and the sliding window.  (Worked out, with the
+      // path the tile takes, before the scores arrive.)
       int hi = min(BN, nk - j * BN);
       if (p.causal) hi = min(hi, ctx + row - j * BN + 1);
       // (Rows past the last take the last real row's window so that they never
       // force the masked path on a warp whose real rows need none.)
       const int lo = p.window > 0 ? ctx + min(row, nq - 1) - p.window + 1 - j * BN : 0;
+      // Only diagonal, window-edge and last tiles carry masked columns;
+      // elsewhere the warp takes the branch-free path.
+      const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= BN);
+      const bool attempt = !kAlibi && !masked && j > jst && __all_sync(0xffffffffu, m != -INFINITY);
+      ok = mbar_wait(&bars->s_full[t], (j - jst) & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
       // The whole 128-column score row of this thread, in one TMEM load.
       uint32_t sv[128];
       tmem_ld128(s_addr, sv);
@@ -667,9 +672,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         cx = 1.0f;
       }
-      // Only diagonal, window-edge and last tiles carry masked columns;
-      // elsewhere the warp takes the branch-free path.
-      const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= BN);
       if (masked) {
 #pragma unroll
         for (int i = 0; i < 128; ++i)
@@ -688,7 +690,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // at once: their scores in registers are no longer those in TMEM (and
       // ALiBi's rise along the row, so the attempt would miss most tiles).
       bool fast = false, missed = false;
-      if (!kAlibi && !masked && j > jst && __all_sync(0xffffffffu, m != -INFINITY)) {
+      if (attempt) {
         uint32_t pk[64];
         const float l_tile = exp_row_held(sv, cx, m, pk);
         missed = !(l_tile <= 255.0f);
