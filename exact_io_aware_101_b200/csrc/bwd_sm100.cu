@@ -402,7 +402,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int it = 0; ok && it < n_items; ++it) {
         const int bb = it & 1;
-        if (!(ok = mbar_wait(&bars->s_read[bb], (it >> 1) & 1, abort_flag, p.status) && wait_b(it)))
+        // dO(it) is checked first: its barrier latency then overlaps the wait
+        // for the elementwise warpgroup instead of following it.
+        if (!(ok = wait_b(it) && mbar_wait(&bars->s_read[bb], (it >> 1) & 1, abort_flag, p.status)))
           break;
         tc_fence_after();
         issue_dp(it);

@@ -78,13 +78,23 @@ __device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t w) {
   return r;
 }
 
-// [u0, 0x64, u1, 0x64] is the f16x2 pair (1024 + u0, 1024 + u1); with
-// u = code + 128 (the code's sign bit flipped) subtracting 1152 leaves the
-// signed code, exactly.
-__device__ __forceinline__ uint32_t biased_f16x2_to_int(uint32_t x) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64806480u));
-  return r;
+// INT8 codes enter the MMAs as f16 values 1024 + u with u = code + 128 (the
+// code's sign bit flipped, the byte placed in the mantissa of 1024 by one byte
+// permute): that is code + kInt8Bias, exactly.  A sum over d of (code + bias)
+// * q is the wanted sum plus bias * (sum of q), and a sum over tokens of
+// P * (code + bias) the wanted one plus bias * (sum of P); both extra terms are
+// formed exactly as the MMAs see their operands and subtracted in f32.
+constexpr float kInt8Bias = 1152.f;
+
+__device__ __forceinline__ float f16_lo(uint32_t w) {
+  float f;
+  asm("{ .reg .f16 h, l; mov.b32 {l, h}, %1; cvt.f32.f16 %0, l; }" : "=f"(f) : "r"(w));
+  return f;
+}
+__device__ __forceinline__ float f16_hi(uint32_t w) {
+  float f;
+  asm("{ .reg .f16 h, l; mov.b32 {l, h}, %1; cvt.f32.f16 %0, h; }" : "=f"(f) : "r"(w));
+  return f;
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -110,13 +120,14 @@ __device__ __forceinline__ uint32_t swz(uint32_t o) {
 }
 
 // The pair of codes (lo = element 0) at bits [16h, 16h+16) of a word -> f16x2.
+// INT8 codes come out biased, as code + 1152 (exact in f16): the MMAs take
+// them so, and the bias is taken back out of their sums (see kInt8Bias).
 template <int FMT>
 __device__ __forceinline__ uint32_t codes_f16x2(uint32_t w, int h) {
   if constexpr (FMT == ATTN_KV_E4M3) {
     return e4m3x2_f16x2(h ? (w >> 16) : w);
   } else {
-    const uint32_t x = w ^ 0x80808080u;
-    return biased_f16x2_to_int(prmt(x, 0x64646464u, h ? 0x4342u : 0x4140u));
+    return prmt(w ^ 0x80808080u, 0x64646464u, h ? 0x4342u : 0x4140u);
   }
 }
 
@@ -133,10 +144,10 @@ __device__ __forceinline__ void vpairs(uint32_t A, uint32_t B, uint32_t (&p)[4])
   } else {
     const uint32_t a = A ^ 0x80808080u, b = B ^ 0x80808080u;
     const uint32_t lo = prmt(a, b, 0x5140u), hi = prmt(a, b, 0x7362u);
-    p[0] = biased_f16x2_to_int(prmt(lo, 0x64646464u, 0x4140u));
-    p[1] = biased_f16x2_to_int(prmt(lo, 0x64646464u, 0x4342u));
-    p[2] = biased_f16x2_to_int(prmt(hi, 0x64646464u, 0x4140u));
-    p[3] = biased_f16x2_to_int(prmt(hi, 0x64646464u, 0x4342u));
+    p[0] = prmt(lo, 0x64646464u, 0x4140u);  // biased, as in codes_f16x2
+    p[1] = prmt(lo, 0x64646464u, 0x4342u);
+    p[2] = prmt(hi, 0x64646464u, 0x4140u);
+    p[3] = prmt(hi, 0x64646464u, 0x4342u);
   }
 }
 
@@ -285,6 +296,7 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     // scale*log2(e)*2^-e back in f32.
     uint32_t qb[KS][2];
     float sq_own;
+    float qsum_own = 0.f;
     {
       float qv[D / 4];
       const bool live = g < GB;
@@ -320,10 +332,26 @@ __global__ void __launch_bounds__((HC + 1) * 32)
         qb[t][1] = pack_f16x2(qv[4 * t + 2] * up, qv[4 * t + 3] * up);
       }
       sq_own = scale_log2 * down;
+      if constexpr (FMT != ATTN_KV_E4M3) {
+        // This head's sum of q over d, from the f16 operands themselves.
+        float qs = 0.f;
+#pragma unroll
+        for (int t = 0; t < KS; ++t)
+          qs += (f16_lo(qb[t][0]) + f16_hi(qb[t][0])) + (f16_lo(qb[t][1]) + f16_hi(qb[t][1]));
+        qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+        qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+        qsum_own = qs * kInt8Bias;
+      }
     }
     // Score multipliers of this thread's two accumulator columns (heads 2c, 2c+1).
     const float sq0 = __shfl_sync(0xffffffffu, sq_own, 8 * c);
     const float sq1 = __shfl_sync(0xffffffffu, sq_own, 8 * c + 4);
+    // (INT8) the bias's share of those columns' scores, before the multipliers.
+    float qb0 = 0.f, qb1 = 0.f;
+    if constexpr (FMT != ATTN_KV_E4M3) {
+      qb0 = __shfl_sync(0xffffffffu, qsum_own, 8 * c);
+      qb1 = __shfl_sync(0xffffffffu, qsum_own, 8 * c + 4);
+    }
 
     // Page scales: lane i holds those of page i of the chunk.
     float ks_r = 0.f, vs_r = 0.f;
@@ -352,6 +380,11 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     for (int i = 0; i < KS; ++i)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+    // (INT8) sum over tokens of the p.v operand, in the accumulator's columns:
+    // the product of an all-ones tile with P^T, so it holds exactly the f16
+    // values the p.v MMAs take.
+    float psum[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr uint32_t kOnes = 0x3c003c00u;  // f16x2 (1, 1)
     // Source lanes of the P^T fragment: tokens 2c and 2c+1 of head g.
     const int src0 = 8 * c + (g >> 1), src1 = src0 + 4;
     const uint32_t psel = (g & 1) ? 0x7632u : 0x5410u;
@@ -379,6 +412,10 @@ __global__ void __launch_bounds__((HC + 1) * 32)
                 codes_f16x2<FMT>(wa, 1), codes_f16x2<FMT>(wb, 1), qb[t][0], qb[t][1]);
       }
       const float kq0 = ks * sq0, kq1 = ks * sq1;
+      if constexpr (FMT != ATTN_KV_E4M3) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[e] -= (e & 1) ? qb1 : qb0;
+      }
       sv[0] = g < ntok ? (sc[0] + sd[0]) * kq0 : -INFINITY;
       sv[1] = g < ntok ? (sc[1] + sd[1]) * kq1 : -INFINITY;
       sv[2] = g + 8 < ntok ? (sc[2] + sd[2]) * kq0 : -INFINITY;
@@ -447,6 +484,12 @@ __global__ void __launch_bounds__((HC + 1) * 32)
           acc[i2][2] *= a0;
           acc[i2][3] *= a1;
         }
+        if constexpr (FMT != ATTN_KV_E4M3) {
+          psum[0] *= a0;
+          psum[1] *= a1;
+          psum[2] *= a0;
+          psum[3] *= a1;
+        }
         mv0 = n0;
         mv1 = n1;
       }
@@ -455,6 +498,10 @@ __global__ void __launch_bounds__((HC + 1) * 32)
       uint32_t pa0, pa1, pb0, pb1;
       p_frag(pa, vsa * e0, vsa * e1, pa0, pa1);
       p_frag(pb, vsb * e0, vsb * e1, pb0, pb1);
+      if constexpr (FMT != ATTN_KV_E4M3) {
+        mma_f16(psum, kOnes, kOnes, kOnes, kOnes, pa0, pa1);
+        mma_f16(psum, kOnes, kOnes, kOnes, kOnes, pb0, pb1);
+      }
       const uint8_t *vta = sga + (HC + warp) * C::SLICE, *vtb = sgb + (HC + warp) * C::SLICE;
       const VRow<D> va = load_vrow<D>(vta, 2 * c, g, 2 * c < na);
       const VRow<D> vb = load_vrow<D>(vta, 2 * c + 1, g, 2 * c + 1 < na);
@@ -503,6 +550,12 @@ __global__ void __launch_bounds__((HC + 1) * 32)
     unsigned bits = *reinterpret_cast<volatile unsigned *>(&sm_status) |
                     (*reinterpret_cast<volatile int *>(&sm_bad) ? ATTN_DEV_BAD_PAGE : 0u);
     if (bad && bits == 0) bits = ATTN_DEV_TIMEOUT;  // aborted by a wait that timed out
+    if constexpr (FMT != ATTN_KV_E4M3) {
+#pragma unroll
+      for (int i = 0; i < KS; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(-kInt8Bias, psum[e], acc[i][e]);
+    }
     // O = acc * 2^(mv - m) / l.
     const float inv0 = (mv0 == -INFINITY ? 0.f : ex2(mv0 - m0)) / l0;
     const float inv1 = (mv1 == -INFINITY ? 0.f : ex2(mv1 - m1)) / l1;
