@@ -185,6 +185,27 @@ def test_bf16_score_jump_after_the_first_tile(col, a, causal):
     assert ea.device_status() == 0
 
 
+def test_bf16_score_jump_inside_a_window():
+    # As above, under a 300-key causal window: the jump sits in the window of
+    # the later rows only, and rows whose window starts in a masked first tile
+    # keep a reference max that a later tile may exceed.
+    B, H, N, d = 1, 2, 1000, 128
+    g = torch.Generator().manual_seed(4321)
+    q = torch.randn(B, H, N, d, generator=g).abs().to(torch.bfloat16)
+    k = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    k[:, :, 520, :] = 4.0
+    scale = 1.0 / math.sqrt(d)
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=scale, causal=True, window=300)
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=scale, window=300)
+    torch.cuda.synchronize()
+    e = np.abs(f32(l) - l_ref) / np.maximum(1.0, np.abs(l_ref))
+    assert e.max() <= 5e-3
+    assert np.abs(f32(o) - o_ref).max() <= 2e-2
+    assert ea.device_status() == 0
+
+
 def test_fp32_tiny_workload():
     cfg = syn.TINY
     q, k, v = syn.prefill_inputs(cfg)

@@ -70,6 +70,26 @@ def test_prefill_paged_small(qlens, ctxs, Hq, Hkv, d):
     assert ea.device_status() == 0
 
 
+# One cached key scores far above every earlier key for every query of its
+# sequence (queries made positive, that key constant), in a KV tile after the
+# first: a tile whose P against the running max sums past 255 must fall back
+# to the max-first step in the paged kernel too.
+@pytest.mark.parametrize("a,key", [(16.0, 300), (1.0, 700), (4.0, 1100)])
+def test_prefill_paged_score_jump(a, key):
+    qlens, ctxs = [200, 96], [1000, 1200]
+    cfg, inp = make(qlens, ctxs, 4, 2, 128, seed=41)
+    inp["q"] = inp["q"].float().abs().to(torch.bfloat16)
+    for s_ in range(len(qlens)):
+        pg = int(inp["block_table"][s_, key // 16])
+        inp["k_pages"][pg, :, key % 16, :] = a
+    o_ref, l_ref = oracle_run(inp, cfg.scale)
+    o, l = gpu_run(inp, cfg.scale)
+    e = np.abs(f32(l) - l_ref) / np.maximum(1.0, np.abs(l_ref))
+    assert e.max() <= 5e-3
+    assert np.abs(f32(o) - o_ref).max() <= 2e-2
+    assert ea.device_status() == 0
+
+
 @pytest.mark.parametrize("qlens,ctxs", [
     # Equal key counts (the work order breaks ties by sequence index).
     ([9, 9, 30, 9, 30], [40, 40, 19, 40, 19]),
