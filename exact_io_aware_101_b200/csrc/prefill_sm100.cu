@@ -81,6 +81,7 @@ struct Bars {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t q_full;
+  uint64_t q_full1;  // whole-pair self-attention: Q tile 1, loaded behind K(jlo)
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
@@ -321,6 +322,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&bars->empty[i], 1);
     }
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_full1, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], BM);
@@ -415,9 +417,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tm_v);
       const int zq = b * p.Hq + hq;
       const int zkv = b * p.Hkv + hkv;
-      // Both Q slots; a split CTA's two warpgroups share its one Q tile.
-      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
-      for (int t = 0; t < 2; ++t)
+      // A whole pair loads Q tile 0 here and Q tile 1 behind K(jlo), on a
+      // barrier of its own, so the first score MMA waits for two tiles, not
+      // three.  A split CTA's two warpgroups share its one Q tile (both slots).
+      constexpr bool kQ2 = !kSplit;
+      mbar_arrive_expect_tx(&bars->q_full, (kQ2 ? 1 : 2) * C::TILE_BYTES);
+      for (int t = 0; t < (kQ2 ? 1 : 2); ++t)
         for (int c = 0; c < C::CH; ++c)
           tma_load_3d(sQ + t * C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full, 64 * c,
                       row0 + (kSplit && split ? 0 : t * BM), zq);
@@ -451,7 +456,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
       int issued = 0;
-      for (int i = 0; i < 2 * (jhi - jlo); ++i) {
+      if constexpr (kQ2) {
+        // Ring entry 0, K(jlo), then Q tile 1: S0's operands arrive first.
+        mbar_arrive_expect_tx(&bars->full[0], C::TILE_BYTES);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sRing + c * CHUNK_BYTES, &tm_k, &bars->full[0], 64 * c, jlo * BN, zkv);
+        mbar_arrive_expect_tx(&bars->q_full1, C::TILE_BYTES);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(sQ + C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full1, 64 * c,
+                      row0 + BM, zq);
+        issued = 1;
+      }
+      for (int i = issued; i < 2 * (jhi - jlo); ++i) {
         const int slot = i % C::NST;
         const int round = i / C::NST;
         if (round > 0 && !mbar_wait(&bars->empty[slot], (round - 1) & 1, abort_flag, p.status))
@@ -474,6 +490,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Drain: no copy may still be writing shared memory when the CTA exits.
       // Normally these phases completed long ago and each wait returns at once.
       mbar_wait_drain(&bars->q_full, 0, p.status);
+      if (kQ2) mbar_wait_drain(&bars->q_full1, 0, p.status);
       for (int i = max(0, issued - C::NST); i < issued; ++i)
         mbar_wait_drain(&bars->full[i % C::NST], (i / C::NST) & 1, p.status);
     }
@@ -572,13 +589,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         if (ok) {
           tc_fence_after();
-  #pragma unroll
-          for (int t = 0; t < 2; ++t)
-            if (has(t, jlo)) {
-              issue_s(t, 0);
-              tc_commit(&bars->s_full[t]);
-            }
-          tc_commit(&bars->empty[slot_of(0)]);
+          if (has(0, jlo)) {
+            issue_s(0, 0);
+            tc_commit(&bars->s_full[0]);
+          }
+          if constexpr (!kPaged && !kSplit) {
+            // Q tile 1 arrives behind K(jlo) on its own barrier.
+            ok = mbar_wait(&bars->q_full1, 0, abort_flag, p.status);
+            tc_fence_after();
+          }
+          if (ok && has(1, jlo)) {
+            issue_s(1, 0);
+            tc_commit(&bars->s_full[1]);
+          }
+          if (ok) tc_commit(&bars->empty[slot_of(0)]);
         }
         for (int j = jlo; ok && j < jhi; ++j) {
           const int rj = j - jlo;
