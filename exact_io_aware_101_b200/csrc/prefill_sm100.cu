@@ -10,8 +10,10 @@
 //
 // How it maps to sm_100a:
 //  * one CTA = 2 Q tiles (256 rows) of one (batch, head); 12 warps:
-//      warp 0      TMA producer: Q once, then K0 V0 K1 V1 ... into a ring of
-//                  NST shared-memory slots (128B-swizzled, no multicast);
+//      warp 0      TMA producer: Q once, then the K/V tiles, K then V of each,
+//                  into a ring of NST shared-memory slots (128B-swizzled, no
+//                  multicast); an ALiBi whole pair walks them from the last
+//                  down, every other CTA from the first up;
 //      warp 1      allocates the 512 TMEM columns and issues every tcgen05.mma
 //                  from one thread;
 //      warps 4-7   softmax/correction/epilogue for Q tile 0 (TMEM lanes 0-127);
@@ -28,7 +30,8 @@
 //    when a row's max grows by more than 8 in log2 units; O/l stays exact.
 //    Once m is set, an unmasked tile first takes P against m as it stands and
 //    keeps it when the row sums stay at most 255, so most tiles never search
-//    for their own max.
+//    for their own max.  ALiBi tiles do so in the downward walk, along which
+//    the bias falls.
 //  * Causal: KV tiles above the diagonal are never loaded or multiplied; only
 //    diagonal tiles are masked (Concepts: causal masking; Lab 01 step 4).
 //  * Grid: one CTA per (Q-tile pair, batch*head).  Consecutive CTAs share K/V
@@ -144,14 +147,50 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float c, flo
   return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
 }
 
+// ALiBi: each score s of the row becomes s*c + slope2*col + rb, the scaled
+// score plus the bias slope * (key - query) in log2 units (rb: column 0's).
+__device__ __forceinline__ void add_alibi(uint32_t (&sv)[128], float c, float slope2, float rb) {
+  const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2), rb2 = make_float2(rb, rb);
+#pragma unroll
+  for (int i = 0; i < 128; i += 2) {
+    const float2 bias = fma2(sl2, make_float2(static_cast<float>(i), static_cast<float>(i + 1)), rb2);
+    const float2 x = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, bias);
+    sv[i] = __float_as_uint(x.x);
+    sv[i + 1] = __float_as_uint(x.y);
+  }
+}
+
 // The same P and row sum kept in registers: TMEM, and with it the S row, is
-// left untouched.
+// left untouched.  (Its ALiBi form below.)
 __device__ __forceinline__ float exp_row_held(const uint32_t (&sv)[128], float c, float m,
                                               uint32_t (&pk)[64]) {
   const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
   float2 sum_a = make_float2(0.f, 0.f), sum_b = make_float2(0.f, 0.f);
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) exp_chunk(sv, cc, c2, nm2, pk + cc * 16, sum_a, sum_b);
+  return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
+}
+
+// exp_row_held for an ALiBi tile: x = s*c + (slope2*col + rb - m), the bias
+// taken into each exponent, so that sv keeps the raw scores.
+__device__ __forceinline__ float exp_row_held_alibi(const uint32_t (&sv)[128], float c, float m,
+                                                    float slope2, float rb, uint32_t (&pk)[64]) {
+  const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2);
+  const float2 b2 = make_float2(rb - m, rb - m);
+  float2 sum_a = make_float2(0.f, 0.f), sum_b = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 128; i += 4) {
+    const float2 o0 = fma2(sl2, make_float2(static_cast<float>(i), static_cast<float>(i + 1)), b2);
+    const float2 o1 = fma2(sl2, make_float2(static_cast<float>(i + 2), static_cast<float>(i + 3)), b2);
+    const float2 x0 = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, o0);
+    const float2 x1 = fma2(make_float2(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])), c2, o1);
+    const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+    const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+    sum_a = add2(sum_a, p0);
+    sum_b = add2(sum_b, p1);
+    pk[i >> 1] = pack_bf16x2(p0.x, p0.y);
+    pk[(i >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+  }
   return (sum_a.x + sum_a.y) + (sum_b.x + sum_b.y);
 }
 
@@ -163,6 +202,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_k1,
                         const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   using C = Cfg<D>;
+  // An ALiBi whole-pair self-attention CTA walks its KV tiles from the last
+  // to the first: the bias then falls along the walk, so that later tiles can
+  // keep P against the running max.  (The other CTAs walk up from the first:
+  // walking down made the causal and GQA launches about 3 % slower.)
+  constexpr bool kRev = kAlibi && !kPaged && !kSplit;
   // The split CTAs of a launch come as a second grid, programmatically
   // dependent on this one: it may be scheduled on the SMs this grid frees.
   if constexpr (!kPaged && !kSplit) grid_dependents_launch();
@@ -434,7 +478,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto entry = [&](int i, bool &v, int &kv) {
         if (!split) {
           v = (i & 1) != 0;
-          kv = jlo + (i >> 1);
+          kv = kRev ? jhi - 1 - (i >> 1) : jlo + (i >> 1);
           return;
         }
         if (i < 2) {
@@ -460,7 +504,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Ring entry 0, K(jlo), then Q tile 1: S0's operands arrive first.
         mbar_arrive_expect_tx(&bars->full[0], C::TILE_BYTES);
         for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(sRing + c * CHUNK_BYTES, &tm_k, &bars->full[0], 64 * c, jlo * BN, zkv);
+          tma_load_3d(sRing + c * CHUNK_BYTES, &tm_k, &bars->full[0], 64 * c,
+                      (kRev ? jhi - 1 : jlo) * BN, zkv);
         mbar_arrive_expect_tx(&bars->q_full1, C::TILE_BYTES);
         for (int c = 0; c < C::CH; ++c)
           tma_load_3d(sQ + C::TILE_BYTES + c * CHUNK_BYTES, &tm_q, &bars->q_full1, 64 * c,
@@ -587,56 +632,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {
+        // KV tile of walk step rj (upward from jlo, or downward from jhi - 1),
+        // and a tile's step count within its own range.
+        auto walk_j = [&](int rj) { return kRev ? jhi - 1 - rj : jlo + rj; };
+        auto step0 = [&](int j) { return kRev ? je0 - 1 - j : j - js0; };
+        auto step1 = [&](int j) { return kRev ? je1 - 1 - j : j - js1; };
+        const int nwalk = jhi - jlo;
         if (ok) {
           tc_fence_after();
-          if (has(0, jlo)) {
+          if (has(0, walk_j(0))) {
             issue_s(0, 0);
             tc_commit(&bars->s_full[0]);
           }
           if constexpr (!kPaged && !kSplit) {
-            // Q tile 1 arrives behind K(jlo) on its own barrier.
+            // Q tile 1 arrives behind the first K tile on its own barrier.
             ok = mbar_wait(&bars->q_full1, 0, abort_flag, p.status);
             tc_fence_after();
           }
-          if (ok && has(1, jlo)) {
+          if (ok && has(1, walk_j(0))) {
             issue_s(1, 0);
             tc_commit(&bars->s_full[1]);
           }
           if (ok) tc_commit(&bars->empty[slot_of(0)]);
         }
-        for (int j = jlo; ok && j < jhi; ++j) {
-          const int rj = j - jlo;
-          // The ring entries this iteration reads, V(j) and K(j+1), are checked
+        for (int rj = 0; ok && rj < nwalk; ++rj) {
+          const int j = walk_j(rj);
+          const bool more = rj + 1 < nwalk;
+          const int jn = more ? walk_j(rj + 1) : -1;  // the next tile of the walk
+          // The ring entries this iteration reads, V(j) and K(jn), are checked
           // before the waits for P: their barrier latency then falls in time
           // the issuing thread spends waiting anyway, not between a P and the
           // MMAs that consume it.
           if (!(ok = wait_full(2 * rj + 1))) break;
-          if (j + 1 < jhi && !(ok = wait_full(2 * rj + 2))) break;
+          if (more && !(ok = wait_full(2 * rj + 2))) break;
           if (has(0, j)) {
-            if (!(ok = mbar_wait(&bars->p_full[0], (j - js0) & 1, abort_flag, p.status))) break;
+            const int st = step0(j);
+            if (!(ok = mbar_wait(&bars->p_full[0], st & 1, abort_flag, p.status))) break;
             tc_fence_after();
-            issue_pv(0, 2 * rj + 1, j > js0);
+            issue_pv(0, 2 * rj + 1, st > 0);
             tc_commit(&bars->o_full[0]);
           }
-          if (has(0, j + 1)) {
+          if (more && has(0, jn)) {
             // P0(j) aliases S0.  tcgen05.mma ops issued by one thread execute in
-            // order, so S0(j+1) overwrites the P0(j) columns only after PV0(j),
+            // order, so S0(jn) overwrites the P0(j) columns only after PV0(j),
             // issued just before, has consumed them: no completion wait needed.
             issue_s(0, 2 * rj + 2);
             tc_commit(&bars->s_full[0]);
           }
           if (has(1, j)) {
-            if (!(ok = mbar_wait(&bars->p_full[1], (j - js1) & 1, abort_flag, p.status))) break;
+            const int st = step1(j);
+            if (!(ok = mbar_wait(&bars->p_full[1], st & 1, abort_flag, p.status))) break;
             tc_fence_after();
-            issue_pv(1, 2 * rj + 1, j > js1);
+            issue_pv(1, 2 * rj + 1, st > 0);
             tc_commit(&bars->o_full[1]);
           }
           tc_commit(&bars->empty[slot_of(2 * rj + 1)]);  // V(j) no longer needed
-          if (has(1, j + 1)) {
+          if (more && has(1, jn)) {
             issue_s(1, 2 * rj + 2);  // in order after PV1(j), as for tile 0
             tc_commit(&bars->s_full[1]);
           }
-          if (j + 1 < jhi) tc_commit(&bars->empty[slot_of(2 * rj + 2)]);  // K(j+1) done
+          if (more) tc_commit(&bars->empty[slot_of(2 * rj + 2)]);  // K(jn) done
         }
       }
       // Every MMA issued above must finish before TMEM is released.
@@ -665,7 +720,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float m = -INFINITY;  // reference max, in log2 units of scaled scores
     float l = 0.f;
     bool ok = true;
-    for (int j = jst; j < jen; ++j) {
+    for (int jj = 0; jj < nt; ++jj) {
+      const int j = kRev ? jen - 1 - jj : jst + jj;  // the walk order of the MMAs
       // Visible columns [lo, hi) of this row in KV tile j: the end of the keys,
       // the causal diagonal and the sliding window.  (Worked out, with the
       // path the tile takes, before the scores arrive.)
@@ -677,8 +733,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Only diagonal, window-edge and last tiles carry masked columns;
       // elsewhere the warp takes the branch-free path.
       const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= BN);
-      const bool attempt = !kAlibi && !masked && j > jst && __all_sync(0xffffffffu, m != -INFINITY);
-      ok = mbar_wait(&bars->s_full[t], (j - jst) & 1, abort_flag, p.status);
+      const bool attempt = (!kAlibi || kRev) && !masked && jj > 0 &&
+                           __all_sync(0xffffffffu, m != -INFINITY);
+      ok = mbar_wait(&bars->s_full[t], jj & 1, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -686,19 +743,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t sv[128];
       tmem_ld128(s_addr, sv);
       tmem_ld_wait128(sv);
-      float cx = c;  // factor still to apply to sv in the exponent
-      if (kAlibi) {
-        const float rb = slope2 * static_cast<float>(j * BN - (ctx + row));
-        const float2 c2 = make_float2(c, c), sl2 = make_float2(slope2, slope2), rb2 = make_float2(rb, rb);
-#pragma unroll
-        for (int i = 0; i < 128; i += 2) {
-          const float2 bias = fma2(sl2, make_float2(static_cast<float>(i), static_cast<float>(i + 1)), rb2);
-          const float2 x = fma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, bias);
-          sv[i] = __float_as_uint(x.x);
-          sv[i + 1] = __float_as_uint(x.y);
-        }
-        cx = 1.0f;
-      }
+      // ALiBi: the bias of key column 0 (the slope per column is slope2).
+      const float rb = kAlibi ? slope2 * static_cast<float>(j * BN - (ctx + row)) : 0.f;
+      const float cx = kAlibi ? 1.0f : c;  // factor still to apply to sv in the exponent
       if (masked) {
 #pragma unroll
         for (int i = 0; i < 128; ++i)
@@ -713,13 +760,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // is read back from TMEM, which the attempt left untouched, and the tile
       // takes the max-first step, which then also moves a row that missed up
       // to its running max, so that a max left low by a window's first tile
-      // does not miss again.  Masked and ALiBi tiles take the max-first step
-      // at once: their scores in registers are no longer those in TMEM (and
-      // ALiBi's rise along the row, so the attempt would miss most tiles).
+      // does not miss again.  Masked tiles take the max-first step at once:
+      // their scores in registers are no longer those in TMEM.  An ALiBi
+      // tile's attempt adds the bias inside each exponent, leaving the scores
+      // raw, and the max-first step adds it to the row; in an upward walk,
+      // where the bias rises from tile to tile and the attempt would miss
+      // most, ALiBi tiles go max first at once.
       bool fast = false, missed = false;
       if (attempt) {
         uint32_t pk[64];
-        const float l_tile = exp_row_held(sv, cx, m, pk);
+        const float l_tile = kAlibi ? exp_row_held_alibi(sv, c, m, slope2, rb, pk)
+                                    : exp_row_held(sv, c, m, pk);
         missed = !(l_tile <= 255.0f);
         fast = !__any_sync(0xffffffffu, missed);
         if (fast) {
@@ -738,6 +789,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (!fast) {
+        if (kAlibi) add_alibi(sv, c, slope2, rb);  // (a masked -inf stays -inf)
         float mx;
         {
           float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
@@ -761,9 +813,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // P = 2^(s*c - m), rounded to bf16 and written over the (already read) S
         // columns; the row sum stays in fp32.
         l += exp_row(sv, cx, m_use, s_addr);
-        if (j > jst && __any_sync(0xffffffffu, resc)) {
+        if (jj > 0 && __any_sync(0xffffffffu, resc)) {
           // Lazy rescale of O (rare once the max settles).  O is stable here:
-          // S(j) completing implies PV(j-1) completed, and PV(j) waits for p_full.
+          // this tile's S completing implies the previous PV completed, and
+          // this tile's PV waits for p_full.
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t ov[32];

@@ -185,6 +185,36 @@ def test_bf16_score_jump_after_the_first_tile(col, a, causal):
     assert ea.device_status() == 0
 
 
+# ALiBi, on the whole-pair grid (74 heads x 2 pairs = one full wave): such a
+# CTA walks its KV tiles from the last down, so the bias falls along the walk
+# and an unmasked tile may keep P against the running max.  One key of the
+# first KV tile (the last one walked) scores far above the rest for every
+# query, so the P of that tile must be dropped and the tile redone max first,
+# with the bias added again to the scores it reads back.
+@pytest.mark.parametrize("col,a,causal", [(46, 16.0, True), (46, 4.0, False), (100, 0.75, True)])
+def test_bf16_alibi_score_jump_whole_pairs(col, a, causal):
+    B, H, N, d = 1, 74, 512, 128
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if grid_kind(B, H, N, sms) != "whole":
+        pytest.skip("this shape takes another grid on a %d-SM device" % sms)
+    g = torch.Generator().manual_seed(2468)
+    q = torch.randn(B, H, N, d, generator=g).abs().to(torch.bfloat16)
+    k = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    k[:, :, col, :] = a
+    scale = 1.0 / math.sqrt(d)
+    sl = slopes_for(H)
+    o_ref, l_ref = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                    scale=scale, causal=causal, alibi_slopes=sl.numpy())
+    o, l = ea.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale,
+                       alibi_slopes=sl.to(DEV))
+    torch.cuda.synchronize()
+    e = np.abs(f32(l) - l_ref) / np.maximum(1.0, np.abs(l_ref))
+    assert e.max() <= 5e-3
+    assert np.abs(f32(o) - o_ref).max() <= 2e-2
+    assert ea.device_status() == 0
+
+
 def test_bf16_score_jump_inside_a_window():
     # As above, under a 300-key causal window: the jump sits in the window of
     # the later rows only, and rows whose window starts in a masked first tile
