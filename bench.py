@@ -349,6 +349,18 @@ def timed_launches(items, flush, reps):
     return [[a.elapsed_time(b) for a, b in row] for row in times], launches
 
 
+def timed_component(items, flush, reps):
+    """A component's 3 warm-up launches, then its timed launches with the SM clock
+    sampled meanwhile (a component that follows a heavy one may run while power
+    capping holds the clock down).  Returns the durations and the clock summary,
+    reduced to the median clock and the reasons seen."""
+    timed_launches(items, flush, 3)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t, _ = timed_launches(items, flush, reps)
+    c = clk.summary()
+    return t, ({"sm_mhz": c["sm_mhz"], "reasons": c["reasons"]} if c else None)
+
+
 def component_time(ms_list):
     """Median (seconds) and mean (ms) of one component's flushed launch times: the
     median is the reported figure, robust to a slow launch while clocks or power
@@ -549,36 +561,36 @@ def run_ours(args):
 
     if not args.skip_components:
         comps = {"_timing": "per component: 3 warm-up launches, then args.component_reps "
-                            "launches each after an L2 flush; ms = median, ms_mean = mean"}
+                            "launches each after an L2 flush; ms = median, ms_mean = mean; "
+                            "clocks = median SM clock and throttle reasons during those launches"}
         for cfg in (syn.CAUSAL, syn.GQA, syn.WINDOW, syn.ALIBI):
             it = Prefill(cfg, lib)
-            timed_launches([it], flush, 3)
-            t, _ = timed_launches([it], flush, args.component_reps)
+            t, ck = timed_component([it], flush, args.component_reps)
             sec, mean_ms = component_time(t[0])
             tf = cfg.flops / sec / 1e12
-            comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3, "ms_mean": mean_ms}
+            comps[cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3, "ms_mean": mean_ms,
+                               "clocks": ck}
             del it
         it = ChunkedPrefill(syn.CHUNKED, lib)
-        timed_launches([it], flush, 3)
-        t, _ = timed_launches([it], flush, args.component_reps)
+        t, ck = timed_component([it], flush, args.component_reps)
         sec, mean_ms = component_time(t[0])
         tf = it.flops / sec / 1e12
         comps[syn.CHUNKED.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf, "ms": sec * 1e3, "ms_mean": mean_ms,
-                                   "flops": it.flops, "flops_counted": "4*d per visible pair"}
+                                   "flops": it.flops, "flops_counted": "4*d per visible pair",
+                                   "clocks": ck}
         del it
         for cfg in (syn.MHA_SWEEP[-1], syn.CAUSAL):
             it = Backward(cfg, lib)
-            timed_launches([it], flush, 3)
-            t, _ = timed_launches([it], flush, args.component_reps)
+            t, ck = timed_component([it], flush, args.component_reps)
             sec, mean_ms = component_time(t[0])
             tf = it.flops / sec / 1e12
             comps["bwd_" + cfg.name] = {"tflops": tf, "frac_of_peak": tf / peak_tf,
                                         "ms": sec * 1e3, "ms_mean": mean_ms, "flops": it.flops,
-                                        "flops_counted": "5 products of the algorithm (2.5x fwd)"}
+                                        "flops_counted": "5 products of the algorithm (2.5x fwd)",
+                                        "clocks": ck}
             del it
         dec = Decode(syn.DECODE, lib)
-        timed_launches([dec], flush, 3)
-        t, _ = timed_launches([dec], flush, args.component_reps)
+        t, ck = timed_component([dec], flush, args.component_reps)
         sec, mean_ms = component_time(t[0])
         torch.cuda.synchronize()
         if ea.decode_read_status(dec.ws) != 0:
@@ -589,12 +601,11 @@ def run_ours(args):
                                      "peak_gbs": peak_hbm,
                                      "traffic": profiled_traffic("decode_paged_gqa.md",
                                                                  "decode_paged.cu"),
-                                     "bound": "hbm"}
+                                     "bound": "hbm", "clocks": ck}
         del dec
         for fmt in ("e4m3", "int8"):
             dq = DecodeQ8(syn.DECODE, lib, fmt)
-            timed_launches([dq], flush, 3)
-            t, _ = timed_launches([dq], flush, args.component_reps)
+            t, ck = timed_component([dq], flush, args.component_reps)
             sec, mean_ms = component_time(t[0])
             torch.cuda.synchronize()
             if ea.decode_read_status(dq.ws) != 0:
@@ -603,7 +614,8 @@ def run_ours(args):
             comps["decode_paged_gqa_" + fmt] = {
                 "gbs": gbs, "frac_of_peak": gbs / peak_hbm, "ms": sec * 1e3, "ms_mean": mean_ms,
                 "algorithmic_bytes": dq.bytes, "peak_gbs": peak_hbm,
-                "traffic": profiled_traffic("decode_q8_gqa.md", "decode_q8.cu"), "bound": "hbm"}
+                "traffic": profiled_traffic("decode_q8_gqa.md", "decode_q8.cu"), "bound": "hbm",
+                "clocks": ck}
             del dq
         if ea.device_status() != 0:
             raise RuntimeError("device status word set in the component runs")
