@@ -139,6 +139,23 @@ def _check(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError("%s must be contiguous" % name)
 
 
+def _dims(t, name: str, ndim: int):
+    """Type and rank of one argument, checked before its dtype or device so that
+    shape errors are reported the same way on any device."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got shape %s" % (name, ndim, tuple(t.shape)))
+
+
+def _same_device(device, **tensors):
+    """Every tensor of one call must live on the device the call runs on: the
+    kernel is launched there, and another GPU's pointer is not valid in it."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError("%s is on %s but q is on %s" % (name, t.device, device))
+
+
 def _raise(rc: int, what: str):
     if rc != 0:
         raise AttnError(rc, what)
@@ -146,11 +163,25 @@ def _raise(rc: int, what: str):
 
 def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype, window=0, alibi_slopes=None):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, dtype, 4)
+        _dims(t, n, 4)
     B, Hq, N, d = q.shape
     if k.shape != v.shape or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
         raise ValueError("k/v must be [B, Hkv, N, d] matching q %s" % (tuple(q.shape),))
     Hkv = k.shape[1]
+    if out is not None:
+        _dims(out, "out", 4)
+    if lse is not None:
+        _dims(lse, "lse", 3)
+    if (out is not None and tuple(out.shape) != tuple(q.shape)) or \
+            (lse is not None and tuple(lse.shape) != (B, Hq, N)):
+        raise ValueError("out/lse shapes do not match q")
+    if alibi_slopes is not None:
+        _dims(alibi_slopes, "alibi_slopes", 1)
+        if alibi_slopes.numel() != Hq:
+            raise ValueError("alibi_slopes needs one value per query head")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, dtype, 4)
+    _same_device(q.device, k=k, v=v, out=out, lse=lse, alibi_slopes=alibi_slopes)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -165,8 +196,6 @@ def _prefill(fn, what, q, k, v, causal, scale, out, lse, dtype, window=0, alibi_
         slopes_ptr = None
         if alibi_slopes is not None:
             _check(alibi_slopes, "alibi_slopes", torch.float32, 1)
-            if alibi_slopes.numel() != Hq:
-                raise ValueError("alibi_slopes needs one value per query head")
             slopes_ptr = alibi_slopes.data_ptr()
         ext = getattr(library(), fn.__name__ + "_ext")
         with torch.cuda.device(q.device):
@@ -209,12 +238,10 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, cu_q, max_q: 
     block_table [S,max_blocks], seq_lens [S], cu_q [S+1] int32 (GPU).  max_q
     bounds every chunk length.  Returns (O bf16 [T,Hq,d], L fp32 [T,Hq]).
     """
-    _check(q, "q", torch.bfloat16, 3)
-    _check(k_pages, "k_pages", torch.bfloat16, 4)
-    _check(v_pages, "v_pages", torch.bfloat16, 4)
-    _check(block_table, "block_table", torch.int32, 2)
-    _check(seq_lens, "seq_lens", torch.int32, 1)
-    _check(cu_q, "cu_q", torch.int32, 1)
+    for name, t, nd in (("q", q, 3), ("k_pages", k_pages, 4), ("v_pages", v_pages, 4),
+                        ("block_table", block_table, 2), ("seq_lens", seq_lens, 1),
+                        ("cu_q", cu_q, 1)):
+        _dims(t, name, nd)
     T, Hq, d = q.shape
     num_pages, Hkv, page_size, d2 = k_pages.shape
     S = seq_lens.shape[0]
@@ -222,6 +249,23 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, cu_q, max_q: 
         raise ValueError("page pools must be [num_pages, Hkv, page_size, d]")
     if block_table.shape[0] != S or cu_q.shape[0] != S + 1:
         raise ValueError("block_table needs S rows and cu_q S+1 entries")
+    if out is not None:
+        _dims(out, "out", 3)
+    if lse is not None:
+        _dims(lse, "lse", 2)
+    if (out is not None and tuple(out.shape) != tuple(q.shape)) or \
+            (lse is not None and tuple(lse.shape) != (T, Hq)):
+        raise ValueError("out must be [T, Hq, d] and lse [T, Hq]")
+    if alibi_slopes is not None:
+        _dims(alibi_slopes, "alibi_slopes", 1)
+        if alibi_slopes.numel() != Hq:
+            raise ValueError("alibi_slopes needs one value per query head")
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _check(cu_q, "cu_q", torch.int32, 1)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out = torch.empty_like(q) if out is None else out
@@ -231,9 +275,9 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, cu_q, max_q: 
     slopes_ptr = None
     if alibi_slopes is not None:
         _check(alibi_slopes, "alibi_slopes", torch.float32, 1)
-        if alibi_slopes.numel() != Hq:
-            raise ValueError("alibi_slopes needs one value per query head")
         slopes_ptr = alibi_slopes.data_ptr()
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens, cu_q=cu_q, out=out, lse=lse, alibi_slopes=alibi_slopes)
     with torch.cuda.device(q.device):
         rc = library().attn_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                           block_table.data_ptr(), seq_lens.data_ptr(),
@@ -257,11 +301,9 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     attn_fwd returned them for the same inputs and options.  Returns bf16
     (dQ [B,Hq,N,d], dK [B,Hkv,N,d], dV [B,Hkv,N,d]).
     """
-    for name, t in (("q", q), ("o", o), ("dout", dout)):
-        _check(t, name, torch.bfloat16, 4)
-    _check(k, "k", torch.bfloat16, 4)
-    _check(v, "v", torch.bfloat16, 4)
-    _check(lse, "lse", torch.float32, 3)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _dims(t, name, 4)
+    _dims(lse, "lse", 3)
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
     if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
@@ -270,6 +312,16 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
         raise ValueError("k and v must be [B, Hkv, N, d]")
     if tuple(lse.shape) != (B, Hq, N):
         raise ValueError("lse must be [B, Hq, N]")
+    for name, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t is not None:
+            _dims(t, name, 4)
+            if tuple(t.shape) != tuple(like.shape):
+                raise ValueError("dq must have q's shape, dk and dv k's shape")
+    for name, t in (("q", q), ("o", o), ("dout", dout)):
+        _check(t, name, torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
@@ -288,6 +340,8 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, 1)
+    _same_device(q.device, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv,
+                 alibi_slopes=alibi_slopes, workspace=workspace)
     with torch.cuda.device(q.device):
         rc = library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                 lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
@@ -308,10 +362,7 @@ def _decode_dims(q, k_pages, v_pages, block_table, seq_lens):
     seq_lens with fewer than S rows would be read past its end on the device."""
     for name, t, nd in (("q", q, 3), ("k_pages", k_pages, 4), ("v_pages", v_pages, 4),
                         ("block_table", block_table, 2), ("seq_lens", seq_lens, 1)):
-        if not isinstance(t, torch.Tensor):
-            raise TypeError("%s must be a torch.Tensor" % name)
-        if t.dim() != nd:
-            raise ValueError("%s must have %d dims, got shape %s" % (name, nd, tuple(t.shape)))
+        _dims(t, name, nd)
     S, Hq, d = q.shape
     num_pages, Hkv, page_size, d2 = k_pages.shape
     if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
@@ -320,6 +371,17 @@ def _decode_dims(q, k_pages, v_pages, block_table, seq_lens):
     if block_table.shape[0] != S or seq_lens.shape[0] != S:
         raise ValueError("block_table/seq_lens must have S rows")
     return S, Hq, d, num_pages, Hkv, page_size, block_table.shape[1]
+
+
+def _decode_out_dims(q, S, Hq, out, lse):
+    """Caller-given outputs of a decode, checked for shape before any device check."""
+    if out is not None:
+        _dims(out, "out", 3)
+    if lse is not None:
+        _dims(lse, "lse", 2)
+    if (out is not None and tuple(out.shape) != tuple(q.shape)) or \
+            (lse is not None and tuple(lse.shape) != (S, Hq)):
+        raise ValueError("out must be [S, Hq, d] and lse [S, Hq]")
 
 
 def _decode_outputs(q, S, Hq, out, lse):
@@ -346,6 +408,7 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float |
     """
     S, Hq, d, num_pages, Hkv, page_size, max_blocks = _decode_dims(q, k_pages, v_pages,
                                                                    block_table, seq_lens)
+    _decode_out_dims(q, S, Hq, out, lse)
     _check(q, "q", torch.bfloat16, 3)
     _check(k_pages, "k_pages", torch.bfloat16, 4)
     _check(v_pages, "v_pages", torch.bfloat16, 4)
@@ -358,6 +421,8 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float |
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, 1)
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens, out=out, lse=lse, workspace=workspace)
     with torch.cuda.device(q.device):
         rc = library().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                          block_table.data_ptr(), seq_lens.data_ptr(),
@@ -383,6 +448,11 @@ def attn_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, block_table, s
         raise ValueError("kv_format must be one of %s" % sorted(KV_FORMATS))
     S, Hq, d, num_pages, Hkv, page_size, max_blocks = _decode_dims(q, k_pages, v_pages,
                                                                    block_table, seq_lens)
+    _decode_out_dims(q, S, Hq, out, lse)
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _dims(t, name, 2)
+        if tuple(t.shape) != (num_pages, Hkv):
+            raise ValueError("scales must be [num_pages, Hkv]")
     _check(q, "q", torch.bfloat16, 3)
     for name, t in (("k_pages", k_pages), ("v_pages", v_pages)):
         if t.dtype not in _KV_DTYPES[kv_format]:
@@ -393,8 +463,6 @@ def attn_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, block_table, s
     _check(v_scales, "v_scales", torch.float32, 2)
     _check(block_table, "block_table", torch.int32, 2)
     _check(seq_lens, "seq_lens", torch.int32, 1)
-    if tuple(k_scales.shape) != (num_pages, Hkv) or tuple(v_scales.shape) != (num_pages, Hkv):
-        raise ValueError("scales must be [num_pages, Hkv]")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out, lse = _decode_outputs(q, S, Hq, out, lse)
@@ -402,6 +470,9 @@ def attn_decode_paged_q8(q, k_pages, v_pages, k_scales, v_scales, block_table, s
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, 1)
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, k_scales=k_scales,
+                 v_scales=v_scales, block_table=block_table, seq_lens=seq_lens, out=out, lse=lse,
+                 workspace=workspace)
     with torch.cuda.device(q.device):
         rc = library().attn_decode_paged_q8(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
                                             k_scales.data_ptr(), v_scales.data_ptr(),
@@ -428,6 +499,7 @@ def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens,
     """
     S, Hq, d, num_pages, Hkv, page_size, max_blocks = _decode_dims(q, k_pages, v_pages,
                                                                    block_table, seq_lens)
+    _decode_out_dims(q, S, Hq, out, lse)
     _check(q, "q", torch.bfloat16, 3)
     _check(k_pages, "k_pages", torch.bfloat16, 4)
     _check(v_pages, "v_pages", torch.bfloat16, 4)
@@ -436,6 +508,8 @@ def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens,
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out, lse = _decode_outputs(q, S, Hq, out, lse)
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens, out=out, lse=lse)
     with torch.cuda.device(q.device):
         rc = library().attn_decode_paged_noalloc(
             q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),

@@ -286,3 +286,70 @@ def test_bwd_argument_checks(lib, kw, code):
 
 def test_bwd_rejects_small_workspace(lib):
     assert bwd(lib, ws_bytes=64) == INVALID
+
+
+def test_binding_checks_output_shapes_before_the_library():
+    # Caller-given outputs and gradients are written by the kernels at the sizes
+    # the inputs imply, so a smaller tensor must be refused before any call
+    # (these CPU tensors never reach the library).
+    import torch
+    bf = torch.bfloat16
+    B, Hq, Hkv, N, d = 1, 4, 2, 8, 64
+    q = torch.zeros(B, Hq, N, d, dtype=bf)
+    k = torch.zeros(B, Hkv, N, d, dtype=bf)
+    lse = torch.zeros(B, Hq, N)
+    with pytest.raises(ValueError, match="out/lse shapes"):
+        ea.attn_fwd(q, k, k, out=q[:, :2].contiguous())
+    with pytest.raises(ValueError, match="out/lse shapes"):
+        ea.attn_fwd(q, k, k, lse=lse[:, :, :4].contiguous())
+    with pytest.raises(ValueError, match="one value per query head"):
+        ea.attn_fwd(q, k, k, causal=True, alibi_slopes=torch.zeros(Hq - 1))
+    with pytest.raises(ValueError, match="out/lse shapes"):
+        ea.attn_fwd_f32(q.float(), k.float(), k.float(), out=q.float()[:, :, :4].contiguous())
+
+    with pytest.raises(ValueError, match="dq must have"):
+        ea.attn_bwd(q, k, k, q, lse, q, dq=q[:, :2].contiguous())
+    with pytest.raises(ValueError, match="dq must have"):
+        ea.attn_bwd(q, k, k, q, lse, q, dk=q)
+    with pytest.raises(ValueError, match="dq must have"):
+        ea.attn_bwd(q, k, k, q, lse, q, dv=k[:, :, :4].contiguous())
+
+    S, P, T = 2, 6, 5
+    qp = torch.zeros(T, Hq, d, dtype=bf)
+    kp = torch.zeros(P, Hkv, 16, d, dtype=bf)
+    bt = torch.zeros(S, 3, dtype=torch.int32)
+    sl = torch.zeros(S, dtype=torch.int32)
+    cu = torch.zeros(S + 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match=r"out must be \[T, Hq, d\]"):
+        ea.attn_prefill_paged(qp, kp, kp, bt, sl, cu, 4, out=qp[:4].contiguous())
+    with pytest.raises(ValueError, match=r"out must be \[T, Hq, d\]"):
+        ea.attn_prefill_paged(qp, kp, kp, bt, sl, cu, 4, lse=torch.zeros(T, Hq - 1))
+    with pytest.raises(ValueError, match="one value per query head"):
+        ea.attn_prefill_paged(qp, kp, kp, bt, sl, cu, 4, alibi_slopes=torch.zeros(Hq + 1))
+
+    qd = torch.zeros(S, Hq, d, dtype=bf)
+    for call in (ea.attn_decode_paged, ea.attn_decode_paged_noalloc):
+        with pytest.raises(ValueError, match=r"out must be \[S, Hq, d\]"):
+            call(qd, kp, kp, bt, sl, out=qd[:1].contiguous())
+        with pytest.raises(ValueError, match=r"out must be \[S, Hq, d\]"):
+            call(qd, kp, kp, bt, sl, lse=torch.zeros(S, Hq // 2))
+    k8 = kp.to(torch.int8)
+    sc = torch.ones(P, Hkv)
+    with pytest.raises(ValueError, match=r"out must be \[S, Hq, d\]"):
+        ea.attn_decode_paged_q8(qd, k8, k8, sc, sc, bt, sl, kv_format="int8",
+                                out=qd[:, :1].contiguous())
+    with pytest.raises(ValueError, match="scales must be"):
+        ea.attn_decode_paged_q8(qd, k8, k8, sc[:1].contiguous(), sc, bt, sl, kv_format="int8")
+
+
+def test_binding_requires_one_device_per_call():
+    # A kernel runs on q's device; a pointer into another device's memory is not
+    # valid there, so the binding refuses such a mix (meta tensors stand in for
+    # a second device here).
+    import torch
+    dev = torch.device("cuda", 0)
+    ea._same_device(dev, k=None)
+    with pytest.raises(ValueError, match="k is on meta"):
+        ea._same_device(dev, k=torch.empty(2, device="meta"))
+    with pytest.raises(ValueError, match="workspace is on cpu"):
+        ea._same_device(dev, out=None, workspace=torch.empty(2))
