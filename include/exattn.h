@@ -22,7 +22,10 @@
  *    device, and the tensors must live on it.  Only the two status reads below
  *    wait for anything: attn_decode_read_status for its own 4-byte copy,
  *    attn_device_status for the stream it is given.
- *  - Pointers must be 16-byte aligned.
+ *  - Tensor data (q, k, v, o, the page pools, dO and the gradients) and
+ *    workspaces must be 16-byte aligned; int32 and float32 vectors (lse,
+ *    block_table, seq_lens, cu_q, the 8-bit scales, ALiBi slopes) 4-byte
+ *    aligned.  A null or misaligned pointer gives ATTN_ERR_INVALID_ARG.
  *  - Errors are reported only through the return value; nothing is written when
  *    a call returns anything but ATTN_OK.  No call aborts or traps.
  *  - Device-side conditions that the host cannot see in advance (a block-table

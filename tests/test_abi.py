@@ -353,3 +353,20 @@ def test_binding_requires_one_device_per_call():
         ea._same_device(dev, k=torch.empty(2, device="meta"))
     with pytest.raises(ValueError, match="workspace is on cpu"):
         ea._same_device(dev, out=None, workspace=torch.empty(2))
+
+
+def test_alignment_rules_match_the_header(lib):
+    # Tensor data needs 16-byte alignment: an 8-byte-aligned q, k, v or o is refused.
+    for name in ("q", "k", "v", "o"):
+        assert fwd(lib, **{name: A + 8}) == INVALID, name
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="the fake addresses would reach a kernel launch on a GPU")
+def test_four_byte_vectors_pass_the_alignment_check(lib):
+    # A 4-byte-aligned lse (a float32 vector) passes validation; with no GPU in
+    # this process the call then stops at the device lookup (ATTN_ERR_CUDA),
+    # never at the argument checks.
+    CUDA = 3
+    assert fwd(lib, lse=A + 4) == CUDA
+    assert lib.attn_fwd_ext(A, A, A, A, A + 4, 1, 2, 1, 16, 128, 0.1, 1, 0, A + 4, None) == CUDA
