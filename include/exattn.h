@@ -26,8 +26,10 @@
  *    workspaces must be 16-byte aligned; int32 and float32 vectors (lse,
  *    block_table, seq_lens, cu_q, the 8-bit scales, ALiBi slopes) 4-byte
  *    aligned.  A null or misaligned pointer gives ATTN_ERR_INVALID_ARG.
- *  - Errors are reported only through the return value; nothing is written when
- *    a call returns anything but ATTN_OK.  No call aborts or traps.
+ *  - Errors are reported only through the return value.  A call that returns
+ *    ATTN_ERR_INVALID_ARG or ATTN_ERR_UNSUPPORTED has written none of its
+ *    outputs; after ATTN_ERR_CUDA (a failed launch or runtime call) the
+ *    outputs are undefined.  No call aborts or traps.
  *  - Device-side conditions that the host cannot see in advance (a block-table
  *    entry outside the page pool, a bounded wait that ran out) set ATTN_DEV_*
  *    bits in a status word.  A decode that takes a workspace (attn_decode_paged,
