@@ -338,7 +338,10 @@ EXATTN_API attn_status_t attn_decode_read_status(const void *workspace, unsigned
  * current device, which every call other than the workspace decodes reports
  * into.  Waits for the work enqueued on `stream` so far, and only for that:
  * pass the stream the calls of interest ran on (kernels still running on other
- * streams may set bits later).  Not for use inside stream capture.
+ * streams may set bits later).  The read and the clear are two steps, so a bit
+ * that a kernel on another stream sets between them is lost: clear only while
+ * no other stream runs library work on the device.  Not for use inside stream
+ * capture.
  */
 EXATTN_API attn_status_t attn_device_status(unsigned *status, int clear, attn_stream_t stream);
 
