@@ -31,10 +31,8 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import re
-import subprocess
 import sys
 import threading
 import time

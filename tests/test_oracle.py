@@ -900,7 +900,6 @@ def test_pins_catch_planted_mistakes(name, tmp_path):
     cpath.write_text(mutated)
     lib = tmp_path / "libmut.so"
     subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(lib), str(cpath), "-lm"])
-    import ctypes
     saved = oracle._lib
     try:
         oracle._lib = None
