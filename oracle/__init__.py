@@ -109,6 +109,26 @@ def _sp(a):
     return None if a is None else _ptr(a, ctypes.c_double)
 
 
+def _qkv_dims(q, k, v, *more):
+    """(B, Hq, Hkv, Nq, Nk, d) of q [B,Hq,Nq,d] and k, v [B,Hkv,Nk,d]; the C code
+    trusts these sizes, so tensors that disagree are refused here.  ``more``
+    are tensors that must have q's shape (dO)."""
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("q, k, v must be 4-D")
+    B, Hq, Nq, d = q.shape
+    if k.shape[0] != B or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, Nk, d] with q's B and d")
+    for t in more:
+        if t.shape != q.shape:
+            raise ValueError("shape mismatch")
+    return B, Hq, k.shape[1], Nq, k.shape[2], d
+
+
+def _table_dims(S, bt, sl):
+    if bt.ndim != 2 or sl.ndim != 1 or bt.shape[0] != S or sl.size != S:
+        raise ValueError("block_table must be [S, max_blocks] and seq_lens [S]")
+
+
 def attention(q, k, v, scale: float, causal: bool = False, nthreads: int | None = None,
               window: int = 0, alibi_slopes=None):
     """Standard attention in fp64.  q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (float32 values).
@@ -118,8 +138,7 @@ def attention(q, k, v, scale: float, causal: bool = False, nthreads: int | None 
     alibi_slopes (one per query head) add slope_h * (j - i) to the scores.
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
-    B, Hq, Nq, d = q.shape
-    _, Hkv, Nk, _ = k.shape
+    B, Hq, Hkv, Nq, Nk, d = _qkv_dims(q, k, v)
     o = np.zeros((B, Hq, Nq, d), dtype=np.float64)
     lse = np.zeros((B, Hq, Nq), dtype=np.float64)
     sl = _slopes(alibi_slopes, Hq)
@@ -137,8 +156,7 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, nthreads: int | No
                    window: int = 0, alibi_slopes=None):
     """The same definition for selected rows; rows[r] = (b*Hq + h)*Nq + i."""
     q, k, v = _f32(q), _f32(k), _f32(v)
-    B, Hq, Nq, d = q.shape
-    _, Hkv, Nk, _ = k.shape
+    B, Hq, Hkv, Nq, Nk, d = _qkv_dims(q, k, v)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     o = np.zeros((rows.size, d), dtype=np.float64)
     lse = np.zeros((rows.size,), dtype=np.float64)
@@ -174,6 +192,7 @@ def prefill_paged(q, k_pages_bf16_bits, v_pages_bf16_bits, block_table, seq_lens
     S = sl.size
     if d2 != d or vp.shape != kp.shape or cq.size != S + 1 or int(cq[-1]) != T:
         raise ValueError("shape mismatch")
+    _table_dims(S, bt, sl)
     o = np.zeros((T, Hq, d), dtype=np.float64)
     lse = np.zeros((T, Hq), dtype=np.float64)
     rc = _load().oracle_prefill_paged(_ptr(q, ctypes.c_float), _ptr(kp, ctypes.c_uint16),
@@ -195,9 +214,8 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool = False, window: int =
     derivatives of sum(do * O) with O = attention(q, k, v, ...).
     """
     q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
-    B, Hq, N, d = q.shape
-    _, Hkv, N2, _ = k.shape
-    if N2 != N or do.shape != q.shape or v.shape != k.shape:
+    B, Hq, Hkv, N, N2, d = _qkv_dims(q, k, v, do)
+    if N2 != N:
         raise ValueError("shape mismatch")
     dq = np.zeros((B, Hq, N, d), dtype=np.float64)
     dk = np.zeros((B, Hkv, N, d), dtype=np.float64)
@@ -218,8 +236,9 @@ def attention_bwd_dq_rows(q, k, v, do, scale: float, causal: bool, rows, window:
                           alibi_slopes=None, nthreads: int | None = None):
     """dQ of selected rows; rows[r] = (b*Hq + h)*N + i.  Returns [len(rows), d]."""
     q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
-    B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    B, Hq, Hkv, N, N2, d = _qkv_dims(q, k, v, do)
+    if N2 != N:
+        raise ValueError("shape mismatch")
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     out = np.zeros((rows.size, d), dtype=np.float64)
     sl = _slopes(alibi_slopes, Hq)
@@ -238,8 +257,9 @@ def attention_bwd_dkv_rows(q, k, v, do, scale: float, causal: bool, keys, window
                            alibi_slopes=None, nthreads: int | None = None):
     """dK and dV of selected keys; keys[r] = (b*Hkv + g)*N + j.  Returns two [len(keys), d]."""
     q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
-    B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    B, Hq, Hkv, N, N2, d = _qkv_dims(q, k, v, do)
+    if N2 != N:
+        raise ValueError("shape mismatch")
     keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
     dk = np.zeros((keys.size, d), dtype=np.float64)
     dv = np.zeros((keys.size, d), dtype=np.float64)
@@ -272,6 +292,7 @@ def decode_paged(q, k_pages_bf16_bits, v_pages_bf16_bits, block_table, seq_lens,
     num_pages, Hkv, page_size, d2 = kp.shape
     if d2 != d or vp.shape != kp.shape:
         raise ValueError("page pool shape mismatch")
+    _table_dims(S, bt, sl)
     max_blocks = bt.shape[1]
     if seq_ids is None:
         seq_ids = np.arange(S, dtype=np.int32)
@@ -322,6 +343,7 @@ def decode_paged_q8(q, k_pages_u8, v_pages_u8, k_scales, v_scales, block_table, 
     num_pages, Hkv, page_size, d2 = kp.shape
     if d2 != d or vp.shape != kp.shape or ks.shape != (num_pages, Hkv) or vs.shape != ks.shape:
         raise ValueError("page pool / scale shape mismatch")
+    _table_dims(S, bt, sl)
     max_blocks = bt.shape[1]
     if seq_ids is None:
         seq_ids = np.arange(S, dtype=np.int32)

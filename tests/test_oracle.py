@@ -927,3 +927,39 @@ def test_pins_catch_planted_mistakes(name, tmp_path):
     finally:
         oracle.build = real_build
         oracle._lib = saved
+
+
+def test_wrappers_refuse_tensors_that_disagree():
+    # The C code trusts the sizes it is given, so the wrappers compare every
+    # tensor with q's shape before calling it (a mismatch would read past an
+    # array instead of failing).
+    z = np.zeros
+    q = z((1, 2, 4, 8), np.float32)
+    with pytest.raises(ValueError):
+        oracle.attention(q, z((2, 1, 4, 8)), z((2, 1, 4, 8)), scale=1.0)   # other B
+    with pytest.raises(ValueError):
+        oracle.attention(q, z((1, 1, 4, 16)), z((1, 1, 4, 16)), scale=1.0)  # other d
+    with pytest.raises(ValueError):
+        oracle.attention(q, z((1, 1, 4, 8)), z((1, 1, 3, 8)), scale=1.0)   # v unlike k
+    with pytest.raises(ValueError):
+        oracle.attention_rows(q, z((1, 1, 4, 8)), z((1, 1, 5, 8)), 1.0, False, [0])
+    for fn, extra in ((oracle.attention_bwd, ()), (oracle.attention_bwd_dq_rows, (False, [0])),
+                      (oracle.attention_bwd_dkv_rows, (False, [0]))):
+        with pytest.raises(ValueError):
+            fn(q, z((1, 1, 4, 8)), z((1, 1, 4, 8)), z((1, 2, 3, 8)), 1.0, *extra)  # dO unlike q
+        with pytest.raises(ValueError):
+            fn(q, z((1, 1, 5, 8)), z((1, 1, 5, 8)), q, 1.0, *extra)  # keys unlike queries
+    qd = z((3, 2, 8), np.float32)
+    pages = z((4, 1, 16, 8), np.uint16)
+    bt, sl = z((3, 2), np.int32), z(3, np.int32)
+    with pytest.raises(ValueError):
+        oracle.decode_paged(qd, pages, pages, bt[:2], sl, scale=1.0)
+    with pytest.raises(ValueError):
+        oracle.decode_paged(qd, pages, pages, bt, sl[:2], scale=1.0)
+    sc = np.ones((4, 1), np.float32)
+    with pytest.raises(ValueError):
+        oracle.decode_paged_q8(qd, pages.astype(np.uint8), pages.astype(np.uint8), sc, sc,
+                               bt[:1], sl, scale=1.0)
+    with pytest.raises(ValueError):
+        oracle.prefill_paged(qd, pages, pages, bt[:2], sl, z(4, np.int32) + [0, 1, 2, 3],
+                             scale=1.0)
