@@ -370,3 +370,18 @@ def test_four_byte_vectors_pass_the_alignment_check(lib):
     CUDA = 3
     assert fwd(lib, lse=A + 4) == CUDA
     assert lib.attn_fwd_ext(A, A, A, A, A + 4, 1, 2, 1, 16, 128, 0.1, 1, 0, A + 4, None) == CUDA
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    # No fallback: without the built library every entry point raises.
+    missing = str(tmp_path / "libexattn.so")
+    with pytest.raises(ImportError, match="not built"):
+        ea.load_library(missing)
+    monkeypatch.setattr(ea, "_lib", None)
+    monkeypatch.setattr(ea, "LIB_PATH", missing)
+    with pytest.raises(ImportError):
+        ea.library()
+    with pytest.raises(ImportError):
+        ea.version()
+    with pytest.raises(ImportError):
+        ea.decode_workspace_bytes(4, 8, 128, 8)
