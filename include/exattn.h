@@ -207,7 +207,8 @@ EXATTN_API attn_status_t attn_bwd(const void *q, const void *k, const void *v, c
  * and at most max_blocks pages per sequence.  The workspace starts with a
  * 256-byte block whose first 32-bit word is the call's status word (see
  * attn_decode_read_status); the chunk partials follow.  Returns 0 for invalid
- * sizes.
+ * sizes.  The pages do not say how a decode is parallelised, so this workspace
+ * has no counterpart there: the split over key chunks is this library's choice.
  */
 EXATTN_API size_t attn_decode_workspace_bytes(int S, int Hq, int d, int max_blocks, int page_size);
 
@@ -338,17 +339,19 @@ EXATTN_API attn_status_t attn_decode_read_status(const void *workspace, unsigned
  * current device, which every call other than the workspace decodes reports
  * into.  Waits for the work enqueued on `stream` so far, and only for that:
  * pass the stream the calls of interest ran on (kernels still running on other
- * streams may set bits later).  The read and the clear are two steps, so a bit
- * that a kernel on another stream sets between them is lost: clear only while
- * no other stream runs library work on the device.  Not for use inside stream
- * capture.
+ * streams may set bits later).  Library plumbing with no counterpart on the
+ * pages; the conditions it reports are those listed with the ATTN_DEV_* bits.
+ * The read and the clear are two steps, so a bit that a kernel on another
+ * stream sets between them is lost: clear only while no other stream runs
+ * library work on the device.  Not for use inside stream capture.
  */
 EXATTN_API attn_status_t attn_device_status(unsigned *status, int clear, attn_stream_t stream);
 
-/* attn_status_string -- a static, human-readable name for a status code. */
+/* attn_status_string -- a static, human-readable name for a status code
+ * (library plumbing; no counterpart on the pages). */
 EXATTN_API const char *attn_status_string(attn_status_t status);
 
-/* attn_version -- library version string. */
+/* attn_version -- library version string (no counterpart on the pages). */
 EXATTN_API const char *attn_version(void);
 
 #ifdef __cplusplus

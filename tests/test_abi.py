@@ -385,3 +385,16 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
         ea.version()
     with pytest.raises(ImportError):
         ea.decode_workspace_bytes(4, 8, 128, 8)
+
+
+def test_every_declaration_is_documented():
+    # Each entry point in the header sits under a comment block that names it;
+    # each compute entry point's block cites the passage it follows.
+    text = open(os.path.join(ROOT, "include", "exattn.h")).read()
+    cites = re.compile(r"Phase 08|Lab 0\d|screna|Concepts|no counterpart")
+    for m in re.finditer(r"EXATTN_API[^;]*?\b(attn_[a-z0-9_]+)\s*\(", text):
+        name, before = m.group(1), text[:m.start()]
+        end = before.rfind("*/")
+        block = before[before.rfind("/*", 0, end):end]
+        assert name.replace("_workspace_bytes", "") in block or name in block, name
+        assert cites.search(block), name
